@@ -1,0 +1,681 @@
+// fl_api.cu — host side of the C ABI declared in include/fused_linear.h.
+//
+// fl_plan validates one layer ([epilog] page: Matmul(...).plan(epilog,
+// epilog_inputs)), picks the kernel configuration for its shape and owns a
+// tiny device workspace; fl_execute encodes the TMA descriptors for the
+// caller's pointers and launches the fused kernel on the caller's stream
+// ([epilog]: execute() is one kernel launch); fl_free releases the plan.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <algorithm>
+#include <mutex>
+#include <new>
+
+#include "../../include/fused_linear.h"
+#include "fl_elementwise.cuh"
+#include "fl_gemm.cuh"
+
+using namespace fl;
+
+// ------------------------------------------------------------------ errors
+static thread_local char g_err[512] = "";
+static uint64_t g_wait_limit_ns = 2000000000ull;
+
+static fl_status fail(fl_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+#define FL_CUDA(call)                                                                      \
+  do {                                                                                     \
+    cudaError_t e_ = (call);                                                               \
+    if (e_ != cudaSuccess) return fail(FL_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+extern "C" const char* fl_last_error(void) { return g_err; }
+
+extern "C" fl_status fl_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns = ns ? ns : 2000000000ull;
+  return FL_OK;
+}
+
+// ------------------------------------------------------------------ driver entry point
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+static std::once_flag g_encode_once;
+
+static fl_status get_encode() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return fail(FL_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  return FL_OK;
+}
+
+static int esize(int dt) { return dt == FL_F32 ? 4 : 2; }
+
+static CUtensorMapDataType tm_dtype(int dt) {
+  if (dt == FL_F32) return CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  if (dt == FL_BF16) return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+}
+
+// 2-D row-major map: `inner` contiguous elements per row, `outer` rows, row pitch in bytes.
+static fl_status make_map(CUtensorMap* m, const void* base, int dt, uint64_t inner, uint64_t outer,
+                          uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, tm_dtype(dt), 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(FL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d): dims %llu x %llu pitch %llu box %u x %u",
+                (int)r, (unsigned long long)inner, (unsigned long long)outer,
+                (unsigned long long)pitch_bytes, box_inner, box_outer);
+  return FL_OK;
+}
+
+// ------------------------------------------------------------------ kernel table
+using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, KParams);
+
+template <int ACT, int OUT>
+static const void* pick_swap(bool swap) {
+  return swap ? reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, OUT, true>)
+              : reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, OUT, false>);
+}
+template <int ACT>
+static const void* pick_out(int out, bool swap) {
+  if (out == FL_BF16) return pick_swap<ACT, DT_BF16>(swap);
+  if (out == FL_F16) return pick_swap<ACT, DT_F16>(swap);
+  return pick_swap<ACT, DT_F32>(swap);
+}
+static const void* pick_kernel(int act, int out, bool swap) {
+  switch (act) {
+    case ACT_NONE: return pick_out<ACT_NONE>(out, swap);
+    case ACT_RELU: return pick_out<ACT_RELU>(out, swap);
+    case ACT_GELU: return pick_out<ACT_GELU>(out, swap);
+    case ACT_GELU_TANH: return pick_out<ACT_GELU_TANH>(out, swap);
+    default: return swap ? nullptr : pick_out<ACT_GEGLU>(out, false);
+  }
+}
+
+// ------------------------------------------------------------------ plan
+struct fl_plan_s {
+  int64_t M, N, K;
+  int dtype, compute;
+  fl_epilogue_desc epi;
+  int act;
+  bool has_bias, has_aux;
+  int device, num_sms, max_smem;
+  // configuration
+  bool swap;
+  int mma_n, out_tile_n, split_k, stages, grid, smem;
+  int tiles_a, tiles_b, num_kb;
+  const void* kernel;
+  int* d_err;
+  // unfused twin
+  void* d_tmp;
+  size_t tmp_bytes;
+  int launches;
+};
+
+static int act_of(int kind) {
+  switch (kind) {
+    case FL_EPI_RELU_BIAS:
+    case FL_EPI_RELU_AUX_BIAS: return ACT_RELU;
+    case FL_EPI_GELU_BIAS: return ACT_GELU;
+    case FL_EPI_GELU_TANH_BIAS: return ACT_GELU_TANH;
+    case FL_EPI_GEGLU_TANH: return ACT_GEGLU;
+    default: return ACT_NONE;
+  }
+}
+
+static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Shared-memory budget of one configuration (bytes, before the 1 KB alignment slack).
+struct Layout {
+  uint32_t a_stage, b_box, b_stage, stage, staging_off, bar_off, red_off, red_pitch, total;
+  int stages;
+};
+
+static Layout layout_for(const fl_plan_s* p, int mma_n, int b_boxes, int max_smem) {
+  Layout L{};
+  const int es = esize(p->dtype);
+  const int bk = 128 / es;
+  L.a_stage = 128u * 128u;  // 128 rows x 128 bytes
+  if (p->epi.b_major) L.b_box = 64u * (uint32_t)bk * (uint32_t)es;  // 64 columns x bk rows
+  else L.b_box = (uint32_t)(mma_n / b_boxes) * 128u;
+  L.b_stage = L.b_box * (uint32_t)b_boxes;
+  L.stage = L.a_stage + L.b_stage;
+  const uint32_t staging = p->swap ? 0u : kStagingBytes;
+  const uint32_t red = (p->swap && p->split_k > 1) ? 128u * ((uint32_t)mma_n * 4u + 16u) : 0u;
+  const uint32_t bars = 8u * (2u * 16u + 8u) + 16u;
+  const uint32_t budget = (uint32_t)max_smem - 1024u - staging - red - bars;
+  int st = (int)(budget / L.stage);
+  if (st > 8) st = 8;
+  L.stages = st;
+  L.staging_off = (uint32_t)st * L.stage;
+  L.red_off = L.staging_off + staging;
+  L.red_pitch = (uint32_t)mma_n * 4u + 16u;
+  L.bar_off = L.red_off + red;
+  L.total = L.bar_off + 8u * (2u * (uint32_t)st + 8u) + 1024u;
+  return L;
+}
+
+static fl_status choose_config(fl_plan_s* p) {
+  const int64_t M = p->M, N = p->N;
+  const int es = esize(p->dtype);
+  const int bk = 128 / es;
+  p->num_kb = (int)cdiv(p->K, bk);
+  const bool geglu = p->epi.kind == FL_EPI_GEGLU_TANH;
+  // Small M: put the weight on the 128-row side of the tensor core (swap-AB)
+  // and split K across a cluster so that every SM streams a slice of W.
+  p->swap = (M <= 128) && !geglu && !p->epi.b_major && p->dtype != FL_F32;
+  if (p->swap) {
+    p->mma_n = (int)std::max<int64_t>(16, cdiv(M, 16) * 16);
+    p->out_tile_n = p->mma_n;
+    p->tiles_a = (int)cdiv(N, 128);
+    p->tiles_b = (int)cdiv(M, p->mma_n);
+    const int tiles = p->tiles_a * p->tiles_b;
+    int S = p->num_sms / std::max(1, tiles);
+    if (S > 8) S = 8;
+    if (S > p->num_kb) S = p->num_kb;
+    if (S < 1) S = 1;
+    p->split_k = S;
+  } else {
+    p->split_k = 1;
+    if (geglu) {
+      p->mma_n = 256;
+      p->out_tile_n = 128;
+    } else {
+      // Pick the N tile that minimises (waves x tile width) on this GPU.
+      int best = 256;
+      double best_cost = 1e300;
+      for (int bn : {256, 128}) {
+        const int64_t tiles = cdiv(M, 128) * cdiv(N, bn);
+        const double waves = (double)cdiv(tiles, p->num_sms);
+        const double cost = waves * bn * (bn == 128 ? 1.04 : 1.0);
+        if (cost < best_cost) { best_cost = cost; best = bn; }
+      }
+      p->mma_n = best;
+      p->out_tile_n = best;
+    }
+    p->tiles_a = (int)cdiv(M, 128);
+    p->tiles_b = (int)cdiv(N, p->out_tile_n);
+  }
+  return FL_OK;
+}
+
+extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, int32_t dtype,
+                             int32_t compute, const fl_epilogue_desc* epi) {
+  g_err[0] = 0;
+  if (!out || !epi) return fail(FL_ERR_INVALID_ARG, "fl_plan: null out or epilogue descriptor");
+  *out = nullptr;
+  if (M < 1 || N < 1 || K < 0) return fail(FL_ERR_INVALID_ARG, "fl_plan: need M>=1, N>=1, K>=0 (got %lld %lld %lld)",
+                                           (long long)M, (long long)N, (long long)K);
+  if (M > (1LL << 31) - 256 || N > (1LL << 30) || K > (1LL << 31) - 256)
+    return fail(FL_ERR_INVALID_ARG, "fl_plan: dimension too large");
+  if (epi->kind < FL_EPI_NONE || epi->kind > FL_EPI_GEGLU_TANH)
+    return fail(FL_ERR_INVALID_ARG, "fl_plan: unknown epilogue kind %d", epi->kind);
+  for (int i = 0; i < 3; ++i)
+    if (epi->reserved[i] != 0) return fail(FL_ERR_INVALID_ARG, "fl_plan: reserved fields must be 0");
+  if (dtype != FL_F16 && dtype != FL_BF16 && dtype != FL_F32)
+    return fail(FL_ERR_INVALID_ARG, "fl_plan: unknown dtype %d", dtype);
+  if (compute != FL_COMPUTE_32F && compute != FL_COMPUTE_32F_3XTF32)
+    return fail(FL_ERR_UNSUPPORTED, "fl_plan: compute type %d not offered (only FP32 accumulation)", compute);
+  if ((compute == FL_COMPUTE_32F) != (dtype != FL_F32))
+    return fail(FL_ERR_UNSUPPORTED, "fl_plan: FL_COMPUTE_32F takes f16/bf16 operands, 3XTF32 takes f32");
+  if (dtype == FL_F32)
+    return fail(FL_ERR_UNSUPPORTED, "fl_plan: the 3xTF32 path is not built yet");
+  if (epi->out_dtype < FL_F16 || epi->out_dtype > FL_F32)
+    return fail(FL_ERR_INVALID_ARG, "fl_plan: unknown out_dtype %d", epi->out_dtype);
+  const bool has_bias = epi->kind != FL_EPI_NONE && epi->kind != FL_EPI_GEGLU_TANH;
+  if (has_bias && (epi->bias_dtype < FL_F16 || epi->bias_dtype > FL_F32))
+    return fail(FL_ERR_INVALID_ARG, "fl_plan: unknown bias_dtype %d", epi->bias_dtype);
+  if (epi->has_residual && (epi->residual_dtype < FL_F16 || epi->residual_dtype > FL_F32))
+    return fail(FL_ERR_INVALID_ARG, "fl_plan: unknown residual_dtype %d", epi->residual_dtype);
+  if (epi->bias_axis != 0 && epi->bias_axis != 1)
+    return fail(FL_ERR_INVALID_ARG, "fl_plan: bias_axis must be 0 or 1");
+  if (epi->b_major != 0 && epi->b_major != 1) return fail(FL_ERR_INVALID_ARG, "fl_plan: b_major must be 0 or 1");
+  if (epi->kind == FL_EPI_GEGLU_TANH && epi->b_major)
+    return fail(FL_ERR_UNSUPPORTED, "fl_plan: GEGLU_TANH takes the stacked [2N,K] weight (b_major 0)");
+  if (epi->kind == FL_EPI_GEGLU_TANH && epi->out_dtype == FL_F32)
+    return fail(FL_ERR_UNSUPPORTED, "fl_plan: GEGLU_TANH writes h in f16/bf16");
+  if (epi->lda < 0 || epi->ldb < 0 || epi->ldo < 0 || epi->ldr < 0)
+    return fail(FL_ERR_INVALID_ARG, "fl_plan: negative leading dimension");
+
+  fl_plan_s* p = new (std::nothrow) fl_plan_s();
+  if (!p) return fail(FL_ERR_OOM, "fl_plan: host allocation failed");
+  p->M = M; p->N = N; p->K = K; p->dtype = dtype; p->compute = compute; p->epi = *epi;
+  if (p->epi.scale == 0.0f) p->epi.scale = 1.0f;
+  p->act = act_of(epi->kind);
+  p->has_bias = has_bias;
+  p->has_aux = epi->kind == FL_EPI_RELU_AUX_BIAS;
+  // leading dimensions default to packed
+  const int64_t a_cols = K, b_cols = epi->b_major ? N : K;
+  if (p->epi.lda == 0) p->epi.lda = a_cols;
+  if (p->epi.ldb == 0) p->epi.ldb = b_cols;
+  if (p->epi.ldo == 0) p->epi.ldo = N;
+  if (p->epi.ldr == 0) p->epi.ldr = N;
+  if (p->epi.lda < a_cols || p->epi.ldb < b_cols || p->epi.ldo < N || (epi->has_residual && p->epi.ldr < N)) {
+    delete p;
+    return fail(FL_ERR_INVALID_ARG, "fl_plan: leading dimension smaller than the row length");
+  }
+  const int es = esize(dtype), eo = esize(epi->out_dtype);
+  if ((p->epi.lda * es) % 16 || (p->epi.ldb * es) % 16 || (p->epi.ldo * eo) % 16 ||
+      (epi->has_residual && (p->epi.ldr * esize(epi->residual_dtype)) % 16)) {
+    delete p;
+    return fail(FL_ERR_ALIGNMENT, "fl_plan: every row pitch must be a multiple of 16 bytes");
+  }
+
+  if (cudaGetDevice(&p->device) != cudaSuccess) { delete p; return fail(FL_ERR_DEVICE, "fl_plan: no CUDA device"); }
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, p->device) != cudaSuccess) {
+    delete p;
+    return fail(FL_ERR_DEVICE, "fl_plan: cannot query the device");
+  }
+  if (prop.major != 10) {
+    delete p;
+    return fail(FL_ERR_DEVICE, "fl_plan: needs an sm_100 (B200-class) GPU, found sm_%d%d", prop.major, prop.minor);
+  }
+  p->num_sms = prop.multiProcessorCount;
+  p->max_smem = (int)prop.sharedMemPerBlockOptin;
+  fl_status st = get_encode();
+  if (st != FL_OK) { delete p; return st; }
+
+  choose_config(p);
+  const int b_boxes = epi->b_major ? p->mma_n / 64 : (p->epi.kind == FL_EPI_GEGLU_TANH ? 2 : 1);
+  Layout L = layout_for(p, p->mma_n, b_boxes, p->max_smem);
+  if (L.stages < 2) { delete p; return fail(FL_ERR_UNSUPPORTED, "fl_plan: shared memory too small"); }
+  p->stages = L.stages;
+  p->smem = (int)L.total;
+  const int tiles = p->tiles_a * p->tiles_b;
+  if (p->swap && p->split_k > 1) p->grid = tiles * p->split_k;
+  else p->grid = std::min(tiles, p->num_sms);
+  p->kernel = pick_kernel(p->act, epi->out_dtype, p->swap);
+  if (!p->kernel) { delete p; return fail(FL_ERR_UNSUPPORTED, "fl_plan: no kernel for this combination"); }
+  cudaError_t e = cudaFuncSetAttribute(p->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, p->smem);
+  if (e != cudaSuccess) { delete p; return fail(FL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e)); }
+  if (p->split_k > 1) {
+    e = cudaFuncSetAttribute(p->kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+    (void)e;
+  }
+  if (cudaMalloc(&p->d_err, sizeof(int)) != cudaSuccess) { delete p; return fail(FL_ERR_OOM, "fl_plan: cudaMalloc(error word)"); }
+  if (cudaMemset(p->d_err, 0, sizeof(int)) != cudaSuccess) {
+    cudaFree(p->d_err);
+    delete p;
+    return fail(FL_ERR_CUDA, "fl_plan: cudaMemset(error word)");
+  }
+  p->launches = 1;
+  if (epi->unfused) {
+    // GEMM into a plan-owned intermediate (the [M, N] or [M, 2N] result), then one
+    // elementwise kernel per epilogue step.
+    const int64_t cols = (epi->kind == FL_EPI_GEGLU_TANH) ? 2 * N : N;
+    p->tmp_bytes = (size_t)M * (size_t)cols * (size_t)eo;
+    if (cudaMalloc(&p->d_tmp, p->tmp_bytes) != cudaSuccess) {
+      cudaFree(p->d_err);
+      delete p;
+      return fail(FL_ERR_OOM, "fl_plan: cudaMalloc(unfused intermediate, %zu bytes)", p->tmp_bytes);
+    }
+  }
+  *out = p;
+  return FL_OK;
+}
+
+extern "C" fl_status fl_get_plan_info(fl_plan_t p, fl_plan_info* info) {
+  if (!p || !info) return fail(FL_ERR_INVALID_ARG, "fl_get_plan_info: null argument");
+  memset(info, 0, sizeof(*info));
+  info->tile_m = p->swap ? p->mma_n : 128;
+  info->tile_n = p->swap ? 128 : p->out_tile_n;
+  info->mma_n = p->mma_n;
+  info->swap_ab = p->swap ? 1 : 0;
+  info->split_k = p->split_k;
+  info->stages = p->stages;
+  info->grid = p->grid;
+  info->smem_bytes = p->smem;
+  info->launches_per_execute = p->launches;
+  return FL_OK;
+}
+
+extern "C" fl_status fl_free(fl_plan_t p) {
+  if (!p) return FL_OK;
+  if (p->d_err) cudaFree(p->d_err);
+  if (p->d_tmp) cudaFree(p->d_tmp);
+  delete p;
+  return FL_OK;
+}
+
+static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+// ------------------------------------------------------------------ launch helpers
+struct GemmArgs {
+  const void* A;
+  const void* W;
+  void* out;
+  int out_dtype;
+  int64_t ldo;
+  int act;
+  const void* bias;
+  const void* residual;
+  uint32_t* aux;
+  float scale;
+  int64_t n_cols;  // columns of the GEMM result written to `out` (N, or 2N for the unfused dual GEMM)
+  bool geglu_fused;
+};
+
+static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t stream, const void* kernel,
+                             bool swap, int act) {
+  const int es = esize(p->dtype);
+  const int bk = 128 / es;
+  const fl_epilogue_desc& e = p->epi;
+  KParams k{};
+  k.M = (int)p->M;
+  k.N = (int)g.n_cols;
+  k.K = (int)p->K;
+  k.num_kb = p->num_kb;
+  k.split_k = p->split_k;
+  k.mma_n = p->mma_n;
+  k.out_tile_n = p->out_tile_n;
+  k.tiles_a = p->tiles_a;
+  k.tiles_b = p->tiles_b;
+  k.bk = bk;
+  k.b_mn_major = e.b_major;
+  k.geglu = g.geglu_fused ? 1 : 0;
+  int b_boxes;
+  if (e.b_major) b_boxes = p->mma_n / 64;
+  else b_boxes = g.geglu_fused ? 2 : 1;
+  Layout L = layout_for(p, p->mma_n, b_boxes, p->max_smem);
+  k.num_stages = p->stages;
+  k.b_boxes = b_boxes;
+  k.b_box_rows = e.b_major ? 64 : p->mma_n / b_boxes;
+  k.a_stage_bytes = L.a_stage;
+  k.b_box_bytes = L.b_box;
+  k.stage_bytes = L.stage;
+  k.staging_off = L.staging_off;
+  k.red_off = L.red_off;
+  k.red_pitch = L.red_pitch;
+  k.bar_off = L.bar_off;
+  const uint32_t fmt = (p->dtype == FL_BF16) ? 1u : 0u;
+  k.idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(e.b_major ? 1 : 0) << 16) |
+            ((uint32_t)(p->mma_n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+  k.ksteps = bk / 16;               // UMMA K = 16 elements (32 bytes) for f16/bf16
+  k.a_kstep = 32;
+  k.b_kstep = e.b_major ? 16u * 128u : 32u;
+  k.b_lbo = e.b_major ? L.b_box : 16u;
+  int tc = 2 * p->mma_n;
+  uint32_t cols = 32;
+  while ((int)cols < tc) cols <<= 1;
+  k.tmem_cols = cols;
+  k.bias = g.bias;
+  k.bias_dtype = e.bias_dtype;
+  k.bias_axis = e.bias_axis;
+  k.residual = g.residual;
+  k.ldr = e.ldr;
+  k.res_dtype = e.residual_dtype;
+  k.out = g.out;
+  k.ldo = g.ldo;
+  k.aux = g.aux;
+  k.ld_aux = cdiv(p->M > 0 ? g.n_cols : 0, 32);
+  k.scale = g.scale;
+  k.err = p->d_err;
+  k.wait_limit_ns = g_wait_limit_ns;
+
+  CUtensorMap tmA, tmB, tmB2, tmOut;
+  memset(&tmB2, 0, sizeof(tmB2));
+  memset(&tmOut, 0, sizeof(tmOut));
+  fl_status st;
+  const uint64_t Kd = (uint64_t)std::max<int64_t>(p->K, 1);
+  const bool no_k = p->K == 0;  // no operand is read: y = epi(0 + bias)
+  memset(&tmA, 0, sizeof(tmA));
+  memset(&tmB, 0, sizeof(tmB));
+  if (!swap) {
+    if (!no_k) st = make_map(&tmA, g.A, p->dtype, Kd, (uint64_t)p->M, (uint64_t)e.lda * es, (uint32_t)bk, 128);
+    else st = FL_OK;
+    if (st) return st;
+    if (no_k) {
+      st = FL_OK;
+    } else if (e.b_major) {
+      st = make_map(&tmB, g.W, p->dtype, (uint64_t)g.n_cols, Kd, (uint64_t)e.ldb * es, 64, (uint32_t)bk);
+    } else if (g.geglu_fused) {
+      st = make_map(&tmB, g.W, p->dtype, Kd, (uint64_t)p->N, (uint64_t)e.ldb * es, (uint32_t)bk, 128);
+      if (st) return st;
+      const char* up = static_cast<const char*>(g.W) + (size_t)p->N * (size_t)e.ldb * es;
+      st = make_map(&tmB2, up, p->dtype, Kd, (uint64_t)p->N, (uint64_t)e.ldb * es, (uint32_t)bk, 128);
+    } else {
+      st = make_map(&tmB, g.W, p->dtype, Kd, (uint64_t)g.n_cols, (uint64_t)e.ldb * es, (uint32_t)bk,
+                    (uint32_t)p->mma_n);
+    }
+    if (st) return st;
+    const int eo = esize(g.out_dtype);
+    st = make_map(&tmOut, g.out, g.out_dtype, (uint64_t)g.n_cols, (uint64_t)p->M, (uint64_t)g.ldo * eo,
+                  (uint32_t)(128 / eo), 32);
+    if (st) return st;
+  } else if (!no_k) {
+    // UMMA A = weight rows (output features), UMMA B = activation rows
+    st = make_map(&tmA, g.W, p->dtype, Kd, (uint64_t)g.n_cols, (uint64_t)e.ldb * es, (uint32_t)bk, 128);
+    if (st) return st;
+    st = make_map(&tmB, g.A, p->dtype, Kd, (uint64_t)p->M, (uint64_t)e.lda * es, (uint32_t)bk,
+                  (uint32_t)p->mma_n);
+    if (st) return st;
+    tmOut = tmA;  // unused in the swap layout
+  } else {
+    tmOut = tmA;  // unused in the swap layout
+  }
+  if (!g.geglu_fused) tmB2 = tmB;  // unused
+
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)p->grid, 1, 1);
+  cfg.blockDim = dim3(kNumThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)p->smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  if (p->split_k > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)p->split_k;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  (void)act;
+  cudaError_t err = cudaLaunchKernelEx(&cfg, reinterpret_cast<KernelFn>(const_cast<void*>(kernel)), tmA, tmB,
+                                       tmB2, tmOut, k);
+  if (err != cudaSuccess) return fail(FL_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(err));
+  return FL_OK;
+}
+
+static int grid_for(long long work, int num_sms) {
+  long long b = (work + 255) / 256;
+  long long cap = (long long)num_sms * 8;
+  if (b > cap) b = cap;
+  if (b < 1) b = 1;
+  return (int)b;
+}
+
+template <int DT>
+static fl_status launch_ew_t(const EwParams& P, int num_sms, cudaStream_t s) {
+  const long long work = P.M * ((P.N + 31) / 32);
+  fl_ew_step_kernel<DT><<<grid_for(work, num_sms), 256, 0, s>>>(P);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FL_ERR_CUDA, "elementwise launch: %s", cudaGetErrorString(e));
+  return FL_OK;
+}
+static fl_status launch_ew(int dt, const EwParams& P, int num_sms, cudaStream_t s) {
+  if (dt == FL_BF16) return launch_ew_t<DT_BF16>(P, num_sms, s);
+  if (dt == FL_F16) return launch_ew_t<DT_F16>(P, num_sms, s);
+  return launch_ew_t<DT_F32>(P, num_sms, s);
+}
+
+// ------------------------------------------------------------------ execute
+extern "C" fl_status fl_execute(fl_plan_t p, const void* A, const void* W, const void* bias, uint32_t* aux,
+                                const void* residual, void* out, void* stream_) {
+  g_err[0] = 0;
+  if (!p) return fail(FL_ERR_INVALID_ARG, "fl_execute: null plan");
+  if (!out || (p->K > 0 && (!A || !W)))
+    return fail(FL_ERR_INVALID_ARG, "fl_execute: A, W (when K > 0) and out are required");
+  if (p->has_bias && !bias) return fail(FL_ERR_INVALID_ARG, "fl_execute: this epilogue needs a bias");
+  if (!p->has_bias && bias) return fail(FL_ERR_INVALID_ARG, "fl_execute: this epilogue takes no bias");
+  if (p->has_aux && !aux) return fail(FL_ERR_INVALID_ARG, "fl_execute: RELU_AUX_BIAS needs the aux mask buffer");
+  if (!p->has_aux && aux) return fail(FL_ERR_INVALID_ARG, "fl_execute: only RELU_AUX_BIAS writes an aux mask");
+  if (p->epi.has_residual && !residual) return fail(FL_ERR_INVALID_ARG, "fl_execute: has_residual needs a residual");
+  if (!p->epi.has_residual && residual) return fail(FL_ERR_INVALID_ARG, "fl_execute: residual given but not planned");
+  if ((p->K > 0 && (!aligned16(A) || !aligned16(W))) || !aligned16(out) || (residual && !aligned16(residual)))
+    return fail(FL_ERR_ALIGNMENT, "fl_execute: A, W, out and residual must be 16-byte aligned");
+  if (bias && (reinterpret_cast<uintptr_t>(bias) % (uintptr_t)esize(p->epi.bias_dtype)))
+    return fail(FL_ERR_ALIGNMENT, "fl_execute: bias is not aligned to its element size");
+  if (aux && (reinterpret_cast<uintptr_t>(aux) & 3u)) return fail(FL_ERR_ALIGNMENT, "fl_execute: aux must be 4-byte aligned");
+  int dev = -1;
+  FL_CUDA(cudaGetDevice(&dev));
+  if (dev != p->device) return fail(FL_ERR_INVALID_ARG, "fl_execute: plan was made on device %d, current is %d", p->device, dev);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const fl_epilogue_desc& e = p->epi;
+  const bool geglu = e.kind == FL_EPI_GEGLU_TANH;
+
+  if (!e.unfused) {
+    GemmArgs g{A, W, out, e.out_dtype, e.ldo, p->act, bias, residual, aux, e.scale, p->N, geglu};
+    return launch_gemm(p, g, stream, p->kernel, p->swap, p->act);
+  }
+
+  // ---- unfused twin: bare GEMM into the intermediate, then one kernel per step
+  const int odt = e.out_dtype;
+  const int64_t cols = geglu ? 2 * p->N : p->N;
+  const bool no_steps = (e.kind == FL_EPI_NONE) && !e.has_residual && e.scale == 1.0f;
+  void* gemm_out = no_steps ? out : p->d_tmp;
+  const int64_t gemm_ld = no_steps ? e.ldo : cols;
+  {
+    // The unfused GEMM uses the same tcgen05 kernel with no epilogue work.
+    fl_plan_s q = *p;
+    q.epi.kind = FL_EPI_NONE;
+    q.N = cols;
+    choose_config(&q);
+    const int b_boxes = e.b_major ? q.mma_n / 64 : 1;
+    Layout L = layout_for(&q, q.mma_n, b_boxes, q.max_smem);
+    q.stages = L.stages;
+    q.smem = (int)L.total;
+    const int tiles = q.tiles_a * q.tiles_b;
+    q.grid = (q.swap && q.split_k > 1) ? tiles * q.split_k : std::min(tiles, q.num_sms);
+    const void* kern = pick_kernel(ACT_NONE, odt, q.swap);
+    FL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, q.smem));
+    q.epi.ldr = 0;
+    q.epi.has_residual = 0;
+    GemmArgs g{A, W, gemm_out, odt, gemm_ld, ACT_NONE, nullptr, nullptr, nullptr, 1.0f, cols, false};
+    fl_status st = launch_gemm(&q, g, stream, kern, q.swap, ACT_NONE);
+    if (st) return st;
+  }
+  if (no_steps) return FL_OK;
+  EwParams P{};
+  P.M = p->M;
+  P.N = p->N;
+  P.src = p->d_tmp;
+  P.lds = cols;
+  P.dst = out;
+  P.ldd = e.ldo;
+  auto step = [&](int op, const void* operand, int odtype, int64_t ldop) -> fl_status {
+    P.op = op;
+    P.operand = operand;
+    P.operand_dtype = odtype;
+    P.ldop = ldop;
+    fl_status st = launch_ew(odt, P, p->num_sms, stream);
+    P.src = out;  // every later step works in place on `out`
+    P.lds = e.ldo;
+    return st;
+  };
+  fl_status st = FL_OK;
+  if (geglu) {
+    // h = gelu_tanh(g) * u, with g = tmp[:, :N] and u = tmp[:, N:]
+    P.op = EW_GEGLU_MUL;
+    st = step(EW_GEGLU_MUL, static_cast<const char*>(p->d_tmp) + (size_t)p->N * esize(odt), odt, cols);
+    if (st) return st;
+  } else {
+    if (p->has_bias) {
+      st = step(e.bias_axis == 0 ? EW_BIAS_N : EW_BIAS_M, bias, e.bias_dtype, 0);
+      if (st) return st;
+    }
+    if (p->act == ACT_RELU) {
+      P.aux = aux;
+      P.ld_aux = cdiv(p->N, 32);
+      st = step(EW_RELU, nullptr, 0, 0);
+      P.aux = nullptr;
+    } else if (p->act == ACT_GELU) {
+      st = step(EW_GELU, nullptr, 0, 0);
+    } else if (p->act == ACT_GELU_TANH) {
+      st = step(EW_GELU_TANH, nullptr, 0, 0);
+    }
+    if (st) return st;
+  }
+  if (e.has_residual) {
+    st = step(EW_RESIDUAL, residual, e.residual_dtype, e.ldr);
+    if (st) return st;
+  }
+  if (e.scale != 1.0f) {
+    P.scale = e.scale;
+    st = step(EW_SCALE, nullptr, 0, 0);
+    if (st) return st;
+  }
+  if (P.src == p->d_tmp) {  // no step ran (e.g. NONE with nothing else): copy through
+    FL_CUDA(cudaMemcpy2DAsync(out, (size_t)e.ldo * esize(odt), p->d_tmp, (size_t)cols * esize(odt),
+                              (size_t)p->N * esize(odt), (size_t)p->M, cudaMemcpyDeviceToDevice, stream));
+  }
+  return FL_OK;
+}
+
+// ------------------------------------------------------------------ dReLU
+extern "C" fl_status fl_relu_backward(const void* grad, const uint32_t* aux, void* dpre, int64_t M, int64_t N,
+                                      int64_t ld_grad, int64_t ld_dpre, int32_t dtype, void* stream_) {
+  g_err[0] = 0;
+  if (!grad || !aux || !dpre) return fail(FL_ERR_INVALID_ARG, "fl_relu_backward: null pointer");
+  if (M < 0 || N < 0) return fail(FL_ERR_INVALID_ARG, "fl_relu_backward: negative size");
+  if (dtype != FL_F16 && dtype != FL_BF16 && dtype != FL_F32)
+    return fail(FL_ERR_INVALID_ARG, "fl_relu_backward: unknown dtype %d", dtype);
+  if (ld_grad == 0) ld_grad = N;
+  if (ld_dpre == 0) ld_dpre = N;
+  if (ld_grad < N || ld_dpre < N) return fail(FL_ERR_INVALID_ARG, "fl_relu_backward: leading dimension < N");
+  const int es = esize(dtype);
+  if (reinterpret_cast<uintptr_t>(grad) % es || reinterpret_cast<uintptr_t>(dpre) % es ||
+      reinterpret_cast<uintptr_t>(aux) % 4)
+    return fail(FL_ERR_ALIGNMENT, "fl_relu_backward: misaligned pointer");
+  if (M == 0 || N == 0) return FL_OK;
+  const int vec_ok = aligned16(grad) && aligned16(dpre) && (ld_grad * es) % 16 == 0 && (ld_dpre * es) % 16 == 0;
+  int dev = 0, sms = 148;
+  FL_CUDA(cudaGetDevice(&dev));
+  FL_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const long long words = cdiv(N, 32);
+  const long long work = M * words;
+  const int grid = grid_for(work, sms);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+  if (dtype == FL_BF16)
+    fl_relu_backward_kernel<DT_BF16><<<grid, 256, 0, s>>>(grad, aux, dpre, M, N, ld_grad, ld_dpre, words, vec_ok);
+  else if (dtype == FL_F16)
+    fl_relu_backward_kernel<DT_F16><<<grid, 256, 0, s>>>(grad, aux, dpre, M, N, ld_grad, ld_dpre, words, vec_ok);
+  else
+    fl_relu_backward_kernel<DT_F32><<<grid, 256, 0, s>>>(grad, aux, dpre, M, N, ld_grad, ld_dpre, words, vec_ok);
+  FL_CUDA(cudaGetLastError());
+  return FL_OK;
+}
+
+// ------------------------------------------------------------------ status
+extern "C" fl_status fl_check_status(fl_plan_t p, void* stream_) {
+  if (!p) return fail(FL_ERR_INVALID_ARG, "fl_check_status: null plan");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+  FL_CUDA(cudaStreamSynchronize(s));
+  int h = 0;
+  FL_CUDA(cudaMemcpy(&h, p->d_err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (h != 0) {
+    FL_CUDA(cudaMemset(p->d_err, 0, sizeof(int)));
+    return fail(FL_ERR_TIMEOUT, "a bounded in-kernel wait gave up (code %d)", h);
+  }
+  return FL_OK;
+}

@@ -1,0 +1,551 @@
+// fl_gemm.cuh — the fused linear layer as one persistent, warp-specialised
+// tcgen05 kernel for sm_100a:
+//
+//     y = ((act(A·Wᵀ + bias)) + residual) · scale       [+ ReLU aux bitmask]
+//
+// The epilogue runs on the fp32 accumulator tile while it sits in tensor
+// memory, so the GEMM result never makes an HBM round trip — the single
+// launch / single write that the cuBLASLt epilog page ("通过 cuBLASLt 的
+// epilog 机制实现单内核偏置融合") describes for RELU_BIAS / GELU_BIAS /
+// RELU_AUX_BIAS, and the GEMM-epilogue fusion of the mHC page
+// (mhpn.cn/news/2504128, §3.3).
+//
+// Roles (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A and B tiles into a multi-stage 128B-swizzled ring
+//   warp 1      TMEM allocator + single-thread UMMA issuer (double-buffered accumulators)
+//   warps 2..5  epilogue: tcgen05.ld → bias/act/aux/residual/scale in registers →
+//               swizzled smem → TMA store (normal layout) or coalesced stores (swap-AB)
+//
+// Layouts:
+//   * normal:  UMMA A = activation rows (128 per tile), UMMA B = weight rows;
+//              TMEM lane = output row m, TMEM column = output column n.
+//   * swap-AB (small M): UMMA A = weight rows (128 output features), UMMA B =
+//              activation rows; TMEM lane = output column n, column = output row m.
+//              Optional split-K across a thread-block cluster, reduced through
+//              distributed shared memory BEFORE the (nonlinear) epilogue.
+//
+// Every wait is bounded (globaltimer); on expiry the kernel records an error
+// code in a device word and unwinds: no trap, no unbounded spin.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "fl_ptx.cuh"
+
+namespace fl {
+
+enum Act : int { ACT_NONE = 0, ACT_RELU = 1, ACT_GELU = 2, ACT_GELU_TANH = 3, ACT_GEGLU = 4 };
+enum DType : int { DT_F16 = 0, DT_BF16 = 1, DT_F32 = 2 };
+
+constexpr int kNumThreads = 192;
+constexpr int kEpiWarp0 = 2;
+constexpr int kNumEpiWarps = 4;
+constexpr uint32_t kStagingBuf = 32 * 128;  // one warp's 32 rows x 128 bytes
+constexpr uint32_t kStagingBytes = kNumEpiWarps * 2 * kStagingBuf;
+constexpr int kErrTimeout = 1;
+
+struct KParams {
+  // output space: y is M x N
+  int M, N, K;
+  // MMA space
+  int tiles_a, tiles_b;  // tiles along UMMA M (128 rows of operand A) / along UMMA N
+  int num_kb;            // BK blocks along K
+  int split_k;           // CTAs of a cluster sharing one tile along K (swap-AB only)
+  int num_stages;
+  int mma_n;             // UMMA N = TMEM columns per accumulator buffer
+  int out_tile_n;        // output columns per tile in the normal layout (mma_n/2 for GeGLU)
+  int bk;                // K elements per stage (128 bytes of operand)
+  int b_boxes;           // TMA boxes of operand B per stage
+  int b_box_rows;        // rows (K-major) or N-columns (MN-major) per B box
+  int b_mn_major;        // 1: B stored [K, N]
+  int geglu;             // 1: B = [gate rows ; up rows] from two tensor maps
+  uint32_t a_stage_bytes, b_box_bytes, stage_bytes;
+  uint32_t idesc;
+  uint32_t a_kstep, b_kstep;  // descriptor start-address advance per UMMA K step (bytes)
+  uint32_t b_lbo;             // leading byte offset of an MN-major B operand
+  int ksteps;                 // UMMA instructions per stage
+  uint32_t tmem_cols;
+  uint32_t staging_off, bar_off, red_off, red_pitch;
+  // epilogue operands
+  const void* bias;
+  int bias_dtype, bias_axis;
+  const void* residual;
+  long long ldr;
+  int res_dtype;
+  void* out;
+  long long ldo;
+  uint32_t* aux;
+  long long ld_aux;
+  float scale;
+  int* err;
+  unsigned long long wait_limit_ns;
+};
+
+// ------------------------------------------------------------------ helpers
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const KParams& p,
+                                             bool cluster_scope = false) {
+  if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t spins = 0;
+  while (true) {
+    if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if ((++spins & 63u) == 0 && globaltimer_ns() - t0 > p.wait_limit_ns) {
+      atomicCAS(p.err, 0, kErrTimeout);
+      return false;
+    }
+  }
+}
+
+// Warp-uniform bounded wait: lane 0 spins, the verdict is broadcast.
+__device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity, const KParams& p,
+                                                  int lane, bool cluster_scope = false) {
+  uint32_t ok = 0;
+  if (lane == 0) ok = wait_bounded(bar, parity, p, cluster_scope) ? 1u : 0u;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) {
+    // The phase has completed and cannot complete again before this warp
+    // arrives elsewhere, so each lane's own test succeeds at once and gives
+    // every lane the barrier's acquire ordering.
+    if (cluster_scope) (void)mbar_try_wait_cluster(bar, parity);
+    else (void)mbar_try_wait(bar, parity);
+  }
+  return ok != 0;
+}
+
+__device__ __forceinline__ float load_elem(const void* p, long long i, int dt) {
+  if (dt == DT_BF16) return __bfloat162float(__ldg(reinterpret_cast<const __nv_bfloat16*>(p) + i));
+  if (dt == DT_F16) return __half2float(__ldg(reinterpret_cast<const __half*>(p) + i));
+  return __ldg(reinterpret_cast<const float*>(p) + i);
+}
+
+template <int OUT>
+__device__ __forceinline__ void store_elem(void* p, long long i, float v) {
+  if constexpr (OUT == DT_BF16) {
+    reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+  } else if constexpr (OUT == DT_F16) {
+    reinterpret_cast<__half*>(p)[i] = __float2half_rn(v);
+  } else {
+    reinterpret_cast<float*>(p)[i] = v;
+  }
+}
+
+__device__ __forceinline__ float gelu_erf_f(float x) {
+  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+}
+__device__ __forceinline__ float gelu_tanh_f(float x) {
+  const float u = 0.79788456080286536f * (x + 0.044715f * x * x * x);
+  return 0.5f * x * (1.0f + tanhf(u));
+}
+
+template <int ACT>
+__device__ __forceinline__ float activate(float v, float u) {
+  if constexpr (ACT == ACT_RELU) return fmaxf(v, 0.0f);
+  if constexpr (ACT == ACT_GELU) return gelu_erf_f(v);
+  if constexpr (ACT == ACT_GELU_TANH) return gelu_tanh_f(v);
+  if constexpr (ACT == ACT_GEGLU) return gelu_tanh_f(v) * u;
+  return v;
+}
+
+// Pack 32 fp32 values into 32 little-endian 32-bit words of OUT type
+// (16-bit: two values per word → 64 values give 32 words; fp32: one per word).
+template <int OUT>
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  if constexpr (OUT == DT_BF16) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  } else {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+__device__ __forceinline__ void tile_coords(int t, const KParams& p, int& ta, int& tb) {
+  // Grouped raster: 8 A-side tiles per group, B-side swept inside the group,
+  // so concurrently resident CTAs share operand panels in L2.
+  constexpr int G = 8;
+  const int group_size = G * p.tiles_b;
+  const int g = t / group_size;
+  const int first = g * G;
+  const int ga = min(G, p.tiles_a - first);
+  const int r = t - g * group_size;
+  ta = first + r % ga;
+  tb = r / ga;
+}
+
+// ------------------------------------------------------------------ kernel
+template <int ACT, int OUT, bool SWAP>
+__global__ void __launch_bounds__(kNumThreads, 1)
+    fl_gemm_epi_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmOut,
+                        const __grid_constant__ KParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int NS = p.num_stages;
+
+  const uint32_t bars = smem_base + p.bar_off;
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  auto empty_bar = [&](int s) { return bars + 8u * (NS + s); };
+  auto tfull_bar = [&](int b) { return bars + 8u * (2 * NS + b); };
+  auto tempty_bar = [&](int b) { return bars + 8u * (2 * NS + 2 + b); };
+  const uint32_t drain_bar = bars + 8u * (2 * NS + 4);
+  const uint32_t red_ready_bar = bars + 8u * (2 * NS + 5);
+  const uint32_t red_done_bar = bars + 8u * (2 * NS + 6);
+  const uint32_t tmem_slot = bars + 8u * (2 * NS + 7);
+
+  const int S = p.split_k;
+  const uint32_t rank = (S > 1) ? cluster_ctarank() : 0u;
+  const int cluster_id = blockIdx.x / S;
+  const int num_clusters = gridDim.x / S;
+  const int total_tiles = p.tiles_a * p.tiles_b;
+  const int kb_begin = (int)(((long long)p.num_kb * rank) / S);
+  const int kb_end = (int)(((long long)p.num_kb * (rank + 1)) / S);
+  const bool have_acc = kb_end > kb_begin;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), kNumEpiWarps);
+    }
+    mbar_init(drain_bar, 1);
+    mbar_init(red_ready_bar, kNumEpiWarps * 32 * (S > 1 ? S - 1 : 1));
+    mbar_init(red_done_bar, kNumEpiWarps * 32);
+    fence_mbarrier_init();
+    if (p.num_kb > 0) {  // with K = 0 the operand maps are left unencoded and never used
+      prefetch_tensormap(&tmA);
+      prefetch_tensormap(&tmB);
+      if (p.geglu) prefetch_tensormap(&tmB2);
+    }
+    if (!SWAP) prefetch_tensormap(&tmOut);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (S > 1) cluster_sync_all();  // peers' barriers are initialised before any remote arrive
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(
+      __cvta_shared_to_generic(tmem_slot));
+
+  if (warp == 0) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = cluster_id; ok && t < total_tiles; t += num_clusters) {
+        int ta, tb;
+        tile_coords(t, p, ta, tb);
+        for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+          const int s = (int)(it % (uint32_t)NS);
+          const uint32_t ph = (it / (uint32_t)NS) & 1u;
+          if (!wait_bounded(empty_bar(s), ph ^ 1u, p)) { ok = false; break; }
+          mbar_arrive_expect_tx(full_bar(s), p.stage_bytes);
+          const uint32_t sa = smem_base + (uint32_t)s * p.stage_bytes;
+          const uint32_t sb = sa + p.a_stage_bytes;
+          const int k0 = kb * p.bk;
+          tma_load_2d(sa, &tmA, full_bar(s), k0, ta * 128);
+          if (p.b_mn_major) {
+            for (int i = 0; i < p.b_boxes; ++i)
+              tma_load_2d(sb + i * p.b_box_bytes, &tmB, full_bar(s), tb * p.mma_n + i * 64, k0);
+          } else if (p.geglu) {
+            tma_load_2d(sb, &tmB, full_bar(s), k0, tb * p.b_box_rows);
+            tma_load_2d(sb + p.b_box_bytes, &tmB2, full_bar(s), k0, tb * p.b_box_rows);
+          } else {
+            for (int i = 0; i < p.b_boxes; ++i)
+              tma_load_2d(sb + i * p.b_box_bytes, &tmB, full_bar(s), k0,
+                          tb * p.mma_n + i * p.b_box_rows);
+          }
+        }
+      }
+      // Never leave the CTA with copies in flight: wait (bounded) for the last
+      // fill of every stage (fill i went to stage i % NS with phase (i / NS) & 1).
+      // In the normal path these have all completed already.
+      for (uint32_t s = 0; s < (uint32_t)NS && s < it; ++s) {
+        const uint32_t last = it - 1u - ((it - 1u - s) % (uint32_t)NS);
+        (void)wait_bounded(full_bar((int)s), (last / (uint32_t)NS) & 1u, p);
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ UMMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, local = 0;
+      bool ok = true, issued = false;
+      for (int t = cluster_id; ok && t < total_tiles; t += num_clusters, ++local) {
+        const uint32_t buf = local & 1u;
+        const uint32_t tph = (local >> 1) & 1u;
+        if (!wait_bounded(tempty_bar(buf), tph ^ 1u, p)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * (uint32_t)p.mma_n;
+        for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+          const int s = (int)(it % (uint32_t)NS);
+          const uint32_t ph = (it / (uint32_t)NS) & 1u;
+          if (!wait_bounded(full_bar(s), ph, p)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_base + (uint32_t)s * p.stage_bytes;
+          const uint32_t sb = sa + p.a_stage_bytes;
+          for (int k = 0; k < p.ksteps; ++k) {
+            const uint64_t adesc = sdesc_sw128(sa + k * p.a_kstep, 16, 1024);
+            const uint64_t bdesc = p.b_mn_major ? sdesc_sw128(sb + k * p.b_kstep, p.b_lbo, 1024)
+                                                : sdesc_sw128(sb + k * p.b_kstep, 16, 1024);
+            umma_f16(d_tmem, adesc, bdesc, p.idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
+          }
+          umma_commit(empty_bar(s));  // frees the stage once these MMAs have read it
+          issued = true;
+        }
+        if (!ok) break;
+        if (have_acc) umma_commit(tfull_bar(buf));
+        else mbar_arrive(tfull_bar(buf));
+      }
+      if (issued) {  // no MMA may still be running when TMEM is released
+        umma_commit(drain_bar);
+        (void)wait_bounded(drain_bar, 0, p);
+      }
+    }
+  } else {
+    // ================================================================ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int ew = warp - kEpiWarp0;
+    const float scale = p.scale;
+    const bool has_bias = p.bias != nullptr;
+    const bool has_res = p.residual != nullptr;
+    const bool has_aux = p.aux != nullptr;
+    uint32_t local = 0;
+    bool ok = true;
+
+    if constexpr (!SWAP) {
+      // ---------------- normal layout: thread = output row, columns in registers
+      constexpr int CH = (OUT == DT_F32) ? 32 : 64;  // output columns per 128-byte staging row
+      const uint32_t stg0 = smem_base + p.staging_off + (uint32_t)ew * 2u * kStagingBuf;
+      int stg_idx = 0;
+      for (int t = cluster_id; t < total_tiles; t += num_clusters, ++local) {
+        int ta, tb;
+        tile_coords(t, p, ta, tb);
+        const uint32_t buf = local & 1u;
+        const uint32_t tph = (local >> 1) & 1u;
+        if (!warp_wait_bounded(tfull_bar(buf), tph, p, lane)) { ok = false; break; }
+        tc_fence_after();
+        const int row0 = ta * 128 + q * 32;
+        const int m = row0 + lane;
+        const bool m_ok = m < p.M;
+        const int n_tile0 = tb * p.out_tile_n;
+        const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
+        float bias_m = 0.0f;
+        if (has_bias && p.bias_axis == 1 && m_ok) bias_m = load_elem(p.bias, m, p.bias_dtype);
+
+        for (int cc = 0; cc < p.out_tile_n; cc += CH) {
+          float v[CH];
+          float u[(ACT == ACT_GEGLU) ? CH : 1];
+          if (have_acc) {
+#pragma unroll
+            for (int h = 0; h < CH / 32; ++h) {
+              uint32_t r[32];
+              tmem_ld32(tacc + (uint32_t)(cc + h * 32), r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[h * 32 + j] = __uint_as_float(r[j]);
+              if constexpr (ACT == ACT_GEGLU) {
+                tmem_ld32(tacc + (uint32_t)(p.out_tile_n + cc + h * 32), r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) u[h * 32 + j] = __uint_as_float(r[j]);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < CH; ++j) v[j] = 0.0f;
+            if constexpr (ACT == ACT_GEGLU) {
+#pragma unroll
+              for (int j = 0; j < CH; ++j) u[j] = 0.0f;
+            }
+          }
+          if (cc + CH >= p.out_tile_n) {
+            // all TMEM reads of this tile are done: hand the buffer back to the MMA warp
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(buf));
+          }
+          const int nc0 = n_tile0 + cc;
+          // ---- bias, activation, aux, residual, scale (all in fp32 registers)
+          uint32_t aux_word[CH / 32];
+#pragma unroll
+          for (int h = 0; h < CH / 32; ++h) aux_word[h] = 0u;
+          const bool full_cols = nc0 + CH <= p.N;
+#pragma unroll
+          for (int j = 0; j < CH; ++j) {
+            const int n = nc0 + j;
+            float x = v[j];
+            if (has_bias) {
+              if (p.bias_axis == 0) x += (n < p.N) ? load_elem(p.bias, n, p.bias_dtype) : 0.0f;
+              else x += bias_m;
+            }
+            if (has_aux && x > 0.0f && (full_cols || n < p.N)) aux_word[j >> 5] |= 1u << (j & 31);
+            float y;
+            if constexpr (ACT == ACT_GEGLU) y = activate<ACT>(x, u[j]);
+            else y = activate<ACT>(x, 0.0f);
+            v[j] = y;
+          }
+          if (has_res && m_ok) {
+#pragma unroll
+            for (int j = 0; j < CH; ++j) {
+              const int n = nc0 + j;
+              if (full_cols || n < p.N) v[j] += load_elem(p.residual, (long long)m * p.ldr + n, p.res_dtype);
+            }
+          }
+          if (scale != 1.0f) {
+#pragma unroll
+            for (int j = 0; j < CH; ++j) v[j] *= scale;
+          }
+          if (has_aux && m_ok) {
+#pragma unroll
+            for (int h = 0; h < CH / 32; ++h) {
+              const int w = (nc0 >> 5) + h;
+              if ((long long)w * 32 < p.N) p.aux[(long long)m * p.ld_aux + w] = aux_word[h];
+            }
+          }
+          // ---- stage the 32 x 128-byte block in 128B-swizzled smem, TMA-store it
+          uint32_t words[32];
+          if constexpr (OUT == DT_F32) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) words[j] = __float_as_uint(v[j]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) words[j] = pack2<OUT>(v[2 * j], v[2 * j + 1]);
+          }
+          if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read smem
+          __syncwarp();
+          const uint32_t sbuf = stg0 + (uint32_t)stg_idx * kStagingBuf;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t addr = sbuf + (uint32_t)lane * 128u + ((uint32_t)(c ^ (lane & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(words[4 * c]),
+                         "r"(words[4 * c + 1]), "r"(words[4 * c + 2]), "r"(words[4 * c + 3])
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmOut, sbuf, nc0, row0);
+            bulk_commit_group();
+          }
+          stg_idx ^= 1;
+        }
+      }
+      if (lane == 0) bulk_wait_group<0>();
+    } else {
+      // ---------------- swap-AB layout: thread = output column n, columns = output rows m
+      const uint32_t red_base = smem_base + p.red_off;
+      for (int t = cluster_id; t < total_tiles; t += num_clusters, ++local) {
+        int ta, tb;
+        tile_coords(t, p, ta, tb);
+        const uint32_t buf = local & 1u;
+        const uint32_t tph = (local >> 1) & 1u;
+        if (!warp_wait_bounded(tfull_bar(buf), tph, p, lane)) { ok = false; break; }
+        tc_fence_after();
+        const int r_lane = q * 32 + lane;            // TMEM lane = row of the W tile
+        const int n = ta * 128 + r_lane;             // output column
+        const bool n_ok = n < p.N;
+        const int m_tile0 = tb * p.mma_n;
+        const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
+        const uint32_t my_row = red_base + (uint32_t)r_lane * p.red_pitch;
+
+        if (S > 1 && rank != 0) {
+          // ---- non-leader of a split-K cluster: publish the partial tile, wait for the leader
+          for (int cc = 0; cc < p.mma_n; cc += 32) {
+            uint32_t r[32];
+            if (have_acc) {
+              tmem_ld32(tacc + (uint32_t)cc, r);
+              tmem_wait_ld();
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) r[j] = 0u;
+            }
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(my_row + (uint32_t)(cc + 4 * c) * 4u),
+                           "r"(r[4 * c]), "r"(r[4 * c + 1]), "r"(r[4 * c + 2]), "r"(r[4 * c + 3])
+                           : "memory");
+          }
+          tc_fence_before();
+          mbar_arrive_remote(mapa_shared(red_ready_bar, 0));
+          if (!warp_wait_bounded(red_done_bar, 0, p, lane, true)) ok = false;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty_bar(buf));
+          break;  // a split-K cluster owns exactly one tile
+        }
+        if (S > 1) {
+          if (!warp_wait_bounded(red_ready_bar, 0, p, lane, true)) { ok = false; }
+        }
+        float bias_n = 0.0f;
+        if (has_bias && p.bias_axis == 0 && n_ok) bias_n = load_elem(p.bias, n, p.bias_dtype);
+        for (int cc = 0; ok && cc < p.mma_n; cc += 32) {
+          float v[32];
+          if (have_acc) {
+            uint32_t r[32];
+            tmem_ld32(tacc + (uint32_t)cc, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+          }
+          for (int rk = 1; rk < S; ++rk) {
+            const uint32_t rrow = mapa_shared(my_row + (uint32_t)cc * 4u, (uint32_t)rk);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const float4 f = ld_shared_cluster_f4(rrow + 16u * c);
+              v[4 * c] += f.x;
+              v[4 * c + 1] += f.y;
+              v[4 * c + 2] += f.z;
+              v[4 * c + 3] += f.w;
+            }
+          }
+          if (cc + 32 >= p.mma_n) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(buf));
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int m = m_tile0 + cc + j;
+            if (m >= p.M) continue;  // uniform across the warp
+            float x = v[j];
+            if (has_bias) x += (p.bias_axis == 0) ? bias_n : load_elem(p.bias, m, p.bias_dtype);
+            if (has_aux) {
+              const uint32_t word = __ballot_sync(0xffffffffu, n_ok && x > 0.0f);
+              const int w = (ta * 128 + q * 32) >> 5;
+              if (lane == 0 && (long long)w * 32 < p.N) p.aux[(long long)m * p.ld_aux + w] = word;
+            }
+            float y = activate<ACT>(x, 0.0f);
+            if (has_res && n_ok) y += load_elem(p.residual, (long long)m * p.ldr + n, p.res_dtype);
+            y *= scale;
+            if (n_ok) store_elem<OUT>(p.out, (long long)m * p.ldo + n, y);
+          }
+        }
+        if (S > 1) {
+          // the leader has read every peer's partial: release them
+          for (int rk = 1; rk < S; ++rk) mbar_arrive_remote(mapa_shared(red_done_bar, (uint32_t)rk));
+          break;
+        }
+        if (!ok) break;
+      }
+    }
+    (void)ok;
+  }
+
+  // ================================================================ teardown
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+}
+
+}  // namespace fl

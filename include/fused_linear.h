@@ -1,0 +1,174 @@
+/*
+ * fused_linear.h — C ABI of the B200 (sm_100a) fused linear layer
+ *
+ *     y = ((act(A·Wᵀ + bias)) + residual) · scale        (one kernel launch)
+ *
+ * Sources (web pages on GEMM epilogue fusion, cited by title and section):
+ *   [epilog] "通过 cuBLASLt 的 epilog 机制实现单内核偏置融合：参数配置与性能收益"
+ *            — the Matmul → plan(epilog, epilog_inputs{"bias"}) → execute → free
+ *            statement of the problem; compute_type; the RELU_BIAS / GELU_BIAS /
+ *            RELU_AUX_BIAS epilogs; bias shape = the result's output-feature
+ *            dimension; inputs must outlive execute().
+ *   [gelu]   zwxr.cn/news/294525 "Linear+GELU 算子融合" — §1/§2.1 exact GELU,
+ *            §2.2.2 tanh form (0.044715), §3.1 the unfused GEMM-then-GELU design.
+ *   [mlp]    "PyTorch MLP 核算子融合：從 nn.Linear 到 Fused MLP" — nn.Linear is
+ *            x·Wᵀ + bias with W stored [out, in]; the GeGLU MLP gelu(g)*u.
+ *   [mhc]    mhpn.cn/news/2504128 "mHC 融合" — §2.2 elementwise chain (bias,
+ *            residual add, multiply by a constant), §3.3 GEMM-epilogue fusion.
+ *
+ * Conventions shared by every entry point
+ *   - All pointers are DEVICE pointers of the current CUDA device except the
+ *     out-parameter of fl_plan and the descriptor struct (host).
+ *   - Matrices are row-major with an explicit leading dimension in ELEMENTS
+ *     (0 = packed).  Every row pitch must be a multiple of 16 bytes and every
+ *     base pointer 16-byte aligned (the tensor-memory-accelerator rule);
+ *     otherwise FL_ERR_ALIGNMENT.  Logical extents may be ragged.
+ *   - The caller owns every buffer and the stream.  Calls are asynchronous and
+ *     stream-ordered; buffers must stay alive and unmodified until the stream
+ *     has been synchronised ([epilog]: epilog inputs must outlive execute()).
+ *   - Nothing aborts.  Every call returns an fl_status; on failure a message
+ *     is available from fl_last_error() (thread-local, valid until the next
+ *     call on that thread).  There is no CPU fallback: without a B200 the
+ *     calls that launch kernels return FL_ERR_CUDA / FL_ERR_UNSUPPORTED.
+ */
+#ifndef FUSED_LINEAR_H_
+#define FUSED_LINEAR_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FL_OK = 0,
+  FL_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad enum, missing operand */
+  FL_ERR_UNSUPPORTED = 2,  /* combination not offered (e.g. a 16-bit accumulate) */
+  FL_ERR_ALIGNMENT = 3,    /* pointer or row pitch not 16-byte aligned */
+  FL_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed (message has the text) */
+  FL_ERR_OOM = 5,          /* plan workspace allocation failed */
+  FL_ERR_TIMEOUT = 6,      /* a bounded in-kernel wait gave up (see fl_check_status) */
+  FL_ERR_DEVICE = 7        /* no usable sm_100 device */
+} fl_status;
+
+/* Storage types of operands and results. */
+typedef enum { FL_F16 = 0, FL_BF16 = 1, FL_F32 = 2 } fl_dtype;
+
+/* Compute type ([epilog] compute_type).  Accumulation is always FP32; the
+ * pages warn against a 16-bit accumulate, so none is offered.
+ *   FL_COMPUTE_32F        fp16/bf16 operands, fp32 accumulate (tensor cores).
+ *   FL_COMPUTE_32F_3XTF32 fp32 operands, each split hi+lo into TF32 and
+ *                         multiplied as hi·hi + hi·lo + lo·hi, fp32 accumulate. */
+typedef enum { FL_COMPUTE_32F = 0, FL_COMPUTE_32F_3XTF32 = 1 } fl_compute;
+
+/* Epilogue kinds ([epilog] MatmulEpilog; [gelu] exact/tanh GELU; [mlp] GeGLU).
+ *   NONE            y = acc
+ *   BIAS            y = acc + bias
+ *   RELU_BIAS       y = max(acc + bias, 0)
+ *   RELU_AUX_BIAS   as RELU_BIAS, and aux bit (m,n) = (acc + bias > 0)
+ *   GELU_BIAS       y = gelu_erf(acc + bias)   = 0.5·v·(1 + erf(v/√2))
+ *   GELU_TANH_BIAS  y = gelu_tanh(acc + bias)  = 0.5·v·(1 + tanh(√(2/π)(v + 0.044715 v³)))
+ *   GEGLU_TANH      W is the stacked [2N, K] matrix [Wg; Wu]; y = gelu_tanh(A·Wgᵀ)·(A·Wuᵀ)
+ * Every kind may add a residual and scale: y = (act(v) + residual)·scale. */
+typedef enum {
+  FL_EPI_NONE = 0,
+  FL_EPI_BIAS = 1,
+  FL_EPI_RELU_BIAS = 2,
+  FL_EPI_RELU_AUX_BIAS = 3,
+  FL_EPI_GELU_BIAS = 4,
+  FL_EPI_GELU_TANH_BIAS = 5,
+  FL_EPI_GEGLU_TANH = 6
+} fl_epi_kind;
+
+/* The "epilog" argument of fl_plan.  Zero-initialise, then set fields. */
+typedef struct {
+  int32_t kind;            /* fl_epi_kind */
+  int32_t out_dtype;       /* fl_dtype of y */
+  int32_t bias_dtype;      /* fl_dtype of bias (ignored for NONE / GEGLU_TANH) */
+  int32_t residual_dtype;  /* fl_dtype of residual (when has_residual) */
+  int32_t bias_axis;       /* 0: bias[n], per output column of A·Wᵀ (nn.Linear);
+                              1: bias[m], per row — [epilog]'s W·x example, where the
+                              output features are the result's first dimension */
+  int32_t has_residual;    /* 1: add residual[m,n] after the activation */
+  float scale;             /* multiply after the residual; 0 is read as 1 */
+  int32_t b_major;         /* 0: W stored [N,K] (K contiguous, nn.Linear weight);
+                              1: second operand stored [K,N] (N contiguous, [epilog]'s x) */
+  int64_t lda, ldb, ldo, ldr; /* leading dimensions in elements, 0 = packed */
+  int32_t unfused;         /* 1: bare GEMM into a plan-owned buffer, then one
+                              elementwise kernel per epilogue step — the unfused
+                              design of [gelu] §3.1, kept only to measure the
+                              round trip that fusion removes */
+  int32_t reserved[3];     /* must be 0 */
+} fl_epilogue_desc;
+
+typedef struct fl_plan_s* fl_plan_t;
+
+/* Plan one fused linear layer of shape M×N×K ([epilog] Matmul(...).plan(epilog)).
+ * Validates the combination, chooses the kernel configuration for the shape,
+ * and allocates the plan's small device workspace (an error word, plus the
+ * intermediate buffer of an unfused plan).  Needs the target device current.
+ *   out     receives the plan handle (host pointer, must not be NULL)
+ *   M, N, K ≥ 1 for M and N, ≥ 0 for K (K = 0 gives y = epi(0 + bias)); for
+ *           GEGLU_TANH, N is the width of h and W has 2N rows
+ *   dtype   fl_dtype of A and W (F16/BF16 with FL_COMPUTE_32F, F32 with 3XTF32)
+ * Errors: FL_ERR_INVALID_ARG, FL_ERR_UNSUPPORTED, FL_ERR_DEVICE, FL_ERR_OOM. */
+fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, int32_t dtype,
+                  int32_t compute, const fl_epilogue_desc* epi);
+
+/* Run the planned layer on `stream` (a cudaStream_t; NULL = legacy default stream)
+ * ([epilog] execute(): one kernel launch for a fused plan).
+ *   A        [M, lda] operand
+ *   W        [N, ldb] weight (b_major 0), [K, ldb] (b_major 1) or [2N, ldb] (GEGLU)
+ *   bias     length N (bias_axis 0) or M (bias_axis 1); required iff the kind has a bias
+ *   aux      [M, ceil(N/32)] uint32, required iff RELU_AUX_BIAS, packed rows;
+ *            bit j of word w of row m is column 32w+j, least significant bit first;
+ *            bits of columns ≥ N are written as 0
+ *   residual [M, ldr], required iff has_residual
+ *   out      [M, ldo] result
+ * Errors: FL_ERR_INVALID_ARG (missing operand), FL_ERR_ALIGNMENT, FL_ERR_CUDA. */
+fl_status fl_execute(fl_plan_t plan, const void* A, const void* W, const void* bias,
+                     uint32_t* aux, const void* residual, void* out, void* stream);
+
+/* Backward of RELU_AUX_BIAS: dpre[m,n] = grad[m,n] · bit(m,n), with the mask
+ * written by a RELU_AUX_BIAS forward ([epilog]: the aux ReLU mask serves the
+ * backward pass).  grad/dpre are [M, ld] of dtype (F16/BF16/F32); ld 0 = packed;
+ * aux is [M, ceil(N/32)] packed.  dpre may alias grad.
+ * Errors: FL_ERR_INVALID_ARG, FL_ERR_ALIGNMENT, FL_ERR_CUDA. */
+fl_status fl_relu_backward(const void* grad, const uint32_t* aux, void* dpre, int64_t M,
+                           int64_t N, int64_t ld_grad, int64_t ld_dpre, int32_t dtype,
+                           void* stream);
+
+/* Synchronise `stream` and read the plan's device error word.  Returns
+ * FL_ERR_TIMEOUT if a bounded wait inside a kernel of this plan gave up
+ * (the error word is then cleared), FL_ERR_CUDA on a CUDA error, else FL_OK. */
+fl_status fl_check_status(fl_plan_t plan, void* stream);
+
+/* Describe the configuration the plan chose (all fields are host-side ints). */
+typedef struct {
+  int32_t tile_m, tile_n;      /* output tile of one CTA (before split-K) */
+  int32_t mma_n;               /* tensor-core N per instruction */
+  int32_t swap_ab;             /* 1: W is the tensor-core A operand (small M) */
+  int32_t split_k;             /* CTAs of a cluster sharing one tile along K */
+  int32_t stages;              /* shared-memory pipeline depth */
+  int32_t grid;                /* CTAs launched by the main kernel */
+  int32_t smem_bytes;          /* dynamic shared memory per CTA */
+  int32_t launches_per_execute;/* kernels one fl_execute launches */
+  int32_t reserved[7];
+} fl_plan_info;
+fl_status fl_get_plan_info(fl_plan_t plan, fl_plan_info* info);
+
+/* Release a plan and its workspace ([epilog] free()).  NULL is accepted.
+ * Synchronises nothing: the caller must not free a plan with work in flight. */
+fl_status fl_free(fl_plan_t plan);
+
+/* Thread-local text of the last failure on this thread ("" if none). */
+const char* fl_last_error(void);
+
+/* Override the bound on every in-kernel wait for plans created afterwards
+ * (nanoseconds; 0 restores the default of 2 s).  Test/debug use. */
+fl_status fl_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FUSED_LINEAR_H_ */

@@ -1,0 +1,214 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Small and ragged shapes are compared element by element over the whole
+output; the full-size synthetic workloads are compared on sampled rows that
+the oracle computes one by one (the GPU computes everything, in the launch
+configuration the benchmark times).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fl():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import gemm_bias_activation_tcgen05_b200 as m
+    return m
+
+
+def _linear_case(fl, M, N, K, *, dtype="bf16", epilogue="GELU_BIAS", out_dtype="bf16", bias_axis=0,
+                 residual=False, scale=1.0, b_major=0, seed=0, bias_dtype=None, unfused=False):
+    bias_dtype = bias_dtype or ("f32" if dtype == "f32" else dtype)
+    has_bias = epilogue not in ("NONE",)
+    inp = workloads.ragged_linear_inputs(M, N, K, dtype, seed, bias_dtype=bias_dtype if has_bias else None,
+                                         bias_axis=bias_axis, residual=residual, b_major=b_major)
+    W = inp["B"] if b_major else inp["W"]
+    got = P.run_linear(fl, M=M, N=N, K=K, dtype=dtype, epilogue=epilogue, out_dtype=out_dtype, A=inp["A"],
+                       W=W, bias=inp.get("bias"), bias_dtype=bias_dtype, bias_axis=bias_axis, b_major=b_major,
+                       residual=inp.get("residual"), residual_dtype=dtype, scale=scale, unfused=unfused)
+    y, aux, v, absdot = P.oracle_linear(A=inp["A"], W=W, bias=inp.get("bias"), bias_axis=bias_axis,
+                                        b_major=b_major, residual=inp.get("residual"), scale=scale,
+                                        epilogue=epilogue, out_dtype=out_dtype, M=M, N=N, K=K)
+    what = f"{epilogue} {dtype}->{out_dtype} M{M} N{N} K{K} info={got['info']}"
+    P.check_close(got["out"], y, out_dtype, absdot, what)
+    if epilogue == "RELU_AUX_BIAS":
+        P.check_mask(got["aux"], v, N, what)
+    return got
+
+
+def test_single_tile_plain_gemm(fl):
+    _linear_case(fl, 128, 128, 64, epilogue="NONE", out_dtype="f32")
+
+
+def test_multi_kblock_multi_tile(fl):
+    _linear_case(fl, 256, 512, 320, epilogue="NONE", out_dtype="f32")
+
+
+@pytest.mark.parametrize("out_dtype", ["bf16", "f32", "f16"])
+@pytest.mark.parametrize("epilogue", ["NONE", "BIAS", "RELU_BIAS", "RELU_AUX_BIAS", "GELU_BIAS", "GELU_TANH_BIAS"])
+def test_epilogues_ragged(fl, epilogue, out_dtype):
+    # ragged in every dimension: M, N not tile multiples, K not a multiple of 64
+    _linear_case(fl, 300, 520, 200, epilogue=epilogue, out_dtype=out_dtype, seed=11)
+
+
+def test_fp16_operands(fl):
+    _linear_case(fl, 257, 264, 136, dtype="f16", epilogue="GELU_TANH_BIAS", out_dtype="f16", bias_dtype="f16")
+
+
+def test_bias_per_row(fl):
+    _linear_case(fl, 200, 384, 96, epilogue="RELU_BIAS", out_dtype="f32", bias_axis=1, bias_dtype="f32")
+
+
+def test_residual_and_scale(fl):
+    _linear_case(fl, 384, 640, 256, epilogue="GELU_BIAS", out_dtype="f32", residual=True, scale=0.5)
+
+
+@pytest.mark.parametrize("M,N,K", [(100, 256, 784), (129, 200, 72), (256, 512, 128)])
+def test_b_stored_k_by_n(fl, M, N, K):
+    _linear_case(fl, M, N, K, dtype="f16", epilogue="RELU_BIAS", out_dtype="f32", bias_axis=1,
+                 bias_dtype="f32", b_major=1)
+
+
+@pytest.mark.parametrize("M", [1, 5, 32, 77, 128])
+def test_small_m_swap_split_k(fl, M):
+    got = _linear_case(fl, M, 1000, 1000, epilogue="GELU_BIAS", out_dtype="f32", residual=True, scale=0.5,
+                       seed=M)
+    assert got["info"]["swap_ab"] == 1
+
+
+@pytest.mark.parametrize("M", [16, 100])
+def test_small_m_relu_aux(fl, M):
+    _linear_case(fl, M, 520, 264, epilogue="RELU_AUX_BIAS", out_dtype="bf16", seed=3)
+
+
+def test_k_zero_is_bias_only(fl):
+    _linear_case(fl, 130, 136, 0, epilogue="GELU_BIAS", out_dtype="f32", residual=True, scale=0.5)
+
+
+@pytest.mark.parametrize("M,N,K", [(200, 300, 136), (128, 128, 64), (257, 136, 768)])
+def test_geglu_dual(fl, M, N, K):
+    inp = workloads.ragged_linear_inputs(M, N, K, "bf16", 5, dual=True)
+    A, W = inp["A"], inp["W"]
+    ldh = -(-N // 8) * 8
+    got = P.run_linear(fl, M=M, N=N, K=K, dtype="bf16", epilogue="GEGLU_TANH", out_dtype="bf16", A=A, W=W)
+    a = P.to64(A)[:, :K]
+    w = P.to64(W)
+    Wg, Wu = w[:N, :K], w[N:2 * N, :K]
+    h = oracle.geglu_h(a, Wg, Wu, "bf16")
+    g = oracle.gemm(a, Wg)
+    u = oracle.gemm(a, Wu)
+    absdot = float((oracle.gemm(np.abs(a), np.abs(Wg)) * np.abs(u) * 1.2
+                    + oracle.gemm(np.abs(a), np.abs(Wu)) * np.abs(oracle.gelu_tanh(g))).max())
+    assert ldh >= N
+    P.check_close(got["out"], h, "bf16", absdot, f"geglu {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("epilogue", ["RELU_AUX_BIAS", "GELU_TANH_BIAS", "NONE"])
+def test_unfused_twin(fl, epilogue):
+    got = _linear_case(fl, 256, 384, 192, epilogue=epilogue, out_dtype="bf16", unfused=True, seed=7)
+    assert got["info"]["launches_per_execute"] >= 1
+
+
+def test_unfused_residual_f32(fl):
+    _linear_case(fl, 200, 264, 128, epilogue="GELU_BIAS", out_dtype="f32", residual=True, scale=0.5,
+                 unfused=True)
+
+
+@pytest.mark.parametrize("M,N,dtype", [(64, 4096, "bf16"), (33, 1000, "bf16"), (7, 77, "f32"), (5, 40, "f16")])
+def test_relu_backward(fl, M, N, dtype):
+    g = torch.Generator().manual_seed(M * N)
+    v = torch.randn(M, N, generator=g, dtype=torch.float64).numpy()
+    aux = oracle.relu_aux_mask(v)
+    grad = torch.randn(M, N, generator=g).to(P.TD[dtype])
+    dgrad = grad.cuda()
+    daux = torch.from_numpy(aux.view(np.int32)).cuda()
+    dpre = P.poison((M, N), dtype)
+    fl.fl_relu_backward(dgrad, daux, dpre, M, N, dtype)
+    torch.cuda.synchronize()
+    ref = oracle.drelu(P.to64(grad), aux, N, dtype)
+    out = P.to64(dpre)
+    assert np.array_equal(out, ref)
+    # grad·0 keeps the sign of grad, as an IEEE multiply does
+    assert np.array_equal(np.signbit(out), np.signbit(ref))
+
+
+# ---------------------------------------------------------------- full-size workloads
+def _run_workload_linear(fl, w, seed=0, rows=256):
+    inp = workloads.make_inputs(w, seed)
+    W = inp["B"] if w.b_major else inp["W"]
+    got = P.run_linear(fl, M=w.M, N=w.N, K=w.K, dtype=w.dtype, epilogue=w.epilogue, out_dtype=w.out_dtype,
+                       A=inp["A"], W=W, bias=inp.get("bias"), bias_dtype=w.bias_dtype or "bf16",
+                       bias_axis=w.bias_axis, b_major=w.b_major, residual=inp.get("residual"),
+                       residual_dtype=w.dtype, scale=w.scale, out_pad=1)
+    sel = P.sample_rows(w.M, rows, seed) if w.M > rows else None
+    y, aux, v, absdot = P.oracle_linear(A=inp["A"], W=W, bias=inp.get("bias"), bias_axis=w.bias_axis,
+                                        b_major=w.b_major, residual=inp.get("residual"), scale=w.scale,
+                                        epilogue=w.epilogue, out_dtype=w.out_dtype, M=w.M, N=w.N, K=w.K,
+                                        rows=sel)
+    out = got["out"] if sel is None else got["out"][sel]
+    P.check_close(out, y, w.out_dtype, absdot, f"{w.name} seed {seed} info={got['info']}")
+    if w.epilogue == "RELU_AUX_BIAS":
+        aux_g = got["aux"] if sel is None else got["aux"][sel]
+        P.check_mask(aux_g, v, w.N, w.name)
+    return got, inp, sel, v
+
+
+@pytest.mark.parametrize("name", ["relu_bias_100x256x784", "linear_gelu_tanh_bf16_1024x3072x768",
+                                  "tail_m32", "tail_m128", "tail_m512", "tail_m2048"])
+def test_workload_linear(fl, name):
+    _run_workload_linear(fl, workloads.get(name))
+
+
+def test_workload_relu_aux_with_backward(fl):
+    w = workloads.get("relu_aux_4096")
+    got, inp, sel, v = _run_workload_linear(fl, w)
+    # backward on the full mask the forward wrote
+    aux = torch.from_numpy(got["aux"].view(np.int32)).cuda()
+    grad = inp["grad"].cuda()
+    dpre = P.poison((w.M, w.N), "bf16")
+    fl.fl_relu_backward(grad, aux, dpre, w.M, w.N, "bf16")
+    torch.cuda.synchronize()
+    ref = oracle.drelu(P.to64(inp["grad"])[sel], got["aux"][sel], w.N, "bf16")
+    assert np.array_equal(P.to64(dpre)[sel], ref)
+
+
+def test_workload_geglu_mlp(fl):
+    w = workloads.get("geglu_mlp_8192x3072x768")
+    inp = workloads.make_inputs(w, 0)
+    x, Wg, Wu, Wd = inp["x"], inp["Wg"], inp["Wu"], inp["Wd"]
+    Wgu = torch.cat([Wg, Wu], 0)
+    dx, dW, dWd = x.cuda(), Wgu.cuda(), Wd.cuda()
+    h = P.poison((w.M, w.N), "bf16")
+    y = P.poison((w.M, w.K), "bf16")
+    up = fl.Plan(w.M, w.N, w.K, kind="GEGLU_TANH", out_dtype="bf16")
+    down = fl.Plan(w.M, w.K, w.N, kind="NONE", out_dtype="bf16")
+    try:
+        up.execute(dx, dW, out=h)
+        down.execute(h, dWd, out=y)
+        assert up.check() == fl.FL_OK and down.check() == fl.FL_OK, fl.fl_last_error()
+    finally:
+        up.free()
+        down.free()
+    sel = P.sample_rows(w.M, 128, 0)
+    a = P.to64(x)[sel]
+    g = oracle.gemm(a, P.to64(Wg))
+    u = oracle.gemm(a, P.to64(Wu))
+    h_ref = oracle.round_to(oracle.gelu_tanh(g) * u, "bf16")
+    h_got = P.to64(h)[sel]
+    absdot_h = float((oracle.gemm(np.abs(a), np.abs(P.to64(Wg))) * np.abs(u) * 1.2
+                      + oracle.gemm(np.abs(a), np.abs(P.to64(Wu))) * np.abs(oracle.gelu_tanh(g))).max())
+    P.check_close(h_got, h_ref, "bf16", absdot_h, "geglu h")
+    # y against the oracle's down projection of the GPU's own bf16 h (isolates the second GEMM)
+    y_ref = oracle.round_to(oracle.gemm(h_got, P.to64(Wd)), "bf16")
+    absdot_y = float(oracle.gemm(np.abs(h_got), np.abs(P.to64(Wd))).max())
+    P.check_close(P.to64(y)[sel], y_ref, "bf16", absdot_y, "geglu down_proj")
