@@ -1,0 +1,502 @@
+"""Benchmark of the B200 fused linear layer.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+every synthetic workload of the fused linear layer once, each through the C ABI
+as a single fused launch —
+  relu_bias_100x256x784                relu(W·x + b), fp16, B stored [K,N], bias per row
+  linear_gelu_f32_1024x3072x768        exact GELU, fp32 operands (3xTF32)   [when built]
+  linear_gelu_tanh_bf16_1024x3072x768  tanh GELU, bf16
+  geglu_mlp_8192x3072x768              dual gate/up GEMM with gelu_tanh(g)·u, then down_proj
+  relu_aux_4096                        RELU_AUX_BIAS forward + dReLU backward
+  tail_m{32,128,512,2048}              bias → GELU(erf) → +residual → ×0.5, fp32 out
+The headline value is the whole step's algorithmic TFLOP/s (2·M·N·K per GEMM);
+each launch is also timed with CUDA events on its stream for the per-workload
+breakdown and the roofline of the dominant kernel.
+
+Every workload owns its tensors, so a kernel's operands were last touched one
+full step (several hundred MB of other traffic) earlier: the inputs of a step
+are larger than L2 and nothing is L2-resident between iterations.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU (torchrun): independent replicas, weak scaling, max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused Linear+bias+act TFLOP/s (% of BF16 tensor peak); GeGLU MLP fwd µs"
+SUITE = ["relu_bias_100x256x784", "linear_gelu_f32_1024x3072x768", "linear_gelu_tanh_bf16_1024x3072x768",
+         "geglu_mlp_8192x3072x768", "relu_aux_4096", "tail_m32", "tail_m128", "tail_m512", "tail_m2048"]
+DOMINANT = "relu_aux_4096"   # the largest single fused launch of the step
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_setup(n_gpus):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        loaded = [s for s in sm if mx and s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm
+class Suite:
+    """Device tensors and plans of every workload; launch() runs one step."""
+
+    def __init__(self, fl, seed=0):
+        import torch
+        import workloads
+        self.fl, self.torch = fl, torch
+        self.items = []
+        self.flops = 0.0
+        self.min_bytes = {}
+        for name in SUITE:
+            w = workloads.get(name)
+            if w.dtype == "f32" and not self._f32_supported():
+                continue
+            inp = workloads.make_inputs(w, seed)
+            it = {"w": w, "host": inp}
+            if w.kind == "geglu":
+                x, Wgu, Wd = inp["x"], torch.cat([inp["Wg"], inp["Wu"]], 0), inp["Wd"]
+                it["dev"] = {"x": x.cuda(), "Wgu": Wgu.cuda(), "Wd": Wd.cuda()}
+                it["h"] = torch.empty(w.M, w.N, dtype=torch.bfloat16, device="cuda")
+                it["y"] = torch.empty(w.M, w.K, dtype=torch.bfloat16, device="cuda")
+                it["plans"] = [fl.Plan(w.M, w.N, w.K, kind="GEGLU_TANH", out_dtype="bf16"),
+                               fl.Plan(w.M, w.K, w.N, kind="NONE", out_dtype="bf16")]
+                it["host_in"] = {"x": x, "Wgu": Wgu, "Wd": Wd}
+                it["outs"] = ["y"]
+                self.min_bytes[name] = 2 * (w.M * w.K + 2 * w.N * w.K + 2 * w.M * w.N + w.K * w.N + w.M * w.K)
+            else:
+                td = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
+                dev = {k: v.cuda() for k, v in inp.items()}
+                it["dev"] = dev
+                it["out"] = torch.empty(w.M, w.N, dtype=td[w.out_dtype], device="cuda")
+                it["aux"] = (torch.empty(w.M, (w.N + 31) // 32, dtype=torch.int32, device="cuda")
+                             if w.epilogue == "RELU_AUX_BIAS" else None)
+                it["dpre"] = (torch.empty(w.M, w.N, dtype=torch.bfloat16, device="cuda")
+                              if w.kind == "relu_aux" else None)
+                it["plans"] = [fl.Plan(w.M, w.N, w.K, dtype=w.dtype,
+                                       compute="32F_3XTF32" if w.dtype == "f32" else "32F",
+                                       kind=w.epilogue, out_dtype=w.out_dtype, bias_dtype=w.bias_dtype or "bf16",
+                                       residual_dtype=w.dtype, bias_axis=w.bias_axis, has_residual=w.residual,
+                                       scale=w.scale, b_major=w.b_major)]
+                it["host_in"] = {k: v for k, v in inp.items() if k != "grad" or w.kind == "relu_aux"}
+                it["outs"] = ["out"] + (["aux"] if it["aux"] is not None else []) + \
+                             (["dpre"] if it["dpre"] is not None else [])
+                es = {"f16": 2, "bf16": 2, "f32": 4}
+                b = es[w.dtype] * (w.M * w.K + w.N * w.K) + es[w.out_dtype] * w.M * w.N
+                if w.bias_dtype:
+                    b += es[w.bias_dtype] * (w.M if w.bias_axis else w.N)
+                if w.residual:
+                    b += es[w.dtype] * w.M * w.N
+                if it["aux"] is not None:
+                    b += 4 * w.M * ((w.N + 31) // 32)
+                self.min_bytes[name] = b
+            self.flops += w.flops
+            self.items.append(it)
+
+    @staticmethod
+    def _f32_supported():
+        return False  # the 3xTF32 path is not in the library yet
+
+    def launches_per_step(self):
+        n = 0
+        for it in self.items:
+            n += len(it["plans"]) + (1 if it.get("dpre") is not None else 0)
+        return n
+
+    def run_item(self, it, stream):
+        fl, w, d = self.fl, it["w"], it["dev"]
+        if w.kind == "geglu":
+            it["plans"][0].execute(d["x"], d["Wgu"], out=it["h"], stream=stream)
+            it["plans"][1].execute(it["h"], d["Wd"], out=it["y"], stream=stream)
+            return
+        W = d["B"] if w.b_major else d["W"]
+        it["plans"][0].execute(d["A"], W, d.get("bias"), it["aux"], d.get("residual"), it["out"], stream=stream)
+        if it["dpre"] is not None:
+            fl.fl_relu_backward(d["grad"], it["aux"], it["dpre"], w.M, w.N, "bf16", stream=stream)
+
+    def check(self):
+        for it in self.items:
+            for p in it["plans"]:
+                st = p.check()
+                if st != self.fl.FL_OK:
+                    raise RuntimeError(f"{it['w'].name}: status {st}: {self.fl.fl_last_error()}")
+
+
+def run_ours(args):
+    import torch
+    import gemm_bias_activation_tcgen05_b200 as fl
+
+    ws, rank, local = dist_setup(args.gpus)
+    pk = peaks()
+    suite = Suite(fl, seed=rank)
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    # ---- warm-up (untimed), then a correctness status check of every plan
+    for _ in range(max(args.warmup, 3)):
+        for it in suite.items:
+            suite.run_item(it, sh)
+    torch.cuda.synchronize()
+    suite.check()
+
+    # ---- timed region: K steps, per-launch events on the launching stream
+    n_items = len(suite.items)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_items)]
+          for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for s in range(args.steps):
+            for i, it in enumerate(suite.items):
+                ev[s][i][0].record(stream)
+                suite.run_item(it, sh)
+                ev[s][i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    total_ms = max_over_ranks(t0.elapsed_time(t1), ws)
+    suite.check()
+    ms_step = total_ms / args.steps
+    per_item = {}
+    for i, it in enumerate(suite.items):
+        times = [ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)]
+        per_item[it["w"].name] = {"ms_mean": sum(times) / len(times), "ms_median": statistics.median(times)}
+
+    # ---- e2e through the public API with host buffers: pinned H2D of every operand,
+    # the launches, D2H of every result, all inside the timed region
+    e2e = e2e_measure(suite, stream, sh, args, ws)
+
+    value = ws * suite.flops * args.steps / (total_ms * 1e-3) / 1e12
+    breakdown = {}
+    for it in suite.items:
+        w = it["w"]
+        t = per_item[w.name]["ms_mean"]
+        tfl = w.flops / (t * 1e-3) / 1e12
+        gbs = suite.min_bytes[w.name] / (t * 1e-3) / 1e9
+        roof_t = max(w.flops / (pk["bf16_tflops"] * 1e12), suite.min_bytes[w.name] / (pk["hbm_gbs"] * 1e9))
+        breakdown[w.name] = {"us": round(t * 1e3, 2), "tflops": round(tfl, 1), "gbs_min_bytes": round(gbs, 1),
+                             "roofline_us": round(roof_t * 1e6, 2), "roofline_frac": round(roof_t / (t * 1e-3), 3)}
+    dom = suite.items[[it["w"].name for it in suite.items].index(DOMINANT)]
+    dom_w = dom["w"]
+    # the dominant fused GEMM launch alone (its dReLU follows inside the same event pair,
+    # so the forward is timed separately below on the same stream)
+    fwd_ms = time_single_launch(suite, dom, stream, sh, reps=max(10, args.steps // 2))
+    achieved = dom_w.flops / (fwd_ms * 1e-3) / 1e12
+    peak = pk["bf16_tflops_sustained"]
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 3), "traffic": profiled_traffic(), "kernel": "fl_gemm_epi_tcgen05",
+                "launch": f"{DOMINANT} forward (M=N=K=4096, RELU_AUX_BIAS)",
+                "peak_kind": f"{pk['src']} bf16 sustained (kernel timed inside a long step)",
+                "frac_of_burst": round(achieved / pk["bf16_tflops"], 3)}
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "all synthetic workloads of the fused linear layer, one fused launch each: "
+                               + ", ".join(it["w"].name for it in suite.items),
+                   "flops_per_step": suite.flops, "parallelism": f"replicas x{ws}",
+                   "l2": "inputs larger than L2: every workload owns its operands; a step touches "
+                         f"{sum(suite.min_bytes.values()) / 1e6:.0f} MB"},
+        "impl": "ours",
+        "geglu_mlp_fwd_us": breakdown.get("geglu_mlp_8192x3072x768", {}).get("us"),
+        "pct_of_bf16_peak": round(100 * value / ws / pk["bf16_tflops"], 1),
+        "e2e": e2e,
+        "gpu_launches": suite.launches_per_step() * args.steps,
+        "roofline": roofline,
+        "clocks": clk.summary(),
+        "breakdown": breakdown,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for it in suite.items:
+        for p in it["plans"]:
+            p.free()
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def time_single_launch(suite, it, stream, sh, reps):
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    w, d = it["w"], it["dev"]
+    # flush L2 between launches with a 256 MB write (outside the event pair)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device="cuda")
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        it["plans"][0].execute(d["A"], d["W"], d.get("bias"), it["aux"], d.get("residual"), it["out"], stream=sh)
+        b.record(stream)
+    torch.cuda.synchronize()
+    del flush
+    return sum(a.elapsed_time(b) for a, b in evs) / reps
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
+    or None when the kernel source changed after the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "fl_gemm_epi_relu_aux_4096.md")
+    if not os.path.exists(p):
+        return None
+    src = os.path.join(ROOT, "gemm_bias_activation_tcgen05_b200", "csrc", "fl_gemm.cuh")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for line in open(p):
+        if ":" in line and line.strip().startswith(("kernel_source_sha256_16", "dram_bytes_per_launch")):
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256_16") != h:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def e2e_measure(suite, stream, sh, args, ws):
+    import torch
+    host = []
+    h2d = d2h = 0
+    for it in suite.items:
+        pin_in = {k: v.pin_memory() for k, v in it["host_in"].items()}
+        outs = {}
+        for k in it["outs"]:
+            t = it[k] if k in it else None
+            if t is None:
+                continue
+            outs[k] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        host.append((it, pin_in, outs))
+        h2d += sum(v.numel() * v.element_size() for v in pin_in.values())
+        d2h += sum(v.numel() * v.element_size() for v in outs.values())
+
+    def step():
+        for it, pin_in, outs in host:
+            for k, v in pin_in.items():
+                it["dev"][k].copy_(v, non_blocking=True)
+            suite.run_item(it, sh)
+            for k, v in outs.items():
+                v.copy_(it[k], non_blocking=True)
+
+    steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), ws) / steps
+    return {"value": round(ws * suite.flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3)}
+
+
+# ---------------------------------------------------------------- oracle on the host cores
+def _oracle_sample(seconds):
+    """Run the oracle (as it stands) over row-slices of every workload until about
+    `seconds` of CPU work is done; returns (flops, elapsed, cores, description)."""
+    import numpy as np
+    import oracle
+    import workloads
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] or [os.cpu_count() or 1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    flops, elapsed, parts = 0.0, 0.0, []
+    rows_per_chunk = 64
+    names = [n for n in SUITE]
+    data = {}
+    for n in names:
+        w = workloads.get(n)
+        data[n] = (w, {k: v.double().numpy() for k, v in workloads.make_inputs(w, 0).items()})
+    r0 = 0
+    while elapsed < seconds and r0 < 8192:
+        for n in names:
+            w, inp = data[n]
+            if r0 >= w.M:
+                continue
+            r1 = min(w.M, r0 + rows_per_chunk)
+            t = time.perf_counter()
+            if w.kind == "geglu":
+                oracle.geglu_mlp(inp["x"][r0:r1], inp["Wg"], inp["Wu"], inp["Wd"], "bf16")
+                f = 2.0 * (r1 - r0) * w.K * 3 * w.N
+            else:
+                Wm = inp["B"] if w.b_major else inp["W"]
+                bias = inp.get("bias")
+                if bias is not None and w.bias_axis == 1:
+                    bias = bias[r0:r1]
+                res = inp.get("residual")
+                y, aux, v = oracle.fused_linear(inp["A"][r0:r1], Wm, bias, epilogue=w.epilogue,
+                                                out_dtype=w.out_dtype, bias_axis=w.bias_axis, b_major=w.b_major,
+                                                residual=None if res is None else res[r0:r1], scale=w.scale)
+                if aux is not None:
+                    oracle.drelu(inp["grad"][r0:r1], aux, w.N, "bf16")
+                f = 2.0 * (r1 - r0) * w.N * w.K
+            elapsed += time.perf_counter() - t
+            flops += f
+        r0 += rows_per_chunk
+    desc = (f"oracle (numpy/scipy fp64) on row slices [0:{r0}) of every workload "
+            f"({flops / 1e9:.1f} GFLOP, {elapsed:.1f} s)")
+    return flops, elapsed, cores, desc
+
+
+def cpu_baseline(seconds):
+    flops, elapsed, cores, desc = _oracle_sample(seconds)
+    return {"value": round(flops / elapsed / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": desc}
+
+
+def run_reference(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    # steps x warmup of bounded oracle samples; the whole run stays within minutes
+    per_step = max(1.0, min(6.0, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        _oracle_sample(per_step / 4)
+    tot_f, tot_t, cores, desc = 0.0, 0.0, 1, ""
+    for _ in range(args.steps):
+        f, t, cores, desc = _oracle_sample(per_step)
+        tot_f += f
+        tot_t += t
+    value = tot_f / tot_t / 1e12
+    line = {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * tot_t / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "all synthetic workloads of the fused linear layer (row-sliced sample)",
+                       "parallelism": "host cores"},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": desc + f"; per step about {per_step:.1f} s"},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

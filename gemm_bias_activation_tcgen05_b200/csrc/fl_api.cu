@@ -65,6 +65,25 @@ static fl_status get_encode() {
 
 static int esize(int dt) { return dt == FL_F32 ? 4 : 2; }
 
+// FL_SYNC_EACH_LAUNCH=1 (debug only): synchronise after every launch and name
+// the launch whose execution failed.
+static bool sync_each_launch() {
+  static const bool on = [] {
+    const char* v = getenv("FL_SYNC_EACH_LAUNCH");
+    return v && v[0] == '1';
+  }();
+  return on;
+}
+static fl_status after_launch(cudaStream_t s, const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FL_ERR_CUDA, "%s: launch: %s", what, cudaGetErrorString(e));
+  if (sync_each_launch()) {
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return fail(FL_ERR_CUDA, "%s: execution: %s", what, cudaGetErrorString(e));
+  }
+  return FL_OK;
+}
+
 static CUtensorMapDataType tm_dtype(int dt) {
   if (dt == FL_F32) return CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   if (dt == FL_BF16) return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -128,6 +147,7 @@ struct fl_plan_s {
   int* d_err;
   // unfused twin
   void* d_tmp;
+  int64_t tmp_ld;
   size_t tmp_bytes;
   int launches;
 };
@@ -185,7 +205,8 @@ static fl_status choose_config(fl_plan_s* p) {
   // and split K across a cluster so that every SM streams a slice of W.
   p->swap = (M <= 128) && !geglu && !p->epi.b_major && p->dtype != FL_F32;
   if (p->swap) {
-    p->mma_n = (int)std::max<int64_t>(16, cdiv(M, 16) * 16);
+    // The epilogue moves TMEM in 32-column chunks, so the activation tile is a multiple of 32.
+    p->mma_n = (int)std::max<int64_t>(32, cdiv(M, 32) * 32);
     p->out_tile_n = p->mma_n;
     p->tiles_a = (int)cdiv(N, 128);
     p->tiles_b = (int)cdiv(M, p->mma_n);
@@ -307,7 +328,9 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
   else p->grid = std::min(tiles, p->num_sms);
   p->kernel = pick_kernel(p->act, epi->out_dtype, p->swap);
   if (!p->kernel) { delete p; return fail(FL_ERR_UNSUPPORTED, "fl_plan: no kernel for this combination"); }
-  cudaError_t e = cudaFuncSetAttribute(p->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, p->smem);
+  // Every plan sharing a kernel may need a different amount of dynamic shared
+  // memory, so the kernel's bound is the device maximum, not this plan's size.
+  cudaError_t e = cudaFuncSetAttribute(p->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, p->max_smem);
   if (e != cudaSuccess) { delete p; return fail(FL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e)); }
   if (p->split_k > 1) {
     e = cudaFuncSetAttribute(p->kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
@@ -324,7 +347,8 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
     // GEMM into a plan-owned intermediate (the [M, N] or [M, 2N] result), then one
     // elementwise kernel per epilogue step.
     const int64_t cols = (epi->kind == FL_EPI_GEGLU_TANH) ? 2 * N : N;
-    p->tmp_bytes = (size_t)M * (size_t)cols * (size_t)eo;
+    p->tmp_ld = cdiv(cols * eo, 16) * 16 / eo;  // 16-byte row pitch for the TMA store
+    p->tmp_bytes = (size_t)M * (size_t)p->tmp_ld * (size_t)eo;
     if (cudaMalloc(&p->d_tmp, p->tmp_bytes) != cudaSuccess) {
       cudaFree(p->d_err);
       delete p;
@@ -459,9 +483,13 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
                     (uint32_t)p->mma_n);
     }
     if (st) return st;
+    // The TMA store covers whole 16-byte granules of a row only; the kernel writes
+    // the ragged remainder (< 16 bytes per row) with plain stores.
     const int eo = esize(g.out_dtype);
-    st = make_map(&tmOut, g.out, g.out_dtype, (uint64_t)g.n_cols, (uint64_t)p->M, (uint64_t)g.ldo * eo,
-                  (uint32_t)(128 / eo), 32);
+    const int64_t n_tma = (g.n_cols * eo / 16) * 16 / eo;
+    k.n_tma = (int)n_tma;
+    st = make_map(&tmOut, g.out, g.out_dtype, (uint64_t)std::max<int64_t>(n_tma, 16 / eo), (uint64_t)p->M,
+                  (uint64_t)g.ldo * eo, (uint32_t)(128 / eo), 32);
     if (st) return st;
   } else if (!no_k) {
     // UMMA A = weight rows (output features), UMMA B = activation rows
@@ -494,7 +522,7 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
   cudaError_t err = cudaLaunchKernelEx(&cfg, reinterpret_cast<KernelFn>(const_cast<void*>(kernel)), tmA, tmB,
                                        tmB2, tmOut, k);
   if (err != cudaSuccess) return fail(FL_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(err));
-  return FL_OK;
+  return after_launch(stream, "fused GEMM kernel");
 }
 
 static int grid_for(long long work, int num_sms) {
@@ -509,9 +537,7 @@ template <int DT>
 static fl_status launch_ew_t(const EwParams& P, int num_sms, cudaStream_t s) {
   const long long work = P.M * ((P.N + 31) / 32);
   fl_ew_step_kernel<DT><<<grid_for(work, num_sms), 256, 0, s>>>(P);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(FL_ERR_CUDA, "elementwise launch: %s", cudaGetErrorString(e));
-  return FL_OK;
+  return after_launch(s, "elementwise step kernel");
 }
 static fl_status launch_ew(int dt, const EwParams& P, int num_sms, cudaStream_t s) {
   if (dt == FL_BF16) return launch_ew_t<DT_BF16>(P, num_sms, s);
@@ -554,7 +580,7 @@ extern "C" fl_status fl_execute(fl_plan_t p, const void* A, const void* W, const
   const int64_t cols = geglu ? 2 * p->N : p->N;
   const bool no_steps = (e.kind == FL_EPI_NONE) && !e.has_residual && e.scale == 1.0f;
   void* gemm_out = no_steps ? out : p->d_tmp;
-  const int64_t gemm_ld = no_steps ? e.ldo : cols;
+  const int64_t gemm_ld = no_steps ? e.ldo : p->tmp_ld;
   {
     // The unfused GEMM uses the same tcgen05 kernel with no epilogue work.
     fl_plan_s q = *p;
@@ -568,7 +594,7 @@ extern "C" fl_status fl_execute(fl_plan_t p, const void* A, const void* W, const
     const int tiles = q.tiles_a * q.tiles_b;
     q.grid = (q.swap && q.split_k > 1) ? tiles * q.split_k : std::min(tiles, q.num_sms);
     const void* kern = pick_kernel(ACT_NONE, odt, q.swap);
-    FL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, q.smem));
+    FL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, q.max_smem));
     q.epi.ldr = 0;
     q.epi.has_residual = 0;
     GemmArgs g{A, W, gemm_out, odt, gemm_ld, ACT_NONE, nullptr, nullptr, nullptr, 1.0f, cols, false};
@@ -580,24 +606,36 @@ extern "C" fl_status fl_execute(fl_plan_t p, const void* A, const void* W, const
   P.M = p->M;
   P.N = p->N;
   P.src = p->d_tmp;
-  P.lds = cols;
+  P.lds = p->tmp_ld;
   P.dst = out;
   P.ldd = e.ldo;
+  P.err = p->d_err;
+  const long long tmp_elems = (long long)(p->tmp_bytes / (size_t)esize(odt));
+  const long long out_elems = (p->M - 1) * e.ldo + p->N;
+  P.src_elems = tmp_elems;
+  P.dst_elems = out_elems;
+  P.aux_elems = p->M * cdiv(p->N, 32);
   auto step = [&](int op, const void* operand, int odtype, int64_t ldop) -> fl_status {
     P.op = op;
     P.operand = operand;
     P.operand_dtype = odtype;
     P.ldop = ldop;
+    if (op == EW_BIAS_N) P.op_elems = p->N;
+    else if (op == EW_BIAS_M) P.op_elems = p->M;
+    else if (op == EW_RESIDUAL) P.op_elems = (p->M - 1) * e.ldr + p->N;
+    else if (op == EW_GEGLU_MUL) P.op_elems = tmp_elems - p->N;
+    else P.op_elems = 0;
     fl_status st = launch_ew(odt, P, p->num_sms, stream);
     P.src = out;  // every later step works in place on `out`
     P.lds = e.ldo;
+    P.src_elems = out_elems;
     return st;
   };
   fl_status st = FL_OK;
   if (geglu) {
     // h = gelu_tanh(g) * u, with g = tmp[:, :N] and u = tmp[:, N:]
     P.op = EW_GEGLU_MUL;
-    st = step(EW_GEGLU_MUL, static_cast<const char*>(p->d_tmp) + (size_t)p->N * esize(odt), odt, cols);
+    st = step(EW_GEGLU_MUL, static_cast<const char*>(p->d_tmp) + (size_t)p->N * esize(odt), odt, p->tmp_ld);
     if (st) return st;
   } else {
     if (p->has_bias) {
@@ -626,7 +664,7 @@ extern "C" fl_status fl_execute(fl_plan_t p, const void* A, const void* W, const
     if (st) return st;
   }
   if (P.src == p->d_tmp) {  // no step ran (e.g. NONE with nothing else): copy through
-    FL_CUDA(cudaMemcpy2DAsync(out, (size_t)e.ldo * esize(odt), p->d_tmp, (size_t)cols * esize(odt),
+    FL_CUDA(cudaMemcpy2DAsync(out, (size_t)e.ldo * esize(odt), p->d_tmp, (size_t)p->tmp_ld * esize(odt),
                               (size_t)p->N * esize(odt), (size_t)p->M, cudaMemcpyDeviceToDevice, stream));
   }
   return FL_OK;
@@ -662,8 +700,7 @@ extern "C" fl_status fl_relu_backward(const void* grad, const uint32_t* aux, voi
     fl_relu_backward_kernel<DT_F16><<<grid, 256, 0, s>>>(grad, aux, dpre, M, N, ld_grad, ld_dpre, words, vec_ok);
   else
     fl_relu_backward_kernel<DT_F32><<<grid, 256, 0, s>>>(grad, aux, dpre, M, N, ld_grad, ld_dpre, words, vec_ok);
-  FL_CUDA(cudaGetLastError());
-  return FL_OK;
+  return after_launch(s, "dReLU kernel");
 }
 
 // ------------------------------------------------------------------ status
@@ -675,6 +712,8 @@ extern "C" fl_status fl_check_status(fl_plan_t p, void* stream_) {
   FL_CUDA(cudaMemcpy(&h, p->d_err, sizeof(int), cudaMemcpyDeviceToHost));
   if (h != 0) {
     FL_CUDA(cudaMemset(p->d_err, 0, sizeof(int)));
+    if (h >= 100)
+      return fail(FL_ERR_DEVICE, "an elementwise kernel skipped an out-of-range access (code %d)", h);
     return fail(FL_ERR_TIMEOUT, "a bounded in-kernel wait gave up (code %d)", h);
   }
   return FL_OK;

@@ -117,7 +117,17 @@ struct EwParams {
   float scale;
   uint32_t* aux;
   long long ld_aux;
+  // element counts of every buffer: an access outside them is skipped and
+  // recorded in *err (code 100 + op) instead of being performed
+  long long src_elems, dst_elems, op_elems, aux_elems;
+  int* err;
 };
+
+__device__ __forceinline__ bool ew_in(long long i, long long n, int* err, int code) {
+  if (i >= 0 && i < n) return true;
+  atomicCAS(err, 0, code);
+  return false;
+}
 
 template <int DT>
 __device__ __forceinline__ float ew_ld(const void* p, long long i) {
@@ -143,26 +153,42 @@ __global__ void __launch_bounds__(256) fl_ew_step_kernel(const EwParams P) {
     const long long n0 = w * 32;
     uint32_t mask = 0;
     const int cnt = (int)min(32LL, P.N - n0);
+    const int code = 100 + P.op;
     for (int j = 0; j < cnt; ++j) {
       const long long n = n0 + j;
-      const float x = ew_ld<DT>(P.src, m * P.lds + n);
+      const long long is = m * P.lds + n;
+      if (!ew_in(is, P.src_elems, P.err, code)) continue;
+      const float x = ew_ld<DT>(P.src, is);
       float y;
+      long long io = -1;
       switch (P.op) {
-        case EW_BIAS_N: y = x + load_elem(P.operand, n, P.operand_dtype); break;
-        case EW_BIAS_M: y = x + load_elem(P.operand, m, P.operand_dtype); break;
+        case EW_BIAS_N: io = n; break;
+        case EW_BIAS_M: io = m; break;
+        case EW_RESIDUAL:
+        case EW_GEGLU_MUL: io = m * P.ldop + n; break;
+        default: break;
+      }
+      if (io >= 0 && !ew_in(io, P.op_elems, P.err, code)) continue;
+      switch (P.op) {
+        case EW_BIAS_N:
+        case EW_BIAS_M: y = x + load_elem(P.operand, io, P.operand_dtype); break;
         case EW_RELU:
           y = fmaxf(x, 0.0f);
           if (x > 0.0f) mask |= 1u << j;
           break;
         case EW_GELU: y = gelu_erf_f(x); break;
         case EW_GELU_TANH: y = gelu_tanh_f(x); break;
-        case EW_RESIDUAL: y = x + load_elem(P.operand, m * P.ldop + n, P.operand_dtype); break;
+        case EW_RESIDUAL: y = x + load_elem(P.operand, io, P.operand_dtype); break;
         case EW_SCALE: y = x * P.scale; break;
-        default: y = gelu_tanh_f(x) * load_elem(P.operand, m * P.ldop + n, P.operand_dtype); break;
+        default: y = gelu_tanh_f(x) * load_elem(P.operand, io, P.operand_dtype); break;
       }
-      ew_st<DT>(P.dst, m * P.ldd + n, y);
+      const long long id = m * P.ldd + n;
+      if (ew_in(id, P.dst_elems, P.err, code)) ew_st<DT>(P.dst, id, y);
     }
-    if (P.op == EW_RELU && P.aux != nullptr) P.aux[m * P.ld_aux + w] = mask;
+    if (P.op == EW_RELU && P.aux != nullptr) {
+      const long long ia = m * P.ld_aux + w;
+      if (ew_in(ia, P.aux_elems, P.err, code)) P.aux[ia] = mask;
+    }
   }
 }
 

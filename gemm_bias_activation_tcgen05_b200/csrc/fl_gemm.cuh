@@ -77,6 +77,7 @@ struct KParams {
   uint32_t* aux;
   long long ld_aux;
   float scale;
+  int n_tma;  // columns [0, n_tma) go out by TMA store; n_tma·size is a multiple of 16 bytes
   int* err;
   unsigned long long wait_limit_ns;
 };
@@ -409,6 +410,16 @@ __global__ void __launch_bounds__(kNumThreads, 1)
               if ((long long)w * 32 < p.N) p.aux[(long long)m * p.ld_aux + w] = aux_word[h];
             }
           }
+          // ---- ragged row end: a TMA store writes whole 16-byte granules, so the
+          // columns past the last full granule are written with plain stores.
+          if (nc0 + CH > p.n_tma && nc0 < p.N && m_ok) {
+            const int j0 = max(p.n_tma - nc0, 0);
+            const int j1 = min(p.N - nc0, CH);
+#pragma unroll
+            for (int j = 0; j < CH; ++j)
+              if (j >= j0 && j < j1) store_elem<OUT>(p.out, (long long)m * p.ldo + nc0 + j, v[j]);
+          }
+          if (nc0 >= p.n_tma) continue;
           // ---- stage the 32 x 128-byte block in 128B-swizzled smem, TMA-store it
           uint32_t words[32];
           if constexpr (OUT == DT_F32) {
