@@ -132,6 +132,15 @@ static const void* pick_kernel(int act, int out, bool swap) {
 }
 
 // ------------------------------------------------------------------ plan
+// Tensor maps and kernel parameters of the last launch of one call site: a
+// repeat call with the same operand pointers launches without re-encoding.
+struct LaunchCache {
+  bool valid = false;
+  const void* key[8] = {};
+  CUtensorMap tmA, tmB, tmB2, tmOut;
+  KParams k;
+};
+
 struct fl_plan_s {
   int64_t M, N, K;
   int dtype, compute;
@@ -150,6 +159,8 @@ struct fl_plan_s {
   int64_t tmp_ld;
   size_t tmp_bytes;
   int launches;
+  uint64_t wait_limit_ns;
+  LaunchCache cache_fused, cache_unfused;
 };
 
 static int act_of(int kind) {
@@ -165,9 +176,11 @@ static int act_of(int kind) {
 
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Shared-memory budget of one configuration (bytes, before the 1 KB alignment slack).
+// Shared-memory layout of one configuration: the operand ring, then (normal
+// layout) the epilogue staging buffers and per-warp bias rows, then (split-K)
+// the reduction buffer, then the barriers.
 struct Layout {
-  uint32_t a_stage, b_box, b_stage, stage, staging_off, bar_off, red_off, red_pitch, total;
+  uint32_t a_stage, b_box, b_stage, stage, staging_off, bias_off, bar_off, red_off, red_pitch, total;
   int stages;
 };
 
@@ -180,15 +193,17 @@ static Layout layout_for(const fl_plan_s* p, int mma_n, int b_boxes, int max_sme
   else L.b_box = (uint32_t)(mma_n / b_boxes) * 128u;
   L.b_stage = L.b_box * (uint32_t)b_boxes;
   L.stage = L.a_stage + L.b_stage;
-  const uint32_t staging = p->swap ? 0u : kStagingBytes;
+  const uint32_t staging = p->swap ? Cfg<true>::kStagingBytes : Cfg<false>::kStagingBytes;
+  const uint32_t bias = 0;
   const uint32_t red = (p->swap && p->split_k > 1) ? 128u * ((uint32_t)mma_n * 4u + 16u) : 0u;
-  const uint32_t bars = 8u * (2u * 16u + 8u) + 16u;
-  const uint32_t budget = (uint32_t)max_smem - 1024u - staging - red - bars;
+  const uint32_t bars = 8u * (2u * 8u + 8u);
+  const uint32_t budget = (uint32_t)max_smem - 1024u - staging - bias - red - bars;
   int st = (int)(budget / L.stage);
   if (st > 8) st = 8;
   L.stages = st;
   L.staging_off = (uint32_t)st * L.stage;
-  L.red_off = L.staging_off + staging;
+  L.bias_off = L.staging_off + staging;
+  L.red_off = L.bias_off + bias;
   L.red_pitch = (uint32_t)mma_n * 4u + 16u;
   L.bar_off = L.red_off + red;
   L.total = L.bar_off + 8u * (2u * (uint32_t)st + 8u) + 1024u;
@@ -223,12 +238,15 @@ static fl_status choose_config(fl_plan_s* p) {
       p->out_tile_n = 128;
     } else {
       // Pick the N tile that minimises (waves x tile width) on this GPU.
+      // Cost ~ (rounds of tiles per SM) x (tile width) x (relative cost per column):
+      // a 128-wide UMMA tile moves more operand bytes per FLOP and issues twice
+      // the instructions, measured at about 1.6x the per-column cost of 256.
       int best = 256;
       double best_cost = 1e300;
       for (int bn : {256, 128}) {
         const int64_t tiles = cdiv(M, 128) * cdiv(N, bn);
         const double waves = (double)cdiv(tiles, p->num_sms);
-        const double cost = waves * bn * (bn == 128 ? 1.04 : 1.0);
+        const double cost = waves * bn * (bn == 128 ? 1.6 : 1.0);
         if (cost < best_cost) { best_cost = cost; best = bn; }
       }
       p->mma_n = best;
@@ -343,7 +361,22 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
     return fail(FL_ERR_CUDA, "fl_plan: cudaMemset(error word)");
   }
   p->launches = 1;
+  p->wait_limit_ns = g_wait_limit_ns;
   if (epi->unfused) {
+    // the bare GEMM kernels of both layouts may serve this plan's first step
+    for (int sw = 0; sw < 2; ++sw) {
+      const void* kn = pick_kernel(ACT_NONE, epi->out_dtype, sw == 1);
+      if (cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, p->max_smem) != cudaSuccess) {
+        cudaFree(p->d_err);
+        delete p;
+        return fail(FL_ERR_CUDA, "cudaFuncSetAttribute (unfused GEMM)");
+      }
+    }
+    int steps = 0;
+    if (epi->kind == FL_EPI_GEGLU_TANH) steps += 1;
+    else steps += (has_bias ? 1 : 0) + (p->act != ACT_NONE ? 1 : 0);
+    steps += (epi->has_residual ? 1 : 0) + (p->epi.scale != 1.0f ? 1 : 0);
+    p->launches = 1 + steps;
     // GEMM into a plan-owned intermediate (the [M, N] or [M, 2N] result), then one
     // elementwise kernel per epilogue step.
     const int64_t cols = (epi->kind == FL_EPI_GEGLU_TANH) ? 2 * N : N;
@@ -400,8 +433,32 @@ struct GemmArgs {
   bool geglu_fused;
 };
 
+static fl_status launch_kernel(const fl_plan_s* p, const LaunchCache& c, cudaStream_t stream,
+                               const void* kernel, bool swap) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)p->grid, 1, 1);
+  cfg.blockDim = dim3(swap ? Cfg<true>::kThreads : Cfg<false>::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)p->smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  if (p->split_k > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)p->split_k;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  cudaError_t err = cudaLaunchKernelEx(&cfg, reinterpret_cast<KernelFn>(const_cast<void*>(kernel)), c.tmA, c.tmB,
+                                       c.tmB2, c.tmOut, c.k);
+  if (err != cudaSuccess) return fail(FL_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(err));
+  return after_launch(stream, "fused GEMM kernel");
+}
+
 static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t stream, const void* kernel,
-                             bool swap, int act) {
+                             bool swap, int act, LaunchCache* cache) {
+  const void* key[8] = {g.A, g.W, g.out, g.bias, g.residual, g.aux, kernel, (const void*)(intptr_t)g.ldo};
+  if (cache->valid && memcmp(cache->key, key, sizeof(key)) == 0) return launch_kernel(p, *cache, stream, kernel, swap);
   const int es = esize(p->dtype);
   const int bk = 128 / es;
   const fl_epilogue_desc& e = p->epi;
@@ -429,13 +486,13 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
   k.b_box_bytes = L.b_box;
   k.stage_bytes = L.stage;
   k.staging_off = L.staging_off;
+  k.bias_off = L.bias_off;
   k.red_off = L.red_off;
   k.red_pitch = L.red_pitch;
   k.bar_off = L.bar_off;
   const uint32_t fmt = (p->dtype == FL_BF16) ? 1u : 0u;
   k.idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(e.b_major ? 1 : 0) << 16) |
             ((uint32_t)(p->mma_n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-  k.ksteps = bk / 16;               // UMMA K = 16 elements (32 bytes) for f16/bf16
   k.a_kstep = 32;
   k.b_kstep = e.b_major ? 16u * 128u : 32u;
   k.b_lbo = e.b_major ? L.b_box : 16u;
@@ -455,7 +512,7 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
   k.ld_aux = cdiv(p->M > 0 ? g.n_cols : 0, 32);
   k.scale = g.scale;
   k.err = p->d_err;
-  k.wait_limit_ns = g_wait_limit_ns;
+  k.wait_limit_ns = p->wait_limit_ns;
 
   CUtensorMap tmA, tmB, tmB2, tmOut;
   memset(&tmB2, 0, sizeof(tmB2));
@@ -503,26 +560,15 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
     tmOut = tmA;  // unused in the swap layout
   }
   if (!g.geglu_fused) tmB2 = tmB;  // unused
-
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)p->grid, 1, 1);
-  cfg.blockDim = dim3(kNumThreads, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)p->smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  if (p->split_k > 1) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)p->split_k;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  }
   (void)act;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, reinterpret_cast<KernelFn>(const_cast<void*>(kernel)), tmA, tmB,
-                                       tmB2, tmOut, k);
-  if (err != cudaSuccess) return fail(FL_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(err));
-  return after_launch(stream, "fused GEMM kernel");
+  cache->tmA = tmA;
+  cache->tmB = tmB;
+  cache->tmB2 = tmB2;
+  cache->tmOut = tmOut;
+  cache->k = k;
+  memcpy(cache->key, key, sizeof(key));
+  cache->valid = true;
+  return launch_kernel(p, *cache, stream, kernel, swap);
 }
 
 static int grid_for(long long work, int num_sms) {
@@ -572,7 +618,7 @@ extern "C" fl_status fl_execute(fl_plan_t p, const void* A, const void* W, const
 
   if (!e.unfused) {
     GemmArgs g{A, W, out, e.out_dtype, e.ldo, p->act, bias, residual, aux, e.scale, p->N, geglu};
-    return launch_gemm(p, g, stream, p->kernel, p->swap, p->act);
+    return launch_gemm(p, g, stream, p->kernel, p->swap, p->act, &p->cache_fused);
   }
 
   // ---- unfused twin: bare GEMM into the intermediate, then one kernel per step
@@ -594,11 +640,10 @@ extern "C" fl_status fl_execute(fl_plan_t p, const void* A, const void* W, const
     const int tiles = q.tiles_a * q.tiles_b;
     q.grid = (q.swap && q.split_k > 1) ? tiles * q.split_k : std::min(tiles, q.num_sms);
     const void* kern = pick_kernel(ACT_NONE, odt, q.swap);
-    FL_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, q.max_smem));
     q.epi.ldr = 0;
     q.epi.has_residual = 0;
     GemmArgs g{A, W, gemm_out, odt, gemm_ld, ACT_NONE, nullptr, nullptr, nullptr, 1.0f, cols, false};
-    fl_status st = launch_gemm(&q, g, stream, kern, q.swap, ACT_NONE);
+    fl_status st = launch_gemm(&q, g, stream, kern, q.swap, ACT_NONE, &p->cache_unfused);
     if (st) return st;
   }
   if (no_steps) return FL_OK;

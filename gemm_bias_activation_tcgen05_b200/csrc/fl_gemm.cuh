@@ -37,12 +37,19 @@ namespace fl {
 enum Act : int { ACT_NONE = 0, ACT_RELU = 1, ACT_GELU = 2, ACT_GELU_TANH = 3, ACT_GEGLU = 4 };
 enum DType : int { DT_F16 = 0, DT_BF16 = 1, DT_F32 = 2 };
 
-constexpr int kNumThreads = 192;
-constexpr int kEpiWarp0 = 2;
-constexpr int kNumEpiWarps = 4;
-constexpr uint32_t kStagingBuf = 32 * 128;  // one warp's 32 rows x 128 bytes
-constexpr uint32_t kStagingBytes = kNumEpiWarps * 2 * kStagingBuf;
+constexpr int kEpiWarp0 = 2;                 // warps 0,1: TMA producer, UMMA issuer
+constexpr uint32_t kStagingBuf = 32 * 128;    // one epilogue warp's 32 rows x 128 bytes
+constexpr int kUmmaSteps = 4;                 // UMMA instructions per 128-byte K stage
 constexpr int kErrTimeout = 1;
+
+// Normal layout: 8 epilogue warps (two per TMEM lane quarter, one per column
+// half).  Swap-AB layout: 4 epilogue warps (one per lane quarter).
+template <bool SWAP>
+struct Cfg {
+  static constexpr int kEpiWarps = SWAP ? 4 : 8;
+  static constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
+  static constexpr uint32_t kStagingBytes = SWAP ? 0u : kEpiWarps * kStagingBuf;
+};
 
 struct KParams {
   // output space: y is M x N
@@ -63,9 +70,8 @@ struct KParams {
   uint32_t idesc;
   uint32_t a_kstep, b_kstep;  // descriptor start-address advance per UMMA K step (bytes)
   uint32_t b_lbo;             // leading byte offset of an MN-major B operand
-  int ksteps;                 // UMMA instructions per stage
   uint32_t tmem_cols;
-  uint32_t staging_off, bar_off, red_off, red_pitch;
+  uint32_t staging_off, bias_off, bar_off, red_off, red_pitch;
   // epilogue operands
   const void* bias;
   int bias_dtype, bias_axis;
@@ -173,12 +179,55 @@ __device__ __forceinline__ void tile_coords(int t, const KParams& p, int& ta, in
   tb = r / ga;
 }
 
+// ------------------------------------------------------------------ epilogue helpers
+// Load CH consecutive elements of one row (16-byte vectors when the whole chunk
+// is in range, else guarded scalars) and widen them to fp32.
+template <int CH>
+__device__ __forceinline__ void load_row_chunk(float (&dst)[CH], const void* base, long long row_off, int n0,
+                                               int N, int dt, bool full) {
+  if (full) {
+    if (dt == DT_F32) {
+      const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + row_off + n0);
+#pragma unroll
+      for (int i = 0; i < CH / 4; ++i) {
+        const float4 f = __ldg(src + i);
+        dst[4 * i] = f.x;
+        dst[4 * i + 1] = f.y;
+        dst[4 * i + 2] = f.z;
+        dst[4 * i + 3] = f.w;
+      }
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(base) + row_off + n0);
+#pragma unroll
+      for (int i = 0; i < CH / 8; ++i) {
+        const uint4 u = __ldg(src + i);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (dt == DT_BF16) {
+            dst[8 * i + 2 * e] = __uint_as_float(w[e] << 16);
+            dst[8 * i + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+          } else {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+            dst[8 * i + 2 * e] = f.x;
+            dst[8 * i + 2 * e + 1] = f.y;
+          }
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < CH; ++j) dst[j] = (n0 + j < N) ? load_elem(base, row_off + n0 + j, dt) : 0.0f;
+  }
+}
+
 // ------------------------------------------------------------------ kernel
 template <int ACT, int OUT, bool SWAP>
-__global__ void __launch_bounds__(kNumThreads, 1)
+__global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
     fl_gemm_epi_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmOut,
                         const __grid_constant__ KParams p) {
+  constexpr int kEpiWarps = Cfg<SWAP>::kEpiWarps;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5;
@@ -211,11 +260,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), kNumEpiWarps);
+      mbar_init(tempty_bar(b), kEpiWarps);
     }
     mbar_init(drain_bar, 1);
-    mbar_init(red_ready_bar, kNumEpiWarps * 32 * (S > 1 ? S - 1 : 1));
-    mbar_init(red_done_bar, kNumEpiWarps * 32);
+    mbar_init(red_ready_bar, kEpiWarps * 32 * (S > 1 ? S - 1 : 1));
+    mbar_init(red_done_bar, kEpiWarps * 32);
     fence_mbarrier_init();
     if (p.num_kb > 0) {  // with K = 0 the operand maps are left unencoded and never used
       prefetch_tensormap(&tmA);
@@ -243,25 +292,27 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       for (int t = cluster_id; ok && t < total_tiles; t += num_clusters) {
         int ta, tb;
         tile_coords(t, p, ta, tb);
+        const int a_row = ta * 128;
+        const int b_row = tb * p.mma_n;
+        const int g_row = tb * p.b_box_rows;
         for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
           const int s = (int)(it % (uint32_t)NS);
           const uint32_t ph = (it / (uint32_t)NS) & 1u;
           if (!wait_bounded(empty_bar(s), ph ^ 1u, p)) { ok = false; break; }
-          mbar_arrive_expect_tx(full_bar(s), p.stage_bytes);
+          const uint32_t fb = full_bar(s);
+          mbar_arrive_expect_tx(fb, p.stage_bytes);
           const uint32_t sa = smem_base + (uint32_t)s * p.stage_bytes;
           const uint32_t sb = sa + p.a_stage_bytes;
           const int k0 = kb * p.bk;
-          tma_load_2d(sa, &tmA, full_bar(s), k0, ta * 128);
+          tma_load_2d(sa, &tmA, fb, k0, a_row);
           if (p.b_mn_major) {
-            for (int i = 0; i < p.b_boxes; ++i)
-              tma_load_2d(sb + i * p.b_box_bytes, &tmB, full_bar(s), tb * p.mma_n + i * 64, k0);
+            for (int i = 0; i < p.b_boxes; ++i) tma_load_2d(sb + i * p.b_box_bytes, &tmB, fb, b_row + i * 64, k0);
           } else if (p.geglu) {
-            tma_load_2d(sb, &tmB, full_bar(s), k0, tb * p.b_box_rows);
-            tma_load_2d(sb + p.b_box_bytes, &tmB2, full_bar(s), k0, tb * p.b_box_rows);
+            tma_load_2d(sb, &tmB, fb, k0, g_row);
+            tma_load_2d(sb + p.b_box_bytes, &tmB2, fb, k0, g_row);
           } else {
             for (int i = 0; i < p.b_boxes; ++i)
-              tma_load_2d(sb + i * p.b_box_bytes, &tmB, full_bar(s), k0,
-                          tb * p.mma_n + i * p.b_box_rows);
+              tma_load_2d(sb + i * p.b_box_bytes, &tmB, fb, k0, b_row + i * p.b_box_rows);
           }
         }
       }
@@ -276,6 +327,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   } else if (warp == 1) {
     // ================================================================ UMMA issuer
     if (lane == 0) {
+      // Descriptors of stage 0; a stage s and UMMA step k only move the start
+      // address field (addresses stay below 2^18 bytes, so no carry leaves it).
+      const uint64_t da0 = sdesc_sw128(smem_base, 16, 1024);
+      const uint64_t db0 = sdesc_sw128(smem_base + p.a_stage_bytes, p.b_mn_major ? p.b_lbo : 16u, 1024);
+      const uint64_t stage_step = p.stage_bytes >> 4;
+      const uint64_t ak = p.a_kstep >> 4, bk = p.b_kstep >> 4;
+      const uint32_t idesc = p.idesc;
       uint32_t it = 0, local = 0;
       bool ok = true, issued = false;
       for (int t = cluster_id; ok && t < total_tiles; t += num_clusters, ++local) {
@@ -289,14 +347,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const uint32_t ph = (it / (uint32_t)NS) & 1u;
           if (!wait_bounded(full_bar(s), ph, p)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = smem_base + (uint32_t)s * p.stage_bytes;
-          const uint32_t sb = sa + p.a_stage_bytes;
-          for (int k = 0; k < p.ksteps; ++k) {
-            const uint64_t adesc = sdesc_sw128(sa + k * p.a_kstep, 16, 1024);
-            const uint64_t bdesc = p.b_mn_major ? sdesc_sw128(sb + k * p.b_kstep, p.b_lbo, 1024)
-                                                : sdesc_sw128(sb + k * p.b_kstep, 16, 1024);
-            umma_f16(d_tmem, adesc, bdesc, p.idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
-          }
+          const uint64_t da = da0 + (uint64_t)s * stage_step;
+          const uint64_t db = db0 + (uint64_t)s * stage_step;
+#pragma unroll
+          for (int k = 0; k < kUmmaSteps; ++k)
+            umma_f16(d_tmem, da + k * ak, db + k * bk, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
           umma_commit(empty_bar(s));  // frees the stage once these MMAs have read it
           issued = true;
         }
@@ -321,83 +376,100 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     bool ok = true;
 
     if constexpr (!SWAP) {
-      // ---------------- normal layout: thread = output row, columns in registers
+      // ---------------- normal layout: thread = output row, a warp owns half the tile's columns
       constexpr int CH = (OUT == DT_F32) ? 32 : 64;  // output columns per 128-byte staging row
-      const uint32_t stg0 = smem_base + p.staging_off + (uint32_t)ew * 2u * kStagingBuf;
-      int stg_idx = 0;
+      const int half = ew >> 2;
+      const uint32_t stg = smem_base + p.staging_off + (uint32_t)ew * kStagingBuf;
+      const int half_cols = p.out_tile_n >> 1;
       for (int t = cluster_id; t < total_tiles; t += num_clusters, ++local) {
         int ta, tb;
         tile_coords(t, p, ta, tb);
         const uint32_t buf = local & 1u;
         const uint32_t tph = (local >> 1) & 1u;
-        if (!warp_wait_bounded(tfull_bar(buf), tph, p, lane)) { ok = false; break; }
-        tc_fence_after();
         const int row0 = ta * 128 + q * 32;
         const int m = row0 + lane;
         const bool m_ok = m < p.M;
         const int n_tile0 = tb * p.out_tile_n;
-        const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
         float bias_m = 0.0f;
         if (has_bias && p.bias_axis == 1 && m_ok) bias_m = load_elem(p.bias, m, p.bias_dtype);
+        if (!warp_wait_bounded(tfull_bar(buf), tph, p, lane)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
+        const int c_begin = half * half_cols;
+        const int c_end = c_begin + half_cols;
 
-        for (int cc = 0; cc < p.out_tile_n; cc += CH) {
+        for (int cc = c_begin; cc < c_end; cc += CH) {
+          const int nc0 = n_tile0 + cc;
+          const bool full_cols = nc0 + CH <= p.N;
+          // ---- operands that do not depend on the accumulator first (their latency overlaps)
+          float r[CH];
+          if (has_res && m_ok) load_row_chunk<CH>(r, p.residual, (long long)m * p.ldr, nc0, p.N, p.res_dtype, full_cols);
+          float bl[CH / 32];  // lane l holds bias[nc0 + 32i + l]; broadcast by shuffle below
+#pragma unroll
+          for (int i = 0; i < CH / 32; ++i) {
+            const int n = nc0 + i * 32 + lane;
+            bl[i] = (has_bias && p.bias_axis == 0 && n < p.N) ? load_elem(p.bias, n, p.bias_dtype) : 0.0f;
+          }
+          // ---- accumulator: every TMEM load of the chunk, then one wait
           float v[CH];
-          float u[(ACT == ACT_GEGLU) ? CH : 1];
           if (have_acc) {
+            if constexpr (ACT == ACT_GEGLU) {
+              // gate columns [0, out_tile_n) and up columns [out_tile_n, 2·out_tile_n):
+              // h = gelu_tanh(g)·u, 32 columns at a time to bound register use
 #pragma unroll
-            for (int h = 0; h < CH / 32; ++h) {
-              uint32_t r[32];
-              tmem_ld32(tacc + (uint32_t)(cc + h * 32), r);
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[h * 32 + j] = __uint_as_float(r[j]);
-              if constexpr (ACT == ACT_GEGLU) {
-                tmem_ld32(tacc + (uint32_t)(p.out_tile_n + cc + h * 32), r);
+              for (int h = 0; h < CH / 32; ++h) {
+                uint32_t rg[32], ru[32];
+                tmem_ld32(tacc + (uint32_t)(cc + h * 32), rg);
+                tmem_ld32(tacc + (uint32_t)(p.out_tile_n + cc + h * 32), ru);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) u[h * 32 + j] = __uint_as_float(r[j]);
+                for (int j = 0; j < 32; ++j)
+                  v[h * 32 + j] = activate<ACT>(__uint_as_float(rg[j]), __uint_as_float(ru[j]));
               }
+            } else {
+              uint32_t ra[CH];
+#pragma unroll
+              for (int h = 0; h < CH / 32; ++h)
+                tmem_ld32(tacc + (uint32_t)(cc + h * 32), *reinterpret_cast<uint32_t(*)[32]>(&ra[h * 32]));
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < CH; ++j) v[j] = __uint_as_float(ra[j]);
             }
           } else {
 #pragma unroll
-            for (int j = 0; j < CH; ++j) v[j] = 0.0f;
-            if constexpr (ACT == ACT_GEGLU) {
-#pragma unroll
-              for (int j = 0; j < CH; ++j) u[j] = 0.0f;
-            }
+            for (int j = 0; j < CH; ++j) v[j] = (ACT == ACT_GEGLU) ? activate<ACT>(0.0f, 0.0f) : 0.0f;
           }
-          if (cc + CH >= p.out_tile_n) {
-            // all TMEM reads of this tile are done: hand the buffer back to the MMA warp
+          if (cc + CH >= c_end) {
+            // this warp's TMEM reads of the tile are done: hand its share back to the MMA warp
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(buf));
           }
-          const int nc0 = n_tile0 + cc;
           // ---- bias, activation, aux, residual, scale (all in fp32 registers)
+          if (has_bias) {
+            if (p.bias_axis == 0) {
+#pragma unroll
+              for (int j = 0; j < CH; ++j) v[j] += __shfl_sync(0xffffffffu, bl[j >> 5], j & 31);
+            } else {
+#pragma unroll
+              for (int j = 0; j < CH; ++j) v[j] += bias_m;
+            }
+          }
           uint32_t aux_word[CH / 32];
 #pragma unroll
           for (int h = 0; h < CH / 32; ++h) aux_word[h] = 0u;
-          const bool full_cols = nc0 + CH <= p.N;
+          if (has_aux) {
 #pragma unroll
-          for (int j = 0; j < CH; ++j) {
-            const int n = nc0 + j;
-            float x = v[j];
-            if (has_bias) {
-              if (p.bias_axis == 0) x += (n < p.N) ? load_elem(p.bias, n, p.bias_dtype) : 0.0f;
-              else x += bias_m;
-            }
-            if (has_aux && x > 0.0f && (full_cols || n < p.N)) aux_word[j >> 5] |= 1u << (j & 31);
-            float y;
-            if constexpr (ACT == ACT_GEGLU) y = activate<ACT>(x, u[j]);
-            else y = activate<ACT>(x, 0.0f);
-            v[j] = y;
+            for (int j = 0; j < CH; ++j)
+              if (v[j] > 0.0f && (full_cols || nc0 + j < p.N)) aux_word[j >> 5] |= 1u << (j & 31);
+          }
+          if constexpr (ACT != ACT_GEGLU) {
+#pragma unroll
+            for (int j = 0; j < CH; ++j) v[j] = activate<ACT>(v[j], 0.0f);
           }
           if (has_res && m_ok) {
 #pragma unroll
-            for (int j = 0; j < CH; ++j) {
-              const int n = nc0 + j;
-              if (full_cols || n < p.N) v[j] += load_elem(p.residual, (long long)m * p.ldr + n, p.res_dtype);
-            }
+            for (int j = 0; j < CH; ++j) v[j] += r[j];
           }
           if (scale != 1.0f) {
 #pragma unroll
@@ -429,12 +501,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) words[j] = pack2<OUT>(v[2 * j], v[2 * j + 1]);
           }
-          if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read smem
+          if (lane == 0) bulk_wait_group_read<0>();  // the previous store has finished reading smem
           __syncwarp();
-          const uint32_t sbuf = stg0 + (uint32_t)stg_idx * kStagingBuf;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const uint32_t addr = sbuf + (uint32_t)lane * 128u + ((uint32_t)(c ^ (lane & 7)) << 4);
+            const uint32_t addr = stg + (uint32_t)lane * 128u + ((uint32_t)(c ^ (lane & 7)) << 4);
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(words[4 * c]),
                          "r"(words[4 * c + 1]), "r"(words[4 * c + 2]), "r"(words[4 * c + 3])
                          : "memory");
@@ -442,10 +513,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tmOut, sbuf, nc0, row0);
+            tma_store_2d(&tmOut, stg, nc0, row0);
             bulk_commit_group();
           }
-          stg_idx ^= 1;
         }
       }
       if (lane == 0) bulk_wait_group<0>();
@@ -457,12 +527,14 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         tile_coords(t, p, ta, tb);
         const uint32_t buf = local & 1u;
         const uint32_t tph = (local >> 1) & 1u;
-        if (!warp_wait_bounded(tfull_bar(buf), tph, p, lane)) { ok = false; break; }
-        tc_fence_after();
         const int r_lane = q * 32 + lane;            // TMEM lane = row of the W tile
         const int n = ta * 128 + r_lane;             // output column
         const bool n_ok = n < p.N;
         const int m_tile0 = tb * p.mma_n;
+        float bias_n = 0.0f;
+        if (has_bias && p.bias_axis == 0 && n_ok) bias_n = load_elem(p.bias, n, p.bias_dtype);
+        if (!warp_wait_bounded(tfull_bar(buf), tph, p, lane)) { ok = false; break; }
+        tc_fence_after();
         const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
         const uint32_t my_row = red_base + (uint32_t)r_lane * p.red_pitch;
 
@@ -493,8 +565,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         if (S > 1) {
           if (!warp_wait_bounded(red_ready_bar, 0, p, lane, true)) { ok = false; }
         }
-        float bias_n = 0.0f;
-        if (has_bias && p.bias_axis == 0 && n_ok) bias_n = load_elem(p.bias, n, p.bias_dtype);
         for (int cc = 0; ok && cc < p.mma_n; cc += 32) {
           float v[32];
           if (have_acc) {
@@ -508,14 +578,17 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             for (int j = 0; j < 32; ++j) v[j] = 0.0f;
           }
           for (int rk = 1; rk < S; ++rk) {
+            // issue all eight remote loads of this peer's row chunk, then add
             const uint32_t rrow = mapa_shared(my_row + (uint32_t)cc * 4u, (uint32_t)rk);
+            float4 f[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) f[c] = ld_shared_cluster_f4(rrow + 16u * c);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-              const float4 f = ld_shared_cluster_f4(rrow + 16u * c);
-              v[4 * c] += f.x;
-              v[4 * c + 1] += f.y;
-              v[4 * c + 2] += f.z;
-              v[4 * c + 3] += f.w;
+              v[4 * c] += f[c].x;
+              v[4 * c + 1] += f[c].y;
+              v[4 * c + 2] += f[c].z;
+              v[4 * c + 3] += f[c].w;
             }
           }
           if (cc + 32 >= p.mma_n) {
@@ -523,21 +596,30 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(buf));
           }
+          // residual column n of rows m: one coalesced 32-lane load per row, issued up front
+          float rr[32];
+          if (has_res) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int mm = m_tile0 + cc + j;
+              rr[j] = (n_ok && mm < p.M) ? load_elem(p.residual, (long long)mm * p.ldr + n, p.res_dtype) : 0.0f;
+            }
+          }
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const int m = m_tile0 + cc + j;
-            if (m >= p.M) continue;  // uniform across the warp
+            const int mm = m_tile0 + cc + j;
+            if (mm >= p.M) continue;  // uniform across the warp
             float x = v[j];
-            if (has_bias) x += (p.bias_axis == 0) ? bias_n : load_elem(p.bias, m, p.bias_dtype);
+            if (has_bias) x += (p.bias_axis == 0) ? bias_n : load_elem(p.bias, mm, p.bias_dtype);
             if (has_aux) {
               const uint32_t word = __ballot_sync(0xffffffffu, n_ok && x > 0.0f);
               const int w = (ta * 128 + q * 32) >> 5;
-              if (lane == 0 && (long long)w * 32 < p.N) p.aux[(long long)m * p.ld_aux + w] = word;
+              if (lane == 0 && (long long)w * 32 < p.N) p.aux[(long long)mm * p.ld_aux + w] = word;
             }
             float y = activate<ACT>(x, 0.0f);
-            if (has_res && n_ok) y += load_elem(p.residual, (long long)m * p.ldr + n, p.res_dtype);
+            if (has_res) y += rr[j];
             y *= scale;
-            if (n_ok) store_elem<OUT>(p.out, (long long)m * p.ldo + n, y);
+            if (n_ok) store_elem<OUT>(p.out, (long long)mm * p.ldo + n, y);
           }
         }
         if (S > 1) {
