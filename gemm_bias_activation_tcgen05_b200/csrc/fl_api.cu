@@ -226,10 +226,10 @@ static fl_status choose_config(fl_plan_s* p) {
     p->tiles_a = (int)cdiv(N, 128);
     p->tiles_b = (int)cdiv(M, p->mma_n);
     const int tiles = p->tiles_a * p->tiles_b;
-    int S = p->num_sms / std::max(1, tiles);
-    if (S > 8) S = 8;
-    if (S > p->num_kb) S = p->num_kb;
-    if (S < 1) S = 1;
+    // split K over 1, 2 or 4 CTAs of a cluster (a reduce-scatter gives each CTA
+    // 128/S output columns of the tile to finish)
+    int S = 4;
+    while (S > 1 && ((int64_t)tiles * S > p->num_sms || S > p->num_kb)) S >>= 1;
     p->split_k = S;
   } else {
     p->split_k = 1;

@@ -169,18 +169,22 @@ __global__ void __launch_bounds__(256) fl_ew_step_kernel(const EwParams P) {
         default: break;
       }
       if (io >= 0 && !ew_in(io, P.op_elems, P.err, code)) continue;
+      // the operand load sits in its own branch (never folded into a select that
+      // would issue it for an op that has no operand)
+      float opv = 0.0f;
+      if (io >= 0) opv = ldg_pinned(P.operand, io, P.operand_dtype);
       switch (P.op) {
         case EW_BIAS_N:
-        case EW_BIAS_M: y = x + load_elem(P.operand, io, P.operand_dtype); break;
+        case EW_BIAS_M: y = x + opv; break;
         case EW_RELU:
           y = fmaxf(x, 0.0f);
           if (x > 0.0f) mask |= 1u << j;
           break;
         case EW_GELU: y = gelu_erf_f(x); break;
         case EW_GELU_TANH: y = gelu_tanh_f(x); break;
-        case EW_RESIDUAL: y = x + load_elem(P.operand, io, P.operand_dtype); break;
+        case EW_RESIDUAL: y = x + opv; break;
         case EW_SCALE: y = x * P.scale; break;
-        default: y = gelu_tanh_f(x) * load_elem(P.operand, io, P.operand_dtype); break;
+        default: y = gelu_tanh_f(x) * opv; break;
       }
       const long long id = m * P.ldd + n;
       if (ew_in(id, P.dst_elems, P.err, code)) ew_st<DT>(P.dst, id, y);

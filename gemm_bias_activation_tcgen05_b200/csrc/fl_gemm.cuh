@@ -179,6 +179,20 @@ __device__ __forceinline__ void tile_coords(int t, const KParams& p, int& ta, in
   tb = r / ga;
 }
 
+// Pinned read-only global loads: volatile with a memory clobber, so a batch of
+// them stays ahead of the stores that follow and all are in flight together.
+__device__ __forceinline__ float ldg_pinned(const void* base, long long i, int dt) {
+  if (dt == DT_F32) {
+    float v;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(reinterpret_cast<const float*>(base) + i) : "memory");
+    return v;
+  }
+  unsigned short h;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(h) : "l"(reinterpret_cast<const uint16_t*>(base) + i) : "memory");
+  if (dt == DT_BF16) return __uint_as_float(static_cast<uint32_t>(h) << 16);
+  return __half2float(__ushort_as_half(h));
+}
+
 // ------------------------------------------------------------------ epilogue helpers
 // Load CH consecutive elements of one row (16-byte vectors when the whole chunk
 // is in range, else guarded scalars) and widen them to fp32.
@@ -217,7 +231,49 @@ __device__ __forceinline__ void load_row_chunk(float (&dst)[CH], const void* bas
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < CH; ++j) dst[j] = (n0 + j < N) ? load_elem(base, row_off + n0 + j, dt) : 0.0f;
+    for (int j = 0; j < CH; ++j) {
+      dst[j] = 0.0f;
+      if (n0 + j < N) dst[j] = ldg_pinned(base, row_off + n0 + j, dt);
+    }
+  }
+}
+
+// Epilogue of the swap-AB layout for one thread: output column n, rows
+// m0 .. m0+cnt-1 with pre-activations v[0..cnt).  The warp's 32 lanes hold 32
+// consecutive columns starting at n_warp0 (a multiple of 32), so every row's
+// residual load and output store is one coalesced access and the ReLU mask
+// word of the row is one ballot.
+template <int ACT, int OUT>
+__device__ __forceinline__ void swap_finish(const KParams& p, const float (&v)[32], int n, int n_warp0, int m0,
+                                            int cnt, int lane) {
+  const bool n_ok = n < p.N;
+  const bool has_res = p.residual != nullptr;
+  const bool has_bias = p.bias != nullptr;
+  float rr[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) rr[j] = 0.0f;
+  if (has_res && n_ok) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < cnt) rr[j] = ldg_pinned(p.residual, (long long)(m0 + j) * p.ldr + n, p.res_dtype);
+  }
+  float bias_n = 0.0f;
+  if (has_bias && p.bias_axis == 0 && n_ok) bias_n = ldg_pinned(p.bias, n, p.bias_dtype);
+  const int w = n_warp0 >> 5;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    if (j >= cnt) continue;  // uniform across the warp
+    const int m = m0 + j;
+    float x = v[j];
+    if (has_bias) x += (p.bias_axis == 0) ? bias_n : ldg_pinned(p.bias, m, p.bias_dtype);
+    if (p.aux != nullptr) {
+      const uint32_t word = __ballot_sync(0xffffffffu, n_ok && x > 0.0f);
+      if (lane == 0 && (long long)w * 32 < p.N) p.aux[(long long)m * p.ld_aux + w] = word;
+    }
+    float y = activate<ACT>(x, 0.0f);
+    if (has_res) y += rr[j];
+    y *= p.scale;
+    if (n_ok) store_elem<OUT>(p.out, (long long)m * p.ldo + n, y);
   }
 }
 
@@ -263,8 +319,10 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
       mbar_init(tempty_bar(b), kEpiWarps);
     }
     mbar_init(drain_bar, 1);
-    mbar_init(red_ready_bar, kEpiWarps * 32 * (S > 1 ? S - 1 : 1));
-    mbar_init(red_done_bar, kEpiWarps * 32);
+    // split-K hand-off: one arrive per epilogue warp (after __syncwarp, so the
+    // release covers the whole warp's shared-memory writes)
+    mbar_init(red_ready_bar, kEpiWarps * S);
+    mbar_init(red_done_bar, kEpiWarps * S);
     fence_mbarrier_init();
     if (p.num_kb > 0) {  // with K = 0 the operand maps are left unencoded and never used
       prefetch_tensormap(&tmA);
@@ -324,6 +382,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         (void)wait_bounded(full_bar((int)s), (last / (uint32_t)NS) & 1u, p);
       }
     }
+    __syncwarp();  // reconverge: the CTA barrier below is warp-aligned
   } else if (warp == 1) {
     // ================================================================ UMMA issuer
     if (lane == 0) {
@@ -364,6 +423,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         (void)wait_bounded(drain_bar, 0, p);
       }
     }
+    __syncwarp();  // reconverge: the CTA barrier below is warp-aligned
   } else {
     // ================================================================ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
@@ -391,7 +451,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         const bool m_ok = m < p.M;
         const int n_tile0 = tb * p.out_tile_n;
         float bias_m = 0.0f;
-        if (has_bias && p.bias_axis == 1 && m_ok) bias_m = load_elem(p.bias, m, p.bias_dtype);
+        if (has_bias && p.bias_axis == 1 && m_ok) bias_m = ldg_pinned(p.bias, m, p.bias_dtype);
         if (!warp_wait_bounded(tfull_bar(buf), tph, p, lane)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
@@ -408,7 +468,8 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < CH / 32; ++i) {
             const int n = nc0 + i * 32 + lane;
-            bl[i] = (has_bias && p.bias_axis == 0 && n < p.N) ? load_elem(p.bias, n, p.bias_dtype) : 0.0f;
+            bl[i] = 0.0f;
+            if (has_bias && p.bias_axis == 0 && n < p.N) bl[i] = ldg_pinned(p.bias, n, p.bias_dtype);
           }
           // ---- accumulator: every TMEM load of the chunk, then one wait
           float v[CH];
@@ -520,26 +581,49 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
       }
       if (lane == 0) bulk_wait_group<0>();
     } else {
-      // ---------------- swap-AB layout: thread = output column n, columns = output rows m
+      // ---------------- swap-AB layout: TMEM lane = output column n, TMEM column = output row m
       const uint32_t red_base = smem_base + p.red_off;
       for (int t = cluster_id; t < total_tiles; t += num_clusters, ++local) {
         int ta, tb;
         tile_coords(t, p, ta, tb);
         const uint32_t buf = local & 1u;
         const uint32_t tph = (local >> 1) & 1u;
-        const int r_lane = q * 32 + lane;            // TMEM lane = row of the W tile
-        const int n = ta * 128 + r_lane;             // output column
-        const bool n_ok = n < p.N;
         const int m_tile0 = tb * p.mma_n;
-        float bias_n = 0.0f;
-        if (has_bias && p.bias_axis == 0 && n_ok) bias_n = load_elem(p.bias, n, p.bias_dtype);
         if (!warp_wait_bounded(tfull_bar(buf), tph, p, lane)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
-        const uint32_t my_row = red_base + (uint32_t)r_lane * p.red_pitch;
 
-        if (S > 1 && rank != 0) {
-          // ---- non-leader of a split-K cluster: publish the partial tile, wait for the leader
+        if (S == 1) {
+          // the whole tile is this CTA's: warp q finishes TMEM lanes [32q, 32q+32) over every row m
+          const int n = ta * 128 + q * 32 + lane;
+          for (int cc = 0; cc < p.mma_n; cc += 32) {
+            float v[32];
+            if (have_acc) {
+              uint32_t r[32];
+              tmem_ld32(tacc + (uint32_t)cc, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+            }
+            if (cc + 32 >= p.mma_n) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(tempty_bar(buf));
+            }
+            swap_finish<ACT, OUT>(p, v, n, ta * 128 + q * 32, m_tile0 + cc, min(32, p.M - (m_tile0 + cc)), lane);
+          }
+          continue;
+        }
+
+        // ---- split-K over a cluster of S CTAs, reduced as a reduce-scatter through shared
+        // memory: every CTA publishes its fp32 partial tile in its own shared memory; CTA r
+        // then sums all S partials (in rank order) for TMEM lanes [r·128/S, (r+1)·128/S) and
+        // finishes those output columns.
+        {
+          const uint32_t my_row = red_base + (uint32_t)(q * 32 + lane) * p.red_pitch;
           for (int cc = 0; cc < p.mma_n; cc += 32) {
             uint32_t r[32];
             if (have_acc) {
@@ -556,84 +640,69 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
                            : "memory");
           }
           tc_fence_before();
-          mbar_arrive_remote(mapa_shared(red_ready_bar, 0));
-          if (!warp_wait_bounded(red_done_bar, 0, p, lane, true)) ok = false;
           __syncwarp();
-          if (lane == 0) mbar_arrive(tempty_bar(buf));
-          break;  // a split-K cluster owns exactly one tile
+          if (lane == 0) {
+            mbar_arrive(tempty_bar(buf));
+            for (int rk = 0; rk < S; ++rk) mbar_arrive_remote(mapa_shared(red_ready_bar, (uint32_t)rk));
+          }
         }
-        if (S > 1) {
-          if (!warp_wait_bounded(red_ready_bar, 0, p, lane, true)) { ok = false; }
-        }
-        for (int cc = 0; ok && cc < p.mma_n; cc += 32) {
-          float v[32];
-          if (have_acc) {
-            uint32_t r[32];
-            tmem_ld32(tacc + (uint32_t)cc, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          } else {
+        if (!warp_wait_bounded(red_ready_bar, 0, p, lane, true)) ok = false;
+        if (ok) {
+          const int L = 128 / S;             // TMEM lanes this CTA finishes (S is 2 or 4)
+          const int groups = L / 32;         // 32-lane groups among them
+          const int g = ew % groups;
+          const int parts = kEpiWarps / groups;
+          const int part = ew / groups;
+          const int row = (int)rank * L + g * 32 + lane;
+          const int mcnt = p.mma_n / parts;  // a multiple of 8
+          const int mb = part * mcnt;
+          const uint32_t row_addr = red_base + (uint32_t)row * p.red_pitch;
+          for (int mc = mb; mc < mb + mcnt; mc += 32) {
+            const int cnt = min(32, mb + mcnt - mc);
+            // sum the S partials in rank order, two ranks' loads in flight at a time
+            float v[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-          }
-          for (int rk = 1; rk < S; ++rk) {
-            // issue all eight remote loads of this peer's row chunk, then add
-            const uint32_t rrow = mapa_shared(my_row + (uint32_t)cc * 4u, (uint32_t)rk);
-            float4 f[8];
+            for (int rk = 0; rk < S; rk += 2) {
+              float4 f0[8], f1[8];
+              const uint32_t a0 = mapa_shared(row_addr + (uint32_t)mc * 4u, (uint32_t)rk);
+              const uint32_t a1 = mapa_shared(row_addr + (uint32_t)mc * 4u, (uint32_t)(rk + 1));
 #pragma unroll
-            for (int c = 0; c < 8; ++c) f[c] = ld_shared_cluster_f4(rrow + 16u * c);
+              for (int c = 0; c < 8; ++c) {
+                f0[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+                f1[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (4 * c < cnt) {
+                  f0[c] = ld_shared_cluster_f4(a0 + 16u * c);
+                  f1[c] = ld_shared_cluster_f4(a1 + 16u * c);
+                }
+              }
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              v[4 * c] += f[c].x;
-              v[4 * c + 1] += f[c].y;
-              v[4 * c + 2] += f[c].z;
-              v[4 * c + 3] += f[c].w;
+              for (int c = 0; c < 8; ++c) {
+                v[4 * c] = (v[4 * c] + f0[c].x) + f1[c].x;
+                v[4 * c + 1] = (v[4 * c + 1] + f0[c].y) + f1[c].y;
+                v[4 * c + 2] = (v[4 * c + 2] + f0[c].z) + f1[c].z;
+                v[4 * c + 3] = (v[4 * c + 3] + f0[c].w) + f1[c].w;
+              }
             }
-          }
-          if (cc + 32 >= p.mma_n) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar(buf));
-          }
-          // residual column n of rows m: one coalesced 32-lane load per row, issued up front
-          float rr[32];
-          if (has_res) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int mm = m_tile0 + cc + j;
-              rr[j] = (n_ok && mm < p.M) ? load_elem(p.residual, (long long)mm * p.ldr + n, p.res_dtype) : 0.0f;
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int mm = m_tile0 + cc + j;
-            if (mm >= p.M) continue;  // uniform across the warp
-            float x = v[j];
-            if (has_bias) x += (p.bias_axis == 0) ? bias_n : load_elem(p.bias, mm, p.bias_dtype);
-            if (has_aux) {
-              const uint32_t word = __ballot_sync(0xffffffffu, n_ok && x > 0.0f);
-              const int w = (ta * 128 + q * 32) >> 5;
-              if (lane == 0 && (long long)w * 32 < p.N) p.aux[(long long)mm * p.ld_aux + w] = word;
-            }
-            float y = activate<ACT>(x, 0.0f);
-            if (has_res) y += rr[j];
-            y *= scale;
-            if (n_ok) store_elem<OUT>(p.out, (long long)mm * p.ldo + n, y);
+            swap_finish<ACT, OUT>(p, v, ta * 128 + row, ta * 128 + (int)rank * L + g * 32, m_tile0 + mc,
+                                  min(cnt, p.M - (m_tile0 + mc)), lane);
           }
         }
-        if (S > 1) {
-          // the leader has read every peer's partial: release them
-          for (int rk = 1; rk < S; ++rk) mbar_arrive_remote(mapa_shared(red_done_bar, (uint32_t)rk));
-          break;
-        }
-        if (!ok) break;
+        // nobody leaves while a peer may still read its partial
+        __syncwarp();
+        if (lane == 0)
+          for (int rk = 0; rk < S; ++rk) mbar_arrive_remote(mapa_shared(red_done_bar, (uint32_t)rk));
+        if (!warp_wait_bounded(red_done_bar, 0, p, lane, true)) ok = false;
+        break;  // a split-K cluster owns exactly one tile
       }
     }
     (void)ok;
+    __syncwarp();
   }
 
   // ================================================================ teardown
+  // Every thread of every role arrives here converged, after its last TMEM
+  // read, MMA (drained) and copy; only then is TMEM released.
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
