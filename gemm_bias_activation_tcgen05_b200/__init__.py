@@ -8,7 +8,7 @@ without a B200.
 
 The entry points keep the C names: ``fl_plan``, ``fl_execute``, ``fl_free``,
 ``fl_relu_backward``, ``fl_check_status``, ``fl_get_plan_info``,
-``fl_last_error``, ``fl_set_wait_limit_ns``.  ``Plan`` is a small owner of one
+``fl_last_error``, ``fl_set_wait_limit_ns``, ``fl_execute_noalloc``.  ``Plan`` is a small owner of one
 plan handle (the cuBLASLt epilog page's Matmul → plan → execute → free).
 """
 from __future__ import annotations
@@ -33,7 +33,7 @@ DTYPES = {"f16": FL_F16, "bf16": FL_BF16, "f32": FL_F32}
 COMPUTES = {"32F": FL_COMPUTE_32F, "32F_3XTF32": FL_COMPUTE_32F_3XTF32}
 
 EXPORTED = ["fl_plan", "fl_execute", "fl_relu_backward", "fl_check_status", "fl_get_plan_info",
-            "fl_free", "fl_last_error", "fl_set_wait_limit_ns"]
+            "fl_free", "fl_last_error", "fl_set_wait_limit_ns", "fl_execute_noalloc"]
 
 
 class fl_epilogue_desc(ctypes.Structure):
@@ -74,6 +74,9 @@ def _load() -> ctypes.CDLL:
     lib.fl_last_error.restype = ctypes.c_char_p
     lib.fl_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.fl_set_wait_limit_ns.restype = i32
+    lib.fl_execute_noalloc.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(fl_epilogue_desc),
+                                       vp, vp, vp, vp, vp, vp, vp]
+    lib.fl_execute_noalloc.restype = i32
     return lib
 
 
@@ -147,6 +150,15 @@ def fl_plan(M: int, N: int, K: int, dtype: str, compute: str, epi: fl_epilogue_d
 def fl_execute(plan: int, A, W, bias=None, aux=None, residual=None, out=None, stream=None) -> None:
     _check(LIB.fl_execute(plan, _ptr(A), _ptr(W), _ptr(bias), _ptr(aux), _ptr(residual), _ptr(out),
                           _stream(stream)), "fl_execute")
+
+
+def fl_execute_noalloc(M: int, N: int, K: int, dtype: str, compute: str, epi: fl_epilogue_desc, A, W, bias=None,
+                       aux=None, residual=None, out=None, stream=None) -> None:
+    """One layer without device allocation: scratch comes from the library's fixed
+    device array (for callers that cannot allocate; see the header)."""
+    _check(LIB.fl_execute_noalloc(int(M), int(N), int(K), DTYPES[dtype], COMPUTES[compute], ctypes.byref(epi),
+                                  _ptr(A), _ptr(W), _ptr(bias), _ptr(aux), _ptr(residual), _ptr(out),
+                                  _stream(stream)), "fl_execute_noalloc")
 
 
 def fl_relu_backward(grad, aux, dpre, M: int, N: int, dtype: str, ld_grad: int = 0, ld_dpre: int = 0,

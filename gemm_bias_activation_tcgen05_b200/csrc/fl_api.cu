@@ -763,3 +763,133 @@ extern "C" fl_status fl_check_status(fl_plan_t p, void* stream_) {
   }
   return FL_OK;
 }
+
+// ------------------------------------------------------------------ entry point without allocation
+// For callers that must not allocate device memory: a host that hands all GPU
+// memory to its own pool (an allocation outside it could fragment the pool or
+// fail under memory pressure), or a latency-critical path on which cudaMalloc
+// and cudaFree are forbidden because they can synchronise the device.  Such a
+// caller passes inputs and outputs as usual; the scratch that the planned path
+// allocates (the device error word, and the intermediate of the unfused path)
+// comes from the fixed array below, which every GPU that loads this library
+// holds until the process exits.
+static constexpr size_t kNoallocHeadBytes = 256;               // device error word
+static constexpr size_t kNoallocTmpBytes = size_t(32) << 20;   // unfused intermediate, at most 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocHeadBytes + kNoallocTmpBytes];
+
+static constexpr int kMaxDevices = 64;
+static void* g_noalloc_ptr[kMaxDevices] = {};
+static std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on `dev`, looked up once per device with
+// that device current (in host code the array's name is only a stand-in).
+static fl_status noalloc_scratch(int dev, unsigned char** out) {
+  if (dev < 0 || dev >= kMaxDevices) return fail(FL_ERR_DEVICE, "fl_execute_noalloc: device %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || ptr == nullptr)
+      return fail(FL_ERR_CUDA, "fl_execute_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = static_cast<unsigned char*>(g_noalloc_ptr[dev]);
+  return FL_OK;
+}
+
+extern "C" fl_status fl_execute_noalloc(int64_t M, int64_t N, int64_t K, int32_t dtype, int32_t compute,
+                                        const fl_epilogue_desc* epi, const void* A, const void* W,
+                                        const void* bias, uint32_t* aux, const void* residual, void* out,
+                                        void* stream_) {
+  g_err[0] = 0;
+  const char* who = "fl_execute_noalloc";
+  if (!epi) return fail(FL_ERR_INVALID_ARG, "%s: null epilogue descriptor", who);
+  if (M < 1 || N < 1 || K < 0) return fail(FL_ERR_INVALID_ARG, "%s: need M>=1, N>=1, K>=0", who);
+  if (M > (1LL << 31) - 256 || N > (1LL << 30) || K > (1LL << 31) - 256)
+    return fail(FL_ERR_INVALID_ARG, "%s: dimension too large", who);
+  if (epi->kind < FL_EPI_NONE || epi->kind > FL_EPI_GEGLU_TANH)
+    return fail(FL_ERR_INVALID_ARG, "%s: unknown epilogue kind %d", who, epi->kind);
+  for (int i = 0; i < 3; ++i)
+    if (epi->reserved[i] != 0) return fail(FL_ERR_INVALID_ARG, "%s: reserved fields must be 0", who);
+  if (dtype != FL_F16 && dtype != FL_BF16) {
+    if (dtype == FL_F32) return fail(FL_ERR_UNSUPPORTED, "%s: fp32 operands are not offered", who);
+    return fail(FL_ERR_INVALID_ARG, "%s: unknown dtype %d", who, dtype);
+  }
+  if (compute != FL_COMPUTE_32F) return fail(FL_ERR_UNSUPPORTED, "%s: compute type %d not offered", who, compute);
+  if (epi->out_dtype < FL_F16 || epi->out_dtype > FL_F32)
+    return fail(FL_ERR_INVALID_ARG, "%s: unknown out_dtype %d", who, epi->out_dtype);
+  const bool has_bias = epi->kind != FL_EPI_NONE && epi->kind != FL_EPI_GEGLU_TANH;
+  if (has_bias && (epi->bias_dtype < FL_F16 || epi->bias_dtype > FL_F32))
+    return fail(FL_ERR_INVALID_ARG, "%s: unknown bias_dtype %d", who, epi->bias_dtype);
+  if (epi->has_residual && (epi->residual_dtype < FL_F16 || epi->residual_dtype > FL_F32))
+    return fail(FL_ERR_INVALID_ARG, "%s: unknown residual_dtype %d", who, epi->residual_dtype);
+  if ((epi->bias_axis != 0 && epi->bias_axis != 1) || (epi->b_major != 0 && epi->b_major != 1))
+    return fail(FL_ERR_INVALID_ARG, "%s: bias_axis and b_major must be 0 or 1", who);
+  if (epi->kind == FL_EPI_GEGLU_TANH && (epi->b_major || epi->out_dtype == FL_F32))
+    return fail(FL_ERR_UNSUPPORTED, "%s: GEGLU_TANH takes the stacked [2N,K] weight and writes f16/bf16", who);
+  if (epi->lda < 0 || epi->ldb < 0 || epi->ldo < 0 || epi->ldr < 0)
+    return fail(FL_ERR_INVALID_ARG, "%s: negative leading dimension", who);
+
+  // A plan on the host stack: the same configuration choice as fl_plan, but its
+  // scratch points into the fixed array instead of fresh allocations.
+  fl_plan_s p{};
+  p.M = M; p.N = N; p.K = K; p.dtype = dtype; p.compute = compute; p.epi = *epi;
+  if (p.epi.scale == 0.0f) p.epi.scale = 1.0f;
+  p.act = act_of(epi->kind);
+  p.has_bias = has_bias;
+  p.has_aux = epi->kind == FL_EPI_RELU_AUX_BIAS;
+  const int64_t a_cols = K, b_cols = epi->b_major ? N : K;
+  if (p.epi.lda == 0) p.epi.lda = a_cols;
+  if (p.epi.ldb == 0) p.epi.ldb = b_cols;
+  if (p.epi.ldo == 0) p.epi.ldo = N;
+  if (p.epi.ldr == 0) p.epi.ldr = N;
+  if (p.epi.lda < a_cols || p.epi.ldb < b_cols || p.epi.ldo < N || (epi->has_residual && p.epi.ldr < N))
+    return fail(FL_ERR_INVALID_ARG, "%s: leading dimension smaller than the row length", who);
+  const int es = esize(dtype), eo = esize(epi->out_dtype);
+  if ((p.epi.lda * es) % 16 || (p.epi.ldb * es) % 16 || (p.epi.ldo * eo) % 16 ||
+      (epi->has_residual && (p.epi.ldr * esize(epi->residual_dtype)) % 16))
+    return fail(FL_ERR_ALIGNMENT, "%s: every row pitch must be a multiple of 16 bytes", who);
+  if (cudaGetDevice(&p.device) != cudaSuccess) return fail(FL_ERR_DEVICE, "%s: no CUDA device", who);
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, p.device) != cudaSuccess || major != 10)
+    return fail(FL_ERR_DEVICE, "%s: needs an sm_100 (B200-class) GPU", who);
+  FL_CUDA(cudaDeviceGetAttribute(&p.num_sms, cudaDevAttrMultiProcessorCount, p.device));
+  FL_CUDA(cudaDeviceGetAttribute(&p.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, p.device));
+  fl_status st = get_encode();
+  if (st != FL_OK) return st;
+
+  choose_config(&p);
+  const int b_boxes = epi->b_major ? p.mma_n / 64 : (epi->kind == FL_EPI_GEGLU_TANH ? 2 : 1);
+  Layout L = layout_for(&p, p.mma_n, b_boxes, p.max_smem);
+  if (L.stages < 2) return fail(FL_ERR_UNSUPPORTED, "%s: shared memory too small", who);
+  p.stages = L.stages;
+  p.smem = (int)L.total;
+  const int tiles = p.tiles_a * p.tiles_b;
+  p.grid = (p.swap && p.split_k > 1) ? tiles * p.split_k : std::min(tiles, p.num_sms);
+  p.kernel = pick_kernel(p.act, epi->out_dtype, p.swap);
+  if (!p.kernel) return fail(FL_ERR_UNSUPPORTED, "%s: no kernel for this combination", who);
+  FL_CUDA(cudaFuncSetAttribute(p.kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, p.max_smem));
+  p.launches = 1;
+  p.wait_limit_ns = g_wait_limit_ns;
+
+  unsigned char* scratch = nullptr;
+  st = noalloc_scratch(p.device, &scratch);
+  if (st != FL_OK) return st;
+  p.d_err = reinterpret_cast<int*>(scratch);
+  if (epi->unfused) {
+    const int64_t cols = (epi->kind == FL_EPI_GEGLU_TANH) ? 2 * N : N;
+    p.tmp_ld = cdiv(cols * eo, 16) * 16 / eo;
+    const double need = (double)M * (double)p.tmp_ld * (double)eo;
+    if (need > (double)kNoallocTmpBytes)
+      return fail(FL_ERR_INVALID_ARG, "%s: the unfused intermediate needs %.0f bytes, above the %zu-byte scratch", who,
+                  need, kNoallocTmpBytes);
+    p.tmp_bytes = (size_t)need;
+    p.d_tmp = scratch + kNoallocHeadBytes;
+    for (int sw = 0; sw < 2; ++sw)
+      FL_CUDA(cudaFuncSetAttribute(pick_kernel(ACT_NONE, epi->out_dtype, sw == 1),
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, p.max_smem));
+  }
+  // the error word must start at zero; the intermediate is fully overwritten
+  FL_CUDA(cudaMemsetAsync(p.d_err, 0, sizeof(int), reinterpret_cast<cudaStream_t>(stream_)));
+  return fl_execute(&p, A, W, bias, aux, residual, out, stream_);
+}

@@ -164,6 +164,30 @@ fl_status fl_free(fl_plan_t plan);
 /* Thread-local text of the last failure on this thread ("" if none). */
 const char* fl_last_error(void);
 
+/* One fused linear layer without any device allocation (the pages have no
+ * counterpart of this call).  For callers that cannot call cudaMalloc: a host
+ * that owns all device memory through its own pool, or a latency-critical path
+ * on which cudaMalloc/cudaFree are forbidden because they can synchronise the
+ * device.  It takes fl_plan's arguments and fl_execute's operands in one call
+ * and runs the same kernels; the scratch that a plan would allocate comes from
+ * one fixed 32 MiB + 256 B device array inside this library (the device error
+ * word, and the intermediate of an unfused call, which must fit in 32 MiB:
+ * M × (N, or 2N for GEGLU_TANH, rounded up to 16 bytes) × out_dtype size;
+ * larger sizes return FL_ERR_INVALID_ARG).  Every GPU that loads the library
+ * holds the array until the process exits.
+ *   - The first call on a device looks up the array's device address with that
+ *     device current; make that first call before any stream capture.
+ *   - All calls on a device share the array: calls that overlap on the GPU (on
+ *     different streams, or from different threads) race on it.
+ *   - The error word is cleared at each call and not read back: a bounded
+ *     in-kernel wait that gives up is not reported by this entry point.
+ *   - fp16/bf16 operands with FL_COMPUTE_32F only.
+ * Errors: as fl_plan and fl_execute. */
+fl_status fl_execute_noalloc(int64_t M, int64_t N, int64_t K, int32_t dtype, int32_t compute,
+                             const fl_epilogue_desc* epi, const void* A, const void* W,
+                             const void* bias, uint32_t* aux, const void* residual, void* out,
+                             void* stream);
+
 /* Override the bound on every in-kernel wait for plans created afterwards
  * (nanoseconds; 0 restores the default of 2 s).  Test/debug use. */
 fl_status fl_set_wait_limit_ns(uint64_t ns);
