@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of a captured graph")
+    ap.add_argument("--profile", default=None, metavar="WORKLOAD",
+                    help="run only this workload's launches (warm-up + steps), print nothing; for ncu captures")
     return ap.parse_args()
 
 
@@ -248,20 +251,38 @@ def run_ours(args):
     torch.cuda.synchronize()
     suite.check()
 
-    # ---- timed region: K steps, per-launch events on the launching stream
+    # ---- timed region: K steps, per-launch events on the launching stream.  The K
+    # steps are captured once as a CUDA graph (launches + event-record nodes), so
+    # the timed replay has no host enqueue gaps between the launches.
     n_items = len(suite.items)
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_items)]
+    use_graph = not args.no_graph
+    ev = [[(torch.cuda.Event(enable_timing=True, external=use_graph),
+            torch.cuda.Event(enable_timing=True, external=use_graph)) for _ in range(n_items)]
           for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def k_steps(stream_handle):
+        for s in range(args.steps):
+            for i, it in enumerate(suite.items):
+                ev[s][i][0].record()
+                suite.run_item(it, stream_handle)
+                ev[s][i][1].record()
+
+    graph = None
+    if use_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            k_steps(torch.cuda.current_stream().cuda_stream)
+        graph.replay()  # one untimed replay of the captured steps
+        torch.cuda.synchronize()
     barrier(ws)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         t0.record(stream)
-        for s in range(args.steps):
-            for i, it in enumerate(suite.items):
-                ev[s][i][0].record(stream)
-                suite.run_item(it, sh)
-                ev[s][i][1].record(stream)
+        if graph is not None:
+            graph.replay()
+        else:
+            k_steps(sh)
         t1.record(stream)
         torch.cuda.synchronize()
     barrier(ws)
@@ -306,6 +327,7 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": "all synthetic workloads of the fused linear layer, one fused launch each: "
                                + ", ".join(it["w"].name for it in suite.items),
+                   "timed_as": "one CUDA graph of the K steps" if use_graph else "eager launches",
                    "flops_per_step": suite.flops, "parallelism": f"replicas x{ws}",
                    "l2": "inputs larger than L2: every workload owns its operands; a step touches "
                          f"{sum(suite.min_bytes.values()) / 1e6:.0f} MB"},
@@ -322,6 +344,8 @@ def run_ours(args):
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
+    del graph
+    torch.cuda.synchronize()
     for it in suite.items:
         for p in it["plans"]:
             p.free()
@@ -490,8 +514,30 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile(args):
+    """Launch one workload warm-up + steps times and exit: a small, fixed program for ncu."""
+    import torch
+    import gemm_bias_activation_tcgen05_b200 as fl
+    torch.cuda.set_device(0)
+    global SUITE
+    SUITE = [args.profile]
+    suite = Suite(fl, seed=0)
+    sh = torch.cuda.current_stream().cuda_stream
+    for _ in range(args.warmup + args.steps):
+        for it in suite.items:
+            suite.run_item(it, sh)
+    torch.cuda.synchronize()
+    suite.check()
+    for it in suite.items:
+        for p in it["plans"]:
+            p.free()
+
+
 def main():
     args = parse()
+    if args.profile:
+        run_profile(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

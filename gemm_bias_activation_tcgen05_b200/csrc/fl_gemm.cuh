@@ -238,6 +238,38 @@ __device__ __forceinline__ void load_row_chunk(float (&dst)[CH], const void* bas
   }
 }
 
+// Eight read-only loads base[i0], base[i0+stride], ... issued by one asm
+// statement, so all eight are in flight before any result is used.  Every
+// address must be valid (callers clamp the row index).
+__device__ __forceinline__ void ldg8(float (&dst)[8], const void* base, long long i0, long long stride, int dt) {
+  if (dt == DT_F32) {
+    const float* b = reinterpret_cast<const float*>(base) + i0;
+    asm volatile(
+        "ld.global.nc.f32 %0, [%8];\n\tld.global.nc.f32 %1, [%9];\n\tld.global.nc.f32 %2, [%10];\n\t"
+        "ld.global.nc.f32 %3, [%11];\n\tld.global.nc.f32 %4, [%12];\n\tld.global.nc.f32 %5, [%13];\n\t"
+        "ld.global.nc.f32 %6, [%14];\n\tld.global.nc.f32 %7, [%15];"
+        : "=f"(dst[0]), "=f"(dst[1]), "=f"(dst[2]), "=f"(dst[3]), "=f"(dst[4]), "=f"(dst[5]), "=f"(dst[6]),
+          "=f"(dst[7])
+        : "l"(b), "l"(b + stride), "l"(b + 2 * stride), "l"(b + 3 * stride), "l"(b + 4 * stride),
+          "l"(b + 5 * stride), "l"(b + 6 * stride), "l"(b + 7 * stride)
+        : "memory");
+    return;
+  }
+  const uint16_t* b = reinterpret_cast<const uint16_t*>(base) + i0;
+  unsigned short h[8];
+  asm volatile(
+      "ld.global.nc.u16 %0, [%8];\n\tld.global.nc.u16 %1, [%9];\n\tld.global.nc.u16 %2, [%10];\n\t"
+      "ld.global.nc.u16 %3, [%11];\n\tld.global.nc.u16 %4, [%12];\n\tld.global.nc.u16 %5, [%13];\n\t"
+      "ld.global.nc.u16 %6, [%14];\n\tld.global.nc.u16 %7, [%15];"
+      : "=h"(h[0]), "=h"(h[1]), "=h"(h[2]), "=h"(h[3]), "=h"(h[4]), "=h"(h[5]), "=h"(h[6]), "=h"(h[7])
+      : "l"(b), "l"(b + stride), "l"(b + 2 * stride), "l"(b + 3 * stride), "l"(b + 4 * stride),
+        "l"(b + 5 * stride), "l"(b + 6 * stride), "l"(b + 7 * stride)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    dst[i] = (dt == DT_BF16) ? __uint_as_float(static_cast<uint32_t>(h[i]) << 16) : __half2float(__ushort_as_half(h[i]));
+}
+
 // Epilogue of the swap-AB layout for one thread: output column n, rows
 // m0 .. m0+cnt-1 with pre-activations v[0..cnt).  The warp's 32 lanes hold 32
 // consecutive columns starting at n_warp0 (a multiple of 32), so every row's
@@ -252,10 +284,25 @@ __device__ __forceinline__ void swap_finish(const KParams& p, const float (&v)[3
   float rr[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) rr[j] = 0.0f;
-  if (has_res && n_ok) {
+  if (has_res && n_ok && cnt > 0) {
+    // eight rows per batch; rows past M re-read row M-1 (valid memory, result unused)
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (j < cnt) rr[j] = ldg_pinned(p.residual, (long long)(m0 + j) * p.ldr + n, p.res_dtype);
+    for (int g = 0; g < 4; ++g) {
+      if (8 * g < cnt) {
+        float t[8];
+        if (8 * g + 8 <= cnt) {
+          ldg8(t, p.residual, (long long)(m0 + 8 * g) * p.ldr + n, p.ldr, p.res_dtype);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int mm = min(m0 + 8 * g + i, p.M - 1);
+            t[i] = ldg_pinned(p.residual, (long long)mm * p.ldr + n, p.res_dtype);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) rr[8 * g + i] = t[i];
+      }
+    }
   }
   float bias_n = 0.0f;
   if (has_bias && p.bias_axis == 0 && n_ok) bias_n = ldg_pinned(p.bias, n, p.bias_dtype);
@@ -659,30 +706,32 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           const uint32_t row_addr = red_base + (uint32_t)row * p.red_pitch;
           for (int mc = mb; mc < mb + mcnt; mc += 32) {
             const int cnt = min(32, mb + mcnt - mc);
-            // sum the S partials in rank order, two ranks' loads in flight at a time
+            // every rank's loads in flight together, then the sum in rank order
             float v[32];
+            float4 f[4][8];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-            for (int rk = 0; rk < S; rk += 2) {
-              float4 f0[8], f1[8];
-              const uint32_t a0 = mapa_shared(row_addr + (uint32_t)mc * 4u, (uint32_t)rk);
-              const uint32_t a1 = mapa_shared(row_addr + (uint32_t)mc * 4u, (uint32_t)(rk + 1));
+            for (int rk = 0; rk < 4; ++rk) {
+              const uint32_t a = mapa_shared(row_addr + (uint32_t)mc * 4u, (uint32_t)(rk < S ? rk : 0));
 #pragma unroll
               for (int c = 0; c < 8; ++c) {
-                f0[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-                f1[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (4 * c < cnt) {
-                  f0[c] = ld_shared_cluster_f4(a0 + 16u * c);
-                  f1[c] = ld_shared_cluster_f4(a1 + 16u * c);
-                }
+                f[rk][c] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (rk < S && 4 * c < cnt) f[rk][c] = ld_shared_cluster_f4(a + 16u * c);
               }
+            }
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                v[4 * c] = (v[4 * c] + f0[c].x) + f1[c].x;
-                v[4 * c + 1] = (v[4 * c + 1] + f0[c].y) + f1[c].y;
-                v[4 * c + 2] = (v[4 * c + 2] + f0[c].z) + f1[c].z;
-                v[4 * c + 3] = (v[4 * c + 3] + f0[c].w) + f1[c].w;
+            for (int c = 0; c < 8; ++c) {
+              float4 acc = f[0][c];
+#pragma unroll
+              for (int rk = 1; rk < 4; ++rk) {
+                acc.x += f[rk][c].x;
+                acc.y += f[rk][c].y;
+                acc.z += f[rk][c].z;
+                acc.w += f[rk][c].w;
               }
+              v[4 * c] = acc.x;
+              v[4 * c + 1] = acc.y;
+              v[4 * c + 2] = acc.z;
+              v[4 * c + 3] = acc.w;
             }
             swap_finish<ACT, OUT>(p, v, ta * 128 + row, ta * 128 + (int)rank * L + g * 32, m_tile0 + mc,
                                   min(cnt, p.M - (m_tile0 + mc)), lane);
