@@ -48,7 +48,8 @@ class fl_plan_info(ctypes.Structure):
     _fields_ = [("tile_m", ctypes.c_int32), ("tile_n", ctypes.c_int32), ("mma_n", ctypes.c_int32),
                 ("swap_ab", ctypes.c_int32), ("split_k", ctypes.c_int32), ("stages", ctypes.c_int32),
                 ("grid", ctypes.c_int32), ("smem_bytes", ctypes.c_int32),
-                ("launches_per_execute", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
+                ("launches_per_execute", ctypes.c_int32), ("cta_pair", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 6)]
 
 
 def _load() -> ctypes.CDLL:

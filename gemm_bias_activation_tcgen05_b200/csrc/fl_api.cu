@@ -115,11 +115,43 @@ static const void* pick_swap(bool swap) {
   return swap ? reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, OUT, true>)
               : reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, OUT, false>);
 }
+// fp32 operands (3xTF32): normal layout only
+template <int ACT>
+static const void* pick_tf32(int out) {
+  if (out == FL_BF16) return reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, DT_BF16, false, true>);
+  if (out == FL_F16) return reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, DT_F16, false, true>);
+  return reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, DT_F32, false, true>);
+}
+static const void* pick_kernel_tf32(int act, int out) {
+  switch (act) {
+    case ACT_NONE: return pick_tf32<ACT_NONE>(out);
+    case ACT_RELU: return pick_tf32<ACT_RELU>(out);
+    case ACT_GELU: return pick_tf32<ACT_GELU>(out);
+    case ACT_GELU_TANH: return pick_tf32<ACT_GELU_TANH>(out);
+    default: return nullptr;
+  }
+}
 template <int ACT>
 static const void* pick_out(int out, bool swap) {
   if (out == FL_BF16) return pick_swap<ACT, DT_BF16>(swap);
   if (out == FL_F16) return pick_swap<ACT, DT_F16>(swap);
   return pick_swap<ACT, DT_F32>(swap);
+}
+// CTA-pair (256-row UMMA) kernels: normal layout, 16-bit operands
+template <int ACT>
+static const void* pick_pair(int out) {
+  if (out == FL_BF16) return reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, DT_BF16, false, false, true>);
+  if (out == FL_F16) return reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, DT_F16, false, false, true>);
+  return reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, DT_F32, false, false, true>);
+}
+static const void* pick_kernel_pair(int act, int out) {
+  switch (act) {
+    case ACT_NONE: return pick_pair<ACT_NONE>(out);
+    case ACT_RELU: return pick_pair<ACT_RELU>(out);
+    case ACT_GELU: return pick_pair<ACT_GELU>(out);
+    case ACT_GELU_TANH: return pick_pair<ACT_GELU_TANH>(out);
+    default: return pick_pair<ACT_GEGLU>(out);
+  }
 }
 static const void* pick_kernel(int act, int out, bool swap) {
   switch (act) {
@@ -150,6 +182,7 @@ struct fl_plan_s {
   int device, num_sms, max_smem;
   // configuration
   bool swap;
+  bool pair;  // two CTAs share one 256-row UMMA tile (cluster of 2)
   int mma_n, out_tile_n, split_k, stages, grid, smem;
   int tiles_a, tiles_b, num_kb;
   const void* kernel;
@@ -180,7 +213,7 @@ static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // layout) the epilogue staging buffers and per-warp bias rows, then (split-K)
 // the reduction buffer, then the barriers.
 struct Layout {
-  uint32_t a_stage, b_box, b_stage, stage, staging_off, bias_off, bar_off, red_off, red_pitch, total;
+  uint32_t a_stage, b_box, b_stage, stage, stride, staging_off, bias_off, bar_off, red_off, red_pitch, total;
   int stages;
 };
 
@@ -188,26 +221,48 @@ static Layout layout_for(const fl_plan_s* p, int mma_n, int b_boxes, int max_sme
   Layout L{};
   const int es = esize(p->dtype);
   const int bk = 128 / es;
+  const int rows_b = p->pair ? mma_n / 2 : mma_n;  // B rows (or columns) held by one CTA
   L.a_stage = 128u * 128u;  // 128 rows x 128 bytes
   if (p->epi.b_major) L.b_box = 64u * (uint32_t)bk * (uint32_t)es;  // 64 columns x bk rows
-  else L.b_box = (uint32_t)(mma_n / b_boxes) * 128u;
+  else L.b_box = (uint32_t)(rows_b / b_boxes) * 128u;
   L.b_stage = L.b_box * (uint32_t)b_boxes;
   L.stage = L.a_stage + L.b_stage;
+  // fp32 operands: each stage also holds the TF32 lo halves of both tiles
+  L.stride = (p->dtype == FL_F32) ? 2u * L.stage : L.stage;
   const uint32_t staging = p->swap ? Cfg<true>::kStagingBytes : Cfg<false>::kStagingBytes;
   const uint32_t bias = 0;
   const uint32_t red = (p->swap && p->split_k > 1) ? 128u * ((uint32_t)mma_n * 4u + 16u) : 0u;
-  const uint32_t bars = 8u * (2u * 8u + 8u);
+  const uint32_t bars = 8u * (3u * 8u + 8u);
   const uint32_t budget = (uint32_t)max_smem - 1024u - staging - bias - red - bars;
-  int st = (int)(budget / L.stage);
+  int st = (int)(budget / L.stride);
   if (st > 8) st = 8;
   L.stages = st;
-  L.staging_off = (uint32_t)st * L.stage;
+  L.staging_off = (uint32_t)st * L.stride;
   L.bias_off = L.staging_off + staging;
   L.red_off = L.bias_off + bias;
   L.red_pitch = (uint32_t)mma_n * 4u + 16u;
   L.bar_off = L.red_off + red;
-  L.total = L.bar_off + 8u * (2u * (uint32_t)st + 8u) + 1024u;
+  L.total = L.bar_off + 8u * (3u * (uint32_t)st + 8u) + 1024u;
   return L;
+}
+
+// TMA boxes of operand B per stage and CTA.
+static int b_boxes_of(const fl_plan_s* p, bool geglu) {
+  const int rows_b = p->pair ? p->mma_n / 2 : p->mma_n;
+  if (p->epi.b_major) return rows_b / 64;
+  if (geglu) return p->pair ? 1 : 2;
+  return 1;
+}
+static int grid_of(const fl_plan_s* p) {
+  const int tiles = p->tiles_a * p->tiles_b;
+  if (p->swap && p->split_k > 1) return tiles * p->split_k;
+  if (p->pair) return 2 * std::min(tiles, p->num_sms / 2);
+  return std::min(tiles, p->num_sms);
+}
+static const void* kernel_of(const fl_plan_s* p, int act, int out) {
+  if (p->dtype == FL_F32) return pick_kernel_tf32(act, out);
+  if (p->pair) return pick_kernel_pair(act, out);
+  return pick_kernel(act, out, p->swap);
 }
 
 static fl_status choose_config(fl_plan_s* p) {
@@ -233,8 +288,15 @@ static fl_status choose_config(fl_plan_s* p) {
     p->split_k = S;
   } else {
     p->split_k = 1;
+    // 16-bit operands beyond one 128-row tile: CTA pairs with 256-row UMMA tiles
+    p->pair = p->dtype != FL_F32 && M > 128;
+    const int rows = p->pair ? 256 : 128;
+    const int units = p->pair ? p->num_sms / 2 : p->num_sms;
     if (geglu) {
       p->mma_n = 256;
+      p->out_tile_n = 128;
+    } else if (p->dtype == FL_F32) {
+      p->mma_n = 128;  // a 3xTF32 stage holds hi and lo tiles: 128 wide keeps three stages
       p->out_tile_n = 128;
     } else {
       // Pick the N tile that minimises (waves x tile width) on this GPU.
@@ -244,15 +306,15 @@ static fl_status choose_config(fl_plan_s* p) {
       int best = 256;
       double best_cost = 1e300;
       for (int bn : {256, 128}) {
-        const int64_t tiles = cdiv(M, 128) * cdiv(N, bn);
-        const double waves = (double)cdiv(tiles, p->num_sms);
+        const int64_t tiles = cdiv(M, rows) * cdiv(N, bn);
+        const double waves = (double)cdiv(tiles, units);
         const double cost = waves * bn * (bn == 128 ? 1.6 : 1.0);
         if (cost < best_cost) { best_cost = cost; best = bn; }
       }
       p->mma_n = best;
       p->out_tile_n = best;
     }
-    p->tiles_a = (int)cdiv(M, 128);
+    p->tiles_a = (int)cdiv(M, rows);
     p->tiles_b = (int)cdiv(N, p->out_tile_n);
   }
   return FL_OK;
@@ -277,8 +339,8 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
     return fail(FL_ERR_UNSUPPORTED, "fl_plan: compute type %d not offered (only FP32 accumulation)", compute);
   if ((compute == FL_COMPUTE_32F) != (dtype != FL_F32))
     return fail(FL_ERR_UNSUPPORTED, "fl_plan: FL_COMPUTE_32F takes f16/bf16 operands, 3XTF32 takes f32");
-  if (dtype == FL_F32)
-    return fail(FL_ERR_UNSUPPORTED, "fl_plan: the 3xTF32 path is not built yet");
+  if (dtype == FL_F32 && (epi->b_major || epi->kind == FL_EPI_GEGLU_TANH))
+    return fail(FL_ERR_UNSUPPORTED, "fl_plan: fp32 operands take a K-contiguous W and no GeGLU");
   if (epi->out_dtype < FL_F16 || epi->out_dtype > FL_F32)
     return fail(FL_ERR_INVALID_ARG, "fl_plan: unknown out_dtype %d", epi->out_dtype);
   const bool has_bias = epi->kind != FL_EPI_NONE && epi->kind != FL_EPI_GEGLU_TANH;
@@ -336,15 +398,13 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
   if (st != FL_OK) { delete p; return st; }
 
   choose_config(p);
-  const int b_boxes = epi->b_major ? p->mma_n / 64 : (p->epi.kind == FL_EPI_GEGLU_TANH ? 2 : 1);
+  const int b_boxes = b_boxes_of(p, p->epi.kind == FL_EPI_GEGLU_TANH);
   Layout L = layout_for(p, p->mma_n, b_boxes, p->max_smem);
   if (L.stages < 2) { delete p; return fail(FL_ERR_UNSUPPORTED, "fl_plan: shared memory too small"); }
   p->stages = L.stages;
   p->smem = (int)L.total;
-  const int tiles = p->tiles_a * p->tiles_b;
-  if (p->swap && p->split_k > 1) p->grid = tiles * p->split_k;
-  else p->grid = std::min(tiles, p->num_sms);
-  p->kernel = pick_kernel(p->act, epi->out_dtype, p->swap);
+  p->grid = grid_of(p);
+  p->kernel = kernel_of(p, p->act, epi->out_dtype);
   if (!p->kernel) { delete p; return fail(FL_ERR_UNSUPPORTED, "fl_plan: no kernel for this combination"); }
   // Every plan sharing a kernel may need a different amount of dynamic shared
   // memory, so the kernel's bound is the device maximum, not this plan's size.
@@ -364,8 +424,10 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
   p->wait_limit_ns = g_wait_limit_ns;
   if (epi->unfused) {
     // the bare GEMM kernels of both layouts may serve this plan's first step
-    for (int sw = 0; sw < 2; ++sw) {
-      const void* kn = pick_kernel(ACT_NONE, epi->out_dtype, sw == 1);
+    for (int sw = 0; sw < 3; ++sw) {
+      const void* kn = (dtype == FL_F32) ? pick_kernel_tf32(ACT_NONE, epi->out_dtype)
+                       : (sw == 2 ? pick_kernel_pair(ACT_NONE, epi->out_dtype)
+                                  : pick_kernel(ACT_NONE, epi->out_dtype, sw == 1));
       if (cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, p->max_smem) != cudaSuccess) {
         cudaFree(p->d_err);
         delete p;
@@ -395,7 +457,7 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
 extern "C" fl_status fl_get_plan_info(fl_plan_t p, fl_plan_info* info) {
   if (!p || !info) return fail(FL_ERR_INVALID_ARG, "fl_get_plan_info: null argument");
   memset(info, 0, sizeof(*info));
-  info->tile_m = p->swap ? p->mma_n : 128;
+  info->tile_m = p->swap ? p->mma_n : (p->pair ? 256 : 128);
   info->tile_n = p->swap ? 128 : p->out_tile_n;
   info->mma_n = p->mma_n;
   info->swap_ab = p->swap ? 1 : 0;
@@ -404,6 +466,7 @@ extern "C" fl_status fl_get_plan_info(fl_plan_t p, fl_plan_info* info) {
   info->grid = p->grid;
   info->smem_bytes = p->smem;
   info->launches_per_execute = p->launches;
+  info->cta_pair = p->pair ? 1 : 0;
   return FL_OK;
 }
 
@@ -441,9 +504,9 @@ static fl_status launch_kernel(const fl_plan_s* p, const LaunchCache& c, cudaStr
   cfg.dynamicSmemBytes = (size_t)p->smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  if (p->split_k > 1) {
+  if (p->split_k > 1 || p->pair) {
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)p->split_k;
+    attr[0].val.clusterDim.x = p->pair ? 2u : (unsigned)p->split_k;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
@@ -475,24 +538,23 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
   k.bk = bk;
   k.b_mn_major = e.b_major;
   k.geglu = g.geglu_fused ? 1 : 0;
-  int b_boxes;
-  if (e.b_major) b_boxes = p->mma_n / 64;
-  else b_boxes = g.geglu_fused ? 2 : 1;
+  const int b_boxes = b_boxes_of(p, g.geglu_fused);
   Layout L = layout_for(p, p->mma_n, b_boxes, p->max_smem);
   k.num_stages = p->stages;
   k.b_boxes = b_boxes;
-  k.b_box_rows = e.b_major ? 64 : p->mma_n / b_boxes;
+  k.b_box_rows = e.b_major ? 64 : (p->pair ? p->mma_n / 2 : p->mma_n) / b_boxes;
   k.a_stage_bytes = L.a_stage;
   k.b_box_bytes = L.b_box;
   k.stage_bytes = L.stage;
+  k.stage_stride = L.stride;
   k.staging_off = L.staging_off;
   k.bias_off = L.bias_off;
   k.red_off = L.red_off;
   k.red_pitch = L.red_pitch;
   k.bar_off = L.bar_off;
-  const uint32_t fmt = (p->dtype == FL_BF16) ? 1u : 0u;
+  const uint32_t fmt = (p->dtype == FL_BF16) ? 1u : (p->dtype == FL_F32 ? 2u : 0u);  // F16 / BF16 / TF32
   k.idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(e.b_major ? 1 : 0) << 16) |
-            ((uint32_t)(p->mma_n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+            ((uint32_t)(p->mma_n >> 3) << 17) | ((uint32_t)((p->pair ? 256 : 128) >> 4) << 24);
   k.a_kstep = 32;
   k.b_kstep = e.b_major ? 16u * 128u : 32u;
   k.b_lbo = e.b_major ? L.b_box : 16u;
@@ -537,7 +599,7 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
       st = make_map(&tmB2, up, p->dtype, Kd, (uint64_t)p->N, (uint64_t)e.ldb * es, (uint32_t)bk, 128);
     } else {
       st = make_map(&tmB, g.W, p->dtype, Kd, (uint64_t)g.n_cols, (uint64_t)e.ldb * es, (uint32_t)bk,
-                    (uint32_t)p->mma_n);
+                    (uint32_t)(p->pair ? p->mma_n / 2 : p->mma_n));
     }
     if (st) return st;
     // The TMA store covers whole 16-byte granules of a row only; the kernel writes
@@ -633,13 +695,14 @@ extern "C" fl_status fl_execute(fl_plan_t p, const void* A, const void* W, const
     q.epi.kind = FL_EPI_NONE;
     q.N = cols;
     choose_config(&q);
-    const int b_boxes = e.b_major ? q.mma_n / 64 : 1;
+    const int b_boxes = b_boxes_of(&q, false);
     Layout L = layout_for(&q, q.mma_n, b_boxes, q.max_smem);
     q.stages = L.stages;
     q.smem = (int)L.total;
     const int tiles = q.tiles_a * q.tiles_b;
-    q.grid = (q.swap && q.split_k > 1) ? tiles * q.split_k : std::min(tiles, q.num_sms);
-    const void* kern = pick_kernel(ACT_NONE, odt, q.swap);
+    (void)tiles;
+    q.grid = grid_of(&q);
+    const void* kern = kernel_of(&q, ACT_NONE, odt);
     q.epi.ldr = 0;
     q.epi.has_residual = 0;
     GemmArgs g{A, W, gemm_out, odt, gemm_ld, ACT_NONE, nullptr, nullptr, nullptr, 1.0f, cols, false};
@@ -859,14 +922,15 @@ extern "C" fl_status fl_execute_noalloc(int64_t M, int64_t N, int64_t K, int32_t
   if (st != FL_OK) return st;
 
   choose_config(&p);
-  const int b_boxes = epi->b_major ? p.mma_n / 64 : (epi->kind == FL_EPI_GEGLU_TANH ? 2 : 1);
+  const int b_boxes = b_boxes_of(&p, epi->kind == FL_EPI_GEGLU_TANH);
   Layout L = layout_for(&p, p.mma_n, b_boxes, p.max_smem);
   if (L.stages < 2) return fail(FL_ERR_UNSUPPORTED, "%s: shared memory too small", who);
   p.stages = L.stages;
   p.smem = (int)L.total;
   const int tiles = p.tiles_a * p.tiles_b;
-  p.grid = (p.swap && p.split_k > 1) ? tiles * p.split_k : std::min(tiles, p.num_sms);
-  p.kernel = pick_kernel(p.act, epi->out_dtype, p.swap);
+  (void)tiles;
+  p.grid = grid_of(&p);
+  p.kernel = kernel_of(&p, p.act, epi->out_dtype);
   if (!p.kernel) return fail(FL_ERR_UNSUPPORTED, "%s: no kernel for this combination", who);
   FL_CUDA(cudaFuncSetAttribute(p.kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, p.max_smem));
   p.launches = 1;
@@ -885,8 +949,9 @@ extern "C" fl_status fl_execute_noalloc(int64_t M, int64_t N, int64_t K, int32_t
                   need, kNoallocTmpBytes);
     p.tmp_bytes = (size_t)need;
     p.d_tmp = scratch + kNoallocHeadBytes;
-    for (int sw = 0; sw < 2; ++sw)
-      FL_CUDA(cudaFuncSetAttribute(pick_kernel(ACT_NONE, epi->out_dtype, sw == 1),
+    for (int sw = 0; sw < 3; ++sw)
+      FL_CUDA(cudaFuncSetAttribute(sw == 2 ? pick_kernel_pair(ACT_NONE, epi->out_dtype)
+                                           : pick_kernel(ACT_NONE, epi->out_dtype, sw == 1),
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, p.max_smem));
   }
   // the error word must start at zero; the intermediate is fully overwritten

@@ -66,7 +66,8 @@ struct KParams {
   int b_box_rows;        // rows (K-major) or N-columns (MN-major) per B box
   int b_mn_major;        // 1: B stored [K, N]
   int geglu;             // 1: B = [gate rows ; up rows] from two tensor maps
-  uint32_t a_stage_bytes, b_box_bytes, stage_bytes;
+  uint32_t a_stage_bytes, b_box_bytes, stage_bytes;  // stage_bytes: bytes one stage's TMA loads deliver
+  uint32_t stage_stride;  // distance between stages (3xTF32 stages also hold the lo halves)
   uint32_t idesc;
   uint32_t a_kstep, b_kstep;  // descriptor start-address advance per UMMA K step (bytes)
   uint32_t b_lbo;             // leading byte offset of an MN-major B operand
@@ -191,6 +192,20 @@ __device__ __forceinline__ float ldg_pinned(const void* base, long long i, int d
   asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(h) : "l"(reinterpret_cast<const uint16_t*>(base) + i) : "memory");
   if (dt == DT_BF16) return __uint_as_float(static_cast<uint32_t>(h) << 16);
   return __half2float(__ushort_as_half(h));
+}
+
+// ------------------------------------------------------------------ 3xTF32 split
+// x = hi + lo with hi = x rounded to TF32 (nearest, ties away) and lo = x - hi
+// (exact in fp32) rounded to TF32 again, so that the tensor core reads both
+// halves exactly: x·y ≈ hi_x·hi_y + hi_x·lo_y + lo_x·hi_y.
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = tf32_rna(x);
+  lo = tf32_rna(x - __uint_as_float(hi));
 }
 
 // ------------------------------------------------------------------ epilogue helpers
@@ -325,7 +340,7 @@ __device__ __forceinline__ void swap_finish(const KParams& p, const float (&v)[3
 }
 
 // ------------------------------------------------------------------ kernel
-template <int ACT, int OUT, bool SWAP>
+template <int ACT, int OUT, bool SWAP, bool TF32 = false, bool PAIR = false>
 __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
     fl_gemm_epi_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmOut,
@@ -346,14 +361,22 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
   const uint32_t red_ready_bar = bars + 8u * (2 * NS + 5);
   const uint32_t red_done_bar = bars + 8u * (2 * NS + 6);
   const uint32_t tmem_slot = bars + 8u * (2 * NS + 7);
+  auto conv_bar = [&](int s) { return bars + 8u * (2 * NS + 8 + s); };  // 3xTF32: stage split done
 
+  // Clusters: split-K groups of S CTAs (swap layout), or CTA pairs that share one
+  // 256-row UMMA (PAIR: rank 0 issues the UMMA for both, each CTA owns 128 rows).
   const int S = p.split_k;
-  const uint32_t rank = (S > 1) ? cluster_ctarank() : 0u;
-  const int cluster_id = blockIdx.x / S;
-  const int num_clusters = gridDim.x / S;
+  constexpr int kCl = PAIR ? 2 : 1;
+  const uint32_t rank = (S > 1 || PAIR) ? cluster_ctarank() : 0u;
+  const int csize = PAIR ? kCl : S;
+  const int cluster_id = blockIdx.x / csize;
+  const int num_clusters = gridDim.x / csize;
   const int total_tiles = p.tiles_a * p.tiles_b;
-  const int kb_begin = (int)(((long long)p.num_kb * rank) / S);
-  const int kb_end = (int)(((long long)p.num_kb * (rank + 1)) / S);
+  const uint32_t krank = PAIR ? 0u : rank;  // split-K slice of this CTA
+  const int kb_begin = (int)(((long long)p.num_kb * krank) / S);
+  const int kb_end = (int)(((long long)p.num_kb * (krank + 1)) / S);
+  const int tile_rows = PAIR ? 256 : 128;   // output rows per tile (both CTAs of a pair)
+  const int cta_row_off = PAIR ? (int)rank * 128 : 0;
   const bool have_acc = kb_end > kb_begin;
 
   if (threadIdx.x == 0) {
@@ -363,13 +386,15 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), kEpiWarps);
+      mbar_init(tempty_bar(b), kEpiWarps * kCl);  // PAIR: the peer's epilogue warps arrive too
     }
     mbar_init(drain_bar, 1);
     // split-K hand-off: one arrive per epilogue warp (after __syncwarp, so the
     // release covers the whole warp's shared-memory writes)
     mbar_init(red_ready_bar, kEpiWarps * S);
     mbar_init(red_done_bar, kEpiWarps * S);
+    if (TF32)
+      for (int s = 0; s < NS; ++s) mbar_init(conv_bar(s), kEpiWarps);
     fence_mbarrier_init();
     if (p.num_kb > 0) {  // with K = 0 the operand maps are left unencoded and never used
       prefetch_tensormap(&tmA);
@@ -379,13 +404,18 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
     if (!SWAP) prefetch_tensormap(&tmOut);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, p.tmem_cols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, p.tmem_cols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, p.tmem_cols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (S > 1) cluster_sync_all();  // peers' barriers are initialised before any remote arrive
+  if (S > 1 || PAIR) cluster_sync_all();  // peers' barriers are initialised before any remote arrive
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(
       __cvta_shared_to_generic(tmem_slot));
 
@@ -397,34 +427,53 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
       for (int t = cluster_id; ok && t < total_tiles; t += num_clusters) {
         int ta, tb;
         tile_coords(t, p, ta, tb);
-        const int a_row = ta * 128;
-        const int b_row = tb * p.mma_n;
+        const int a_row = ta * tile_rows + cta_row_off;
+        // PAIR: each CTA loads its half of the B tile
+        const int b_row = tb * p.mma_n + (PAIR ? (int)rank * (p.mma_n / 2) : 0);
         const int g_row = tb * p.b_box_rows;
         for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
           const int s = (int)(it % (uint32_t)NS);
           const uint32_t ph = (it / (uint32_t)NS) & 1u;
           if (!wait_bounded(empty_bar(s), ph ^ 1u, p)) { ok = false; break; }
-          const uint32_t fb = full_bar(s);
-          mbar_arrive_expect_tx(fb, p.stage_bytes);
-          const uint32_t sa = smem_base + (uint32_t)s * p.stage_bytes;
+          const uint32_t sa = smem_base + (uint32_t)s * p.stage_stride;
           const uint32_t sb = sa + p.a_stage_bytes;
           const int k0 = kb * p.bk;
-          tma_load_2d(sa, &tmA, fb, k0, a_row);
-          if (p.b_mn_major) {
-            for (int i = 0; i < p.b_boxes; ++i) tma_load_2d(sb + i * p.b_box_bytes, &tmB, fb, b_row + i * 64, k0);
-          } else if (p.geglu) {
-            tma_load_2d(sb, &tmB, fb, k0, g_row);
-            tma_load_2d(sb + p.b_box_bytes, &tmB2, fb, k0, g_row);
+          if constexpr (PAIR) {
+            // both CTAs' bytes complete on the leader's full barrier
+            const uint32_t fb = mapa_shared(full_bar(s), 0);
+            if (rank == 0) mbar_arrive_expect_tx(full_bar(s), 2u * p.stage_bytes);
+            tma_load_2d_pair(sa, &tmA, fb, k0, a_row);
+            if (p.b_mn_major) {
+              for (int i = 0; i < p.b_boxes; ++i)
+                tma_load_2d_pair(sb + i * p.b_box_bytes, &tmB, fb, b_row + i * 64, k0);
+            } else if (p.geglu) {
+              // the pair's 256-wide B tile is [128 gate rows (rank 0) ; 128 up rows (rank 1)]
+              tma_load_2d_pair(sb, rank == 0 ? &tmB : &tmB2, fb, k0, g_row);
+            } else {
+              tma_load_2d_pair(sb, &tmB, fb, k0, b_row);
+            }
           } else {
-            for (int i = 0; i < p.b_boxes; ++i)
-              tma_load_2d(sb + i * p.b_box_bytes, &tmB, fb, k0, b_row + i * p.b_box_rows);
+            const uint32_t fb = full_bar(s);
+            mbar_arrive_expect_tx(fb, p.stage_bytes);
+            tma_load_2d(sa, &tmA, fb, k0, a_row);
+            if (p.b_mn_major) {
+              for (int i = 0; i < p.b_boxes; ++i) tma_load_2d(sb + i * p.b_box_bytes, &tmB, fb, b_row + i * 64, k0);
+            } else if (p.geglu) {
+              tma_load_2d(sb, &tmB, fb, k0, g_row);
+              tma_load_2d(sb + p.b_box_bytes, &tmB2, fb, k0, g_row);
+            } else {
+              for (int i = 0; i < p.b_boxes; ++i)
+                tma_load_2d(sb + i * p.b_box_bytes, &tmB, fb, k0, b_row + i * p.b_box_rows);
+            }
           }
         }
       }
       // Never leave the CTA with copies in flight: wait (bounded) for the last
       // fill of every stage (fill i went to stage i % NS with phase (i / NS) & 1).
-      // In the normal path these have all completed already.
-      for (uint32_t s = 0; s < (uint32_t)NS && s < it; ++s) {
+      // In the normal path these have all completed already.  A pair's peer
+      // counts its bytes on the leader's barriers, which the leader waits for; the
+      // final cluster barrier keeps the peer resident until then.
+      for (uint32_t s = 0; (!PAIR || rank == 0) && s < (uint32_t)NS && s < it; ++s) {
         const uint32_t last = it - 1u - ((it - 1u - s) % (uint32_t)NS);
         (void)wait_bounded(full_bar((int)s), (last / (uint32_t)NS) & 1u, p);
       }
@@ -432,12 +481,16 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
     __syncwarp();  // reconverge: the CTA barrier below is warp-aligned
   } else if (warp == 1) {
     // ================================================================ UMMA issuer
-    if (lane == 0) {
+    if (lane == 0 && (!PAIR || rank == 0)) {  // in a pair, rank 0 issues for both CTAs
       // Descriptors of stage 0; a stage s and UMMA step k only move the start
       // address field (addresses stay below 2^18 bytes, so no carry leaves it).
       const uint64_t da0 = sdesc_sw128(smem_base, 16, 1024);
       const uint64_t db0 = sdesc_sw128(smem_base + p.a_stage_bytes, p.b_mn_major ? p.b_lbo : 16u, 1024);
-      const uint64_t stage_step = p.stage_bytes >> 4;
+      const uint64_t stage_step = p.stage_stride >> 4;
+      // 3xTF32: lo halves of A and B follow the raw (hi) tiles inside each stage
+      const uint32_t lo_off = p.stage_bytes;
+      const uint64_t dal0 = sdesc_sw128(smem_base + lo_off, 16, 1024);
+      const uint64_t dbl0 = sdesc_sw128(smem_base + lo_off + p.a_stage_bytes, 16, 1024);
       const uint64_t ak = p.a_kstep >> 4, bk = p.b_kstep >> 4;
       const uint32_t idesc = p.idesc;
       uint32_t it = 0, local = 0;
@@ -445,28 +498,59 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
       for (int t = cluster_id; ok && t < total_tiles; t += num_clusters, ++local) {
         const uint32_t buf = local & 1u;
         const uint32_t tph = (local >> 1) & 1u;
-        if (!wait_bounded(tempty_bar(buf), tph ^ 1u, p)) { ok = false; break; }
+        if (!wait_bounded(tempty_bar(buf), tph ^ 1u, p, PAIR)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * (uint32_t)p.mma_n;
         for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
           const int s = (int)(it % (uint32_t)NS);
           const uint32_t ph = (it / (uint32_t)NS) & 1u;
-          if (!wait_bounded(full_bar(s), ph, p)) { ok = false; break; }
+          if (!wait_bounded(TF32 ? conv_bar(s) : full_bar(s), ph, p)) { ok = false; break; }
           tc_fence_after();
           const uint64_t da = da0 + (uint64_t)s * stage_step;
           const uint64_t db = db0 + (uint64_t)s * stage_step;
+          if constexpr (TF32) {
+            const uint64_t dal = dal0 + (uint64_t)s * stage_step;
+            const uint64_t dbl = dbl0 + (uint64_t)s * stage_step;
 #pragma unroll
-          for (int k = 0; k < kUmmaSteps; ++k)
-            umma_f16(d_tmem, da + k * ak, db + k * bk, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
-          umma_commit(empty_bar(s));  // frees the stage once these MMAs have read it
+            for (int k = 0; k < kUmmaSteps; ++k) {
+              umma_tf32(d_tmem, dal + k * ak, db + k * bk, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
+              umma_tf32(d_tmem, da + k * ak, dbl + k * bk, idesc, 1u);
+              umma_tf32(d_tmem, da + k * ak, db + k * bk, idesc, 1u);
+            }
+          } else if constexpr (PAIR) {
+#pragma unroll
+            for (int k = 0; k < kUmmaSteps; ++k)
+              umma_f16_pair(d_tmem, da + k * ak, db + k * bk, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int k = 0; k < kUmmaSteps; ++k)
+              umma_f16(d_tmem, da + k * ak, db + k * bk, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
+          }
+          if constexpr (PAIR) {  // free the stage in both CTAs once these MMAs have read it
+            umma_commit_pair(empty_bar(s));
+            umma_commit_pair(mapa_shared(empty_bar(s), 1));
+          } else {
+            umma_commit(empty_bar(s));  // frees the stage once these MMAs have read it
+          }
           issued = true;
         }
         if (!ok) break;
-        if (have_acc) umma_commit(tfull_bar(buf));
-        else mbar_arrive(tfull_bar(buf));
+        if constexpr (PAIR) {
+          if (have_acc) {
+            umma_commit_pair(tfull_bar(buf));
+            umma_commit_pair(mapa_shared(tfull_bar(buf), 1));
+          } else {
+            mbar_arrive(tfull_bar(buf));
+            mbar_arrive_remote(mapa_shared(tfull_bar(buf), 1));
+          }
+        } else {
+          if (have_acc) umma_commit(tfull_bar(buf));
+          else mbar_arrive(tfull_bar(buf));
+        }
       }
       if (issued) {  // no MMA may still be running when TMEM is released
-        umma_commit(drain_bar);
+        if constexpr (PAIR) umma_commit_pair(drain_bar);
+        else umma_commit(drain_bar);
         (void)wait_bounded(drain_bar, 0, p);
       }
     }
@@ -488,18 +572,53 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
       const int half = ew >> 2;
       const uint32_t stg = smem_base + p.staging_off + (uint32_t)ew * kStagingBuf;
       const int half_cols = p.out_tile_n >> 1;
+      uint32_t cit = 0;  // 3xTF32: stage counter, in step with the producer and the MMA warp
       for (int t = cluster_id; t < total_tiles; t += num_clusters, ++local) {
         int ta, tb;
         tile_coords(t, p, ta, tb);
+        if constexpr (TF32) {
+          // split every stage of this tile into hi (in place) and lo halves; the 256
+          // epilogue threads share the stage's 16-byte words
+          const int et = (warp - kEpiWarp0) * 32 + lane;
+          const uint32_t words = p.stage_bytes >> 4;
+          for (int kb = kb_begin; ok && kb < kb_end; ++kb, ++cit) {
+            const int s = (int)(cit % (uint32_t)NS);
+            const uint32_t ph = (cit / (uint32_t)NS) & 1u;
+            if (!warp_wait_bounded(full_bar(s), ph, p, lane)) { ok = false; break; }
+            const uint32_t st0 = smem_base + (uint32_t)s * p.stage_stride;
+            for (uint32_t w = (uint32_t)et; w < words; w += kEpiWarps * 32) {
+              const uint32_t a = st0 + 16u * w;
+              float4 x;
+              asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                           : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w)
+                           : "r"(a)
+                           : "memory");
+              uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+              split_tf32(x.x, h0, l0);
+              split_tf32(x.y, h1, l1);
+              split_tf32(x.z, h2, l2);
+              split_tf32(x.w, h3, l3);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(h0), "r"(h1), "r"(h2), "r"(h3)
+                           : "memory");
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a + p.stage_bytes), "r"(l0), "r"(l1),
+                           "r"(l2), "r"(l3)
+                           : "memory");
+            }
+            fence_proxy_async_smem();  // the tensor core reads these through the async proxy
+            __syncwarp();
+            if (lane == 0) mbar_arrive(conv_bar(s));
+          }
+          if (!ok) break;
+        }
         const uint32_t buf = local & 1u;
         const uint32_t tph = (local >> 1) & 1u;
-        const int row0 = ta * 128 + q * 32;
+        const int row0 = ta * tile_rows + cta_row_off + q * 32;
         const int m = row0 + lane;
         const bool m_ok = m < p.M;
         const int n_tile0 = tb * p.out_tile_n;
         float bias_m = 0.0f;
         if (has_bias && p.bias_axis == 1 && m_ok) bias_m = ldg_pinned(p.bias, m, p.bias_dtype);
-        if (!warp_wait_bounded(tfull_bar(buf), tph, p, lane)) { ok = false; break; }
+        if (!warp_wait_bounded(tfull_bar(buf), tph, p, lane, PAIR)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
         const int c_begin = half * half_cols;
@@ -549,9 +668,13 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           }
           if (cc + CH >= c_end) {
             // this warp's TMEM reads of the tile are done: hand its share back to the MMA warp
+            // (in a pair, to the leader's barrier)
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar(buf));
+            if (lane == 0) {
+              if (PAIR && rank != 0) mbar_arrive_remote(mapa_shared(tempty_bar(buf), 0));
+              else mbar_arrive(tempty_bar(buf));
+            }
           }
           // ---- bias, activation, aux, residual, scale (all in fp32 registers)
           if (has_bias) {
@@ -753,9 +876,12 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
   // Every thread of every role arrives here converged, after its last TMEM
   // read, MMA (drained) and copy; only then is TMEM released.
   __syncthreads();
+  // a pair stays resident until neither CTA can touch the other's barriers or TMEM
+  if (PAIR) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, p.tmem_cols);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, p.tmem_cols);
+    else tmem_dealloc(tmem_base, p.tmem_cols);
   }
 }
 

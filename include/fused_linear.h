@@ -153,7 +153,8 @@ typedef struct {
   int32_t grid;                /* CTAs launched by the main kernel */
   int32_t smem_bytes;          /* dynamic shared memory per CTA */
   int32_t launches_per_execute;/* kernels one fl_execute launches */
-  int32_t reserved[7];
+  int32_t cta_pair;            /* 1: two CTAs share each 256-row tensor-core tile */
+  int32_t reserved[6];
 } fl_plan_info;
 fl_status fl_get_plan_info(fl_plan_t plan, fl_plan_info* info);
 

@@ -168,7 +168,21 @@ def _run_workload_linear(fl, w, seed=0, rows=256):
     return got, inp, sel, v
 
 
-@pytest.mark.parametrize("name", ["relu_bias_100x256x784", "linear_gelu_tanh_bf16_1024x3072x768",
+@pytest.mark.parametrize("M,N,K,epilogue,out_dtype", [(300, 520, 200, "GELU_BIAS", "f32"),
+                                                       (130, 264, 100, "RELU_AUX_BIAS", "bf16"),
+                                                       (64, 136, 36, "BIAS", "f32"),
+                                                       (257, 384, 768, "GELU_TANH_BIAS", "f16")])
+def test_fp32_operands_3xtf32(fl, M, N, K, epilogue, out_dtype):
+    got = _linear_case(fl, M, N, K, dtype="f32", epilogue=epilogue, out_dtype=out_dtype, seed=13)
+    assert got["info"]["swap_ab"] == 0
+
+
+def test_fp32_residual_scale(fl):
+    _linear_case(fl, 200, 264, 132, dtype="f32", epilogue="GELU_BIAS", out_dtype="f32", residual=True, scale=0.5)
+
+
+@pytest.mark.parametrize("name", ["relu_bias_100x256x784", "linear_gelu_f32_1024x3072x768",
+                                  "linear_gelu_tanh_bf16_1024x3072x768",
                                   "tail_m32", "tail_m128", "tail_m512", "tail_m2048"])
 def test_workload_linear(fl, name):
     _run_workload_linear(fl, workloads.get(name))
