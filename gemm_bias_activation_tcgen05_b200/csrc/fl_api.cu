@@ -183,6 +183,7 @@ struct fl_plan_s {
   // configuration
   bool swap;
   bool pair;  // two CTAs share one 256-row UMMA tile (cluster of 2)
+  int k_atoms;  // 128-byte K atoms per pipeline stage
   int mma_n, out_tile_n, split_k, stages, grid, smem;
   int tiles_a, tiles_b, num_kb;
   const void* kernel;
@@ -220,12 +221,17 @@ struct Layout {
 static Layout layout_for(const fl_plan_s* p, int mma_n, int b_boxes, int max_smem) {
   Layout L{};
   const int es = esize(p->dtype);
-  const int bk = 128 / es;
+  const int atoms = std::max(1, p->k_atoms);
+  const int bk = atoms * 128 / es;
   const int rows_b = p->pair ? mma_n / 2 : mma_n;  // B rows (or columns) held by one CTA
-  L.a_stage = 128u * 128u;  // 128 rows x 128 bytes
-  if (p->epi.b_major) L.b_box = 64u * (uint32_t)bk * (uint32_t)es;  // 64 columns x bk rows
-  else L.b_box = (uint32_t)(rows_b / b_boxes) * 128u;
-  L.b_stage = L.b_box * (uint32_t)b_boxes;
+  L.a_stage = (uint32_t)atoms * 128u * 128u;       // 128 rows x 128 bytes per atom
+  if (p->epi.b_major) {
+    L.b_box = 64u * (uint32_t)bk * (uint32_t)es;   // 64 columns x bk rows
+    L.b_stage = L.b_box * (uint32_t)b_boxes;
+  } else {
+    L.b_box = (uint32_t)(rows_b / b_boxes) * 128u;
+    L.b_stage = L.b_box * (uint32_t)b_boxes * (uint32_t)atoms;
+  }
   L.stage = L.a_stage + L.b_stage;
   // fp32 operands: each stage also holds the TF32 lo halves of both tiles
   L.stride = (p->dtype == FL_F32) ? 2u * L.stage : L.stage;
@@ -268,12 +274,16 @@ static const void* kernel_of(const fl_plan_s* p, int act, int out) {
 static fl_status choose_config(fl_plan_s* p) {
   const int64_t M = p->M, N = p->N;
   const int es = esize(p->dtype);
-  const int bk = 128 / es;
-  p->num_kb = (int)cdiv(p->K, bk);
+  p->pair = false;
   const bool geglu = p->epi.kind == FL_EPI_GEGLU_TANH;
   // Small M: put the weight on the 128-row side of the tensor core (swap-AB)
   // and split K across a cluster so that every SM streams a slice of W.
   p->swap = (M <= 128) && !geglu && !p->epi.b_major && p->dtype != FL_F32;
+  // CTA pairs take 128-deep K stages (two swizzle atoms, eight UMMA steps per
+  // barrier round trip); the other layouts keep one atom per stage.
+  p->pair = !p->swap && p->dtype != FL_F32 && M > 128;
+  p->k_atoms = p->pair ? 2 : 1;
+  p->num_kb = (int)cdiv(p->K, (int64_t)p->k_atoms * 128 / es);
   if (p->swap) {
     // The epilogue moves TMEM in 32-column chunks, so the activation tile is a multiple of 32.
     p->mma_n = (int)std::max<int64_t>(32, cdiv(M, 32) * 32);
@@ -289,7 +299,6 @@ static fl_status choose_config(fl_plan_s* p) {
   } else {
     p->split_k = 1;
     // 16-bit operands beyond one 128-row tile: CTA pairs with 256-row UMMA tiles
-    p->pair = p->dtype != FL_F32 && M > 128;
     const int rows = p->pair ? 256 : 128;
     const int units = p->pair ? p->num_sms / 2 : p->num_sms;
     if (geglu) {
@@ -523,7 +532,7 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
   const void* key[8] = {g.A, g.W, g.out, g.bias, g.residual, g.aux, kernel, (const void*)(intptr_t)g.ldo};
   if (cache->valid && memcmp(cache->key, key, sizeof(key)) == 0) return launch_kernel(p, *cache, stream, kernel, swap);
   const int es = esize(p->dtype);
-  const int bk = 128 / es;
+  const int bk = p->k_atoms * 128 / es;
   const fl_epilogue_desc& e = p->epi;
   KParams k{};
   k.M = (int)p->M;
@@ -547,6 +556,10 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
   k.b_box_bytes = L.b_box;
   k.stage_bytes = L.stage;
   k.stage_stride = L.stride;
+  k.k_atoms = p->k_atoms;
+  k.a_atom_bytes = 128u * 128u;
+  k.b_atom_bytes = e.b_major ? 0u : (uint32_t)(p->pair ? p->mma_n / 2 : p->mma_n) * 128u;
+  k.usteps = kUmmaSteps * p->k_atoms;
   k.staging_off = L.staging_off;
   k.bias_off = L.bias_off;
   k.red_off = L.red_off;
@@ -577,6 +590,7 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
   k.wait_limit_ns = p->wait_limit_ns;
 
   CUtensorMap tmA, tmB, tmB2, tmOut;
+  const int ae = 128 / es;  // K elements of one 128-byte swizzle atom: the inner box of K-major maps
   memset(&tmB2, 0, sizeof(tmB2));
   memset(&tmOut, 0, sizeof(tmOut));
   fl_status st;
@@ -585,7 +599,7 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
   memset(&tmA, 0, sizeof(tmA));
   memset(&tmB, 0, sizeof(tmB));
   if (!swap) {
-    if (!no_k) st = make_map(&tmA, g.A, p->dtype, Kd, (uint64_t)p->M, (uint64_t)e.lda * es, (uint32_t)bk, 128);
+    if (!no_k) st = make_map(&tmA, g.A, p->dtype, Kd, (uint64_t)p->M, (uint64_t)e.lda * es, (uint32_t)ae, 128);
     else st = FL_OK;
     if (st) return st;
     if (no_k) {
@@ -593,12 +607,12 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
     } else if (e.b_major) {
       st = make_map(&tmB, g.W, p->dtype, (uint64_t)g.n_cols, Kd, (uint64_t)e.ldb * es, 64, (uint32_t)bk);
     } else if (g.geglu_fused) {
-      st = make_map(&tmB, g.W, p->dtype, Kd, (uint64_t)p->N, (uint64_t)e.ldb * es, (uint32_t)bk, 128);
+      st = make_map(&tmB, g.W, p->dtype, Kd, (uint64_t)p->N, (uint64_t)e.ldb * es, (uint32_t)ae, 128);
       if (st) return st;
       const char* up = static_cast<const char*>(g.W) + (size_t)p->N * (size_t)e.ldb * es;
-      st = make_map(&tmB2, up, p->dtype, Kd, (uint64_t)p->N, (uint64_t)e.ldb * es, (uint32_t)bk, 128);
+      st = make_map(&tmB2, up, p->dtype, Kd, (uint64_t)p->N, (uint64_t)e.ldb * es, (uint32_t)ae, 128);
     } else {
-      st = make_map(&tmB, g.W, p->dtype, Kd, (uint64_t)g.n_cols, (uint64_t)e.ldb * es, (uint32_t)bk,
+      st = make_map(&tmB, g.W, p->dtype, Kd, (uint64_t)g.n_cols, (uint64_t)e.ldb * es, (uint32_t)ae,
                     (uint32_t)(p->pair ? p->mma_n / 2 : p->mma_n));
     }
     if (st) return st;
@@ -612,9 +626,9 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
     if (st) return st;
   } else if (!no_k) {
     // UMMA A = weight rows (output features), UMMA B = activation rows
-    st = make_map(&tmA, g.W, p->dtype, Kd, (uint64_t)g.n_cols, (uint64_t)e.ldb * es, (uint32_t)bk, 128);
+    st = make_map(&tmA, g.W, p->dtype, Kd, (uint64_t)g.n_cols, (uint64_t)e.ldb * es, (uint32_t)ae, 128);
     if (st) return st;
-    st = make_map(&tmB, g.A, p->dtype, Kd, (uint64_t)p->M, (uint64_t)e.lda * es, (uint32_t)bk,
+    st = make_map(&tmB, g.A, p->dtype, Kd, (uint64_t)p->M, (uint64_t)e.lda * es, (uint32_t)ae,
                   (uint32_t)p->mma_n);
     if (st) return st;
     tmOut = tmA;  // unused in the swap layout

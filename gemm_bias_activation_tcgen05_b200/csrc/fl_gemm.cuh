@@ -39,7 +39,8 @@ enum DType : int { DT_F16 = 0, DT_BF16 = 1, DT_F32 = 2 };
 
 constexpr int kEpiWarp0 = 2;                 // warps 0,1: TMA producer, UMMA issuer
 constexpr uint32_t kStagingBuf = 32 * 128;    // one epilogue warp's 32 rows x 128 bytes
-constexpr int kUmmaSteps = 4;                 // UMMA instructions per 128-byte K stage
+constexpr int kUmmaSteps = 4;                 // UMMA instructions per 128-byte K atom
+constexpr int kMaxSteps = 8;                  // at most two atoms per stage
 constexpr int kErrTimeout = 1;
 
 // Normal layout: 8 epilogue warps (two per TMEM lane quarter, one per column
@@ -68,6 +69,9 @@ struct KParams {
   int geglu;             // 1: B = [gate rows ; up rows] from two tensor maps
   uint32_t a_stage_bytes, b_box_bytes, stage_bytes;  // stage_bytes: bytes one stage's TMA loads deliver
   uint32_t stage_stride;  // distance between stages (3xTF32 stages also hold the lo halves)
+  int k_atoms;            // 128-byte swizzle atoms of K per stage (1, or 2 for 128-deep bf16 stages)
+  uint32_t a_atom_bytes, b_atom_bytes;  // bytes of one atom of A / of (this CTA's) B
+  int usteps;             // UMMA instructions per stage (4 per atom)
   uint32_t idesc;
   uint32_t a_kstep, b_kstep;  // descriptor start-address advance per UMMA K step (bytes)
   uint32_t b_lbo;             // leading byte offset of an MN-major B operand
@@ -438,19 +442,21 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           const uint32_t sa = smem_base + (uint32_t)s * p.stage_stride;
           const uint32_t sb = sa + p.a_stage_bytes;
           const int k0 = kb * p.bk;
+          const int ae = p.bk / p.k_atoms;  // K elements of one 128-byte atom
           if constexpr (PAIR) {
             // both CTAs' bytes complete on the leader's full barrier
             const uint32_t fb = mapa_shared(full_bar(s), 0);
             if (rank == 0) mbar_arrive_expect_tx(full_bar(s), 2u * p.stage_bytes);
-            tma_load_2d_pair(sa, &tmA, fb, k0, a_row);
+            for (int a = 0; a < p.k_atoms; ++a)
+              tma_load_2d_pair(sa + a * p.a_atom_bytes, &tmA, fb, k0 + a * ae, a_row);
             if (p.b_mn_major) {
               for (int i = 0; i < p.b_boxes; ++i)
                 tma_load_2d_pair(sb + i * p.b_box_bytes, &tmB, fb, b_row + i * 64, k0);
-            } else if (p.geglu) {
-              // the pair's 256-wide B tile is [128 gate rows (rank 0) ; 128 up rows (rank 1)]
-              tma_load_2d_pair(sb, rank == 0 ? &tmB : &tmB2, fb, k0, g_row);
             } else {
-              tma_load_2d_pair(sb, &tmB, fb, k0, b_row);
+              // GeGLU: the pair's 256-wide B tile is [128 gate rows (rank 0) ; 128 up rows (rank 1)]
+              const CUtensorMap* mb = (p.geglu && rank != 0) ? &tmB2 : &tmB;
+              const int br = p.geglu ? g_row : b_row;
+              for (int a = 0; a < p.k_atoms; ++a) tma_load_2d_pair(sb + a * p.b_atom_bytes, mb, fb, k0 + a * ae, br);
             }
           } else {
             const uint32_t fb = full_bar(s);
@@ -492,6 +498,16 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
       const uint64_t dal0 = sdesc_sw128(smem_base + lo_off, 16, 1024);
       const uint64_t dbl0 = sdesc_sw128(smem_base + lo_off + p.a_stage_bytes, 16, 1024);
       const uint64_t ak = p.a_kstep >> 4, bk = p.b_kstep >> 4;
+      // start-address offsets (16-byte units) of UMMA step j inside a stage: atom j/4,
+      // then 32 bytes per step inside the atom (an MN-major B advances 16 K rows per step)
+      uint32_t aso[kMaxSteps], bso[kMaxSteps];
+#pragma unroll
+      for (int j = 0; j < kMaxSteps; ++j) {
+        aso[j] = ((uint32_t)(j >> 2) * p.a_atom_bytes + (uint32_t)(j & 3) * p.a_kstep) >> 4;
+        bso[j] = p.b_mn_major ? ((uint32_t)j * p.b_kstep) >> 4
+                              : ((uint32_t)(j >> 2) * p.b_atom_bytes + (uint32_t)(j & 3) * p.b_kstep) >> 4;
+      }
+      const int usteps = p.usteps;
       const uint32_t idesc = p.idesc;
       uint32_t it = 0, local = 0;
       bool ok = true, issued = false;
@@ -519,12 +535,14 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
             }
           } else if constexpr (PAIR) {
 #pragma unroll
-            for (int k = 0; k < kUmmaSteps; ++k)
-              umma_f16_pair(d_tmem, da + k * ak, db + k * bk, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
+            for (int k = 0; k < kMaxSteps; ++k)
+              if (k < usteps)
+                umma_f16_pair(d_tmem, da + aso[k], db + bso[k], idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
           } else {
 #pragma unroll
-            for (int k = 0; k < kUmmaSteps; ++k)
-              umma_f16(d_tmem, da + k * ak, db + k * bk, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
+            for (int k = 0; k < kMaxSteps; ++k)
+              if (k < usteps)
+                umma_f16(d_tmem, da + aso[k], db + bso[k], idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
           }
           if constexpr (PAIR) {  // free the stage in both CTAs once these MMAs have read it
             umma_commit_pair(empty_bar(s));
