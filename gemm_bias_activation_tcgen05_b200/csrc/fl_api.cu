@@ -215,6 +215,7 @@ static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // the reduction buffer, then the barriers.
 struct Layout {
   uint32_t a_stage, b_box, b_stage, stage, stride, staging_off, bias_off, bar_off, red_off, red_pitch, total;
+  uint32_t res_off, res_blk;
   int stages;
 };
 
@@ -238,8 +239,11 @@ static Layout layout_for(const fl_plan_s* p, int mma_n, int b_boxes, int max_sme
   const uint32_t staging = p->swap ? Cfg<true>::kStagingBytes : Cfg<false>::kStagingBytes;
   const uint32_t bias = 0;
   const uint32_t red = (p->swap && p->split_k > 1) ? 128u * ((uint32_t)mma_n * 4u + 16u) : 0u;
+  // swap-AB with a residual: two 32-row x 32-column residual blocks per epilogue warp
+  L.res_blk = 32u * 32u * (uint32_t)esize(p->epi.residual_dtype);
+  const uint32_t res = (p->swap && p->epi.has_residual) ? (uint32_t)Cfg<true>::kEpiWarps * 2u * L.res_blk : 0u;
   const uint32_t bars = 8u * (3u * 8u + 8u);
-  const uint32_t budget = (uint32_t)max_smem - 1024u - staging - bias - red - bars;
+  const uint32_t budget = (uint32_t)max_smem - 1024u - staging - bias - red - res - bars;
   int st = (int)(budget / L.stride);
   if (st > 8) st = 8;
   L.stages = st;
@@ -247,7 +251,8 @@ static Layout layout_for(const fl_plan_s* p, int mma_n, int b_boxes, int max_sme
   L.bias_off = L.staging_off + staging;
   L.red_off = L.bias_off + bias;
   L.red_pitch = (uint32_t)mma_n * 4u + 16u;
-  L.bar_off = L.red_off + red;
+  L.res_off = L.red_off + red;
+  L.bar_off = L.res_off + res;
   L.total = L.bar_off + 8u * (3u * (uint32_t)st + 8u) + 1024u;
   return L;
 }
@@ -564,6 +569,8 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
   k.bias_off = L.bias_off;
   k.red_off = L.red_off;
   k.red_pitch = L.red_pitch;
+  k.res_off = L.res_off;
+  k.res_blk_bytes = L.res_blk;
   k.bar_off = L.bar_off;
   const uint32_t fmt = (p->dtype == FL_BF16) ? 1u : (p->dtype == FL_F32 ? 2u : 0u);  // F16 / BF16 / TF32
   k.idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(e.b_major ? 1 : 0) << 16) |
@@ -581,6 +588,7 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
   k.residual = g.residual;
   k.ldr = e.ldr;
   k.res_dtype = e.residual_dtype;
+  k.res_async = g.residual != nullptr && (reinterpret_cast<uintptr_t>(g.residual) & 15u) == 0;
   k.out = g.out;
   k.ldo = g.ldo;
   k.aux = g.aux;
@@ -707,6 +715,8 @@ extern "C" fl_status fl_execute(fl_plan_t p, const void* A, const void* W, const
     // The unfused GEMM uses the same tcgen05 kernel with no epilogue work.
     fl_plan_s q = *p;
     q.epi.kind = FL_EPI_NONE;
+    q.epi.ldr = 0;
+    q.epi.has_residual = 0;
     q.N = cols;
     choose_config(&q);
     const int b_boxes = b_boxes_of(&q, false);

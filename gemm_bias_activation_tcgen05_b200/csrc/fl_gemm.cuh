@@ -77,6 +77,9 @@ struct KParams {
   uint32_t b_lbo;             // leading byte offset of an MN-major B operand
   uint32_t tmem_cols;
   uint32_t staging_off, bias_off, bar_off, red_off, red_pitch;
+  uint32_t res_off;        // swap-AB: per-warp residual staging (two 32-row blocks per warp)
+  uint32_t res_blk_bytes;  // one 32-row x 32-column block of the residual
+  int res_async;           // 1: the residual is staged by 16-byte cp.async (aligned rows)
   // epilogue operands
   const void* bias;
   int bias_dtype, bias_axis;
@@ -289,58 +292,36 @@ __device__ __forceinline__ void ldg8(float (&dst)[8], const void* base, long lon
     dst[i] = (dt == DT_BF16) ? __uint_as_float(static_cast<uint32_t>(h[i]) << 16) : __half2float(__ushort_as_half(h[i]));
 }
 
-// Epilogue of the swap-AB layout for one thread: output column n, rows
-// m0 .. m0+cnt-1 with pre-activations v[0..cnt).  The warp's 32 lanes hold 32
-// consecutive columns starting at n_warp0 (a multiple of 32), so every row's
-// residual load and output store is one coalesced access and the ReLU mask
-// word of the row is one ballot.
+// Swap-AB epilogue, residual staging: rows [m0, m0+cnt) x columns [n0, n0+32)
+// of the residual go to shared memory (row-major, 32 elements a row) by 16-byte
+// cp.async, one commit group per call.  Bytes past column N are zero-filled;
+// every row copied is below M.  Requires 16-byte aligned rows (res_async).
+__device__ __forceinline__ void stage_residual(const KParams& p, uint32_t dst, int m0, int cnt, int n0, int lane) {
+  const int es = (p.res_dtype == DT_F32) ? 4 : 2;
+  const int cpr = 2 * es;  // 16-byte chunks in a 32-element row
+  const char* base = reinterpret_cast<const char*>(p.residual);
+#pragma unroll 1
+  for (int c = lane; c < cnt * cpr; c += 32) {
+    const int r = c / cpr, k = c - r * cpr;
+    const int col = n0 + k * (16 / es);
+    const int bytes = min(max(p.N - col, 0) * es, 16);
+    const char* src = bytes > 0 ? base + ((long long)(m0 + r) * p.ldr + col) * es : base;
+    cp_async_16(dst + (uint32_t)(r * 32 * es + k * 16), src, (uint32_t)bytes);
+  }
+  cp_async_commit();
+}
+
+// Swap-AB epilogue for one output element: lane = column n, row m, pre-activation
+// x (bias already added).  The mask word of row m is one ballot of the warp.
 template <int ACT, int OUT>
-__device__ __forceinline__ void swap_finish(const KParams& p, const float (&v)[32], int n, int n_warp0, int m0,
-                                            int cnt, int lane) {
-  const bool n_ok = n < p.N;
-  const bool has_res = p.residual != nullptr;
-  const bool has_bias = p.bias != nullptr;
-  float rr[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) rr[j] = 0.0f;
-  if (has_res && n_ok && cnt > 0) {
-    // eight rows per batch; rows past M re-read row M-1 (valid memory, result unused)
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      if (8 * g < cnt) {
-        float t[8];
-        if (8 * g + 8 <= cnt) {
-          ldg8(t, p.residual, (long long)(m0 + 8 * g) * p.ldr + n, p.ldr, p.res_dtype);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int mm = min(m0 + 8 * g + i, p.M - 1);
-            t[i] = ldg_pinned(p.residual, (long long)mm * p.ldr + n, p.res_dtype);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) rr[8 * g + i] = t[i];
-      }
-    }
+__device__ __forceinline__ void swap_store(const KParams& p, float x, float res, int m, int n, bool n_ok, int wcol,
+                                           int lane) {
+  if (p.aux != nullptr) {
+    const uint32_t word = __ballot_sync(0xffffffffu, n_ok && x > 0.0f);
+    if (lane == 0 && (long long)wcol * 32 < p.N) p.aux[(long long)m * p.ld_aux + wcol] = word;
   }
-  float bias_n = 0.0f;
-  if (has_bias && p.bias_axis == 0 && n_ok) bias_n = ldg_pinned(p.bias, n, p.bias_dtype);
-  const int w = n_warp0 >> 5;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    if (j >= cnt) continue;  // uniform across the warp
-    const int m = m0 + j;
-    float x = v[j];
-    if (has_bias) x += (p.bias_axis == 0) ? bias_n : ldg_pinned(p.bias, m, p.bias_dtype);
-    if (p.aux != nullptr) {
-      const uint32_t word = __ballot_sync(0xffffffffu, n_ok && x > 0.0f);
-      if (lane == 0 && (long long)w * 32 < p.N) p.aux[(long long)m * p.ld_aux + w] = word;
-    }
-    float y = activate<ACT>(x, 0.0f);
-    if (has_res) y += rr[j];
-    y *= p.scale;
-    if (n_ok) store_elem<OUT>(p.out, (long long)m * p.ldo + n, y);
-  }
+  const float y = (activate<ACT>(x, 0.0f) + res) * p.scale;
+  if (n_ok) store_elem<OUT>(p.out, (long long)m * p.ldo + n, y);
 }
 
 // ------------------------------------------------------------------ kernel
@@ -769,49 +750,44 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
       }
       if (lane == 0) bulk_wait_group<0>();
     } else {
-      // ---------------- swap-AB layout: TMEM lane = output column n, TMEM column = output row m
+      // ---------------- swap-AB layout: TMEM lane = output column n, TMEM column = output row m.
+      // Split-K (S > 1): every CTA publishes its fp32 partial tile in its own shared
+      // memory; CTA r then sums the S partials (in rank order) of TMEM lanes
+      // [r·128/S, (r+1)·128/S) and finishes those output columns.  Warp ew owns 32
+      // of those lanes and a contiguous range of rows.  The finishing loop is kept
+      // rolled (four rows a trip): it runs once per CTA, so its instructions come
+      // from L2, and a short loop body keeps that fetch small.
       const uint32_t red_base = smem_base + p.red_off;
+      const int L = 128 / S;
+      const int groups = L / 32;
+      const int g = (S == 1) ? q : ew % groups;          // S = 1: a warp finishes its own TMEM quarter
+      const int parts = kEpiWarps / groups;
+      const int part = (S == 1) ? 0 : ew / groups;
+      const int lrow = (int)rank * L + g * 32 + lane;    // TMEM lane = column within the tile
+      const int mcnt = p.mma_n / parts;                  // a multiple of 8
+      const int mb = part * mcnt;
+      const uint32_t my_row = red_base + (uint32_t)(q * 32 + lane) * p.red_pitch;  // published row
+      const uint32_t sum_row = red_base + (uint32_t)lrow * p.red_pitch;            // finished row
+      const uint32_t rst = smem_base + p.res_off + (uint32_t)ew * 2u * p.res_blk_bytes;
+      const bool res_async = has_res && p.res_async;
       for (int t = cluster_id; t < total_tiles; t += num_clusters, ++local) {
         int ta, tb;
         tile_coords(t, p, ta, tb);
         const uint32_t buf = local & 1u;
         const uint32_t tph = (local >> 1) & 1u;
-        const int m_tile0 = tb * p.mma_n;
+        const int m_lo = tb * p.mma_n + mb;                // first output row of this warp
+        const int rows = max(0, min(mcnt, p.M - m_lo));
+        const int n_w0 = ta * 128 + (int)rank * L + g * 32;
+        const int n = n_w0 + lane;
+        const bool n_ok = n < p.N;
+        // the residual's first block travels while the main loop runs
+        if (res_async && rows > 0) stage_residual(p, rst, m_lo, min(32, rows), n_w0, lane);
         if (!warp_wait_bounded(tfull_bar(buf), tph, p, lane)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
 
-        if (S == 1) {
-          // the whole tile is this CTA's: warp q finishes TMEM lanes [32q, 32q+32) over every row m
-          const int n = ta * 128 + q * 32 + lane;
-          for (int cc = 0; cc < p.mma_n; cc += 32) {
-            float v[32];
-            if (have_acc) {
-              uint32_t r[32];
-              tmem_ld32(tacc + (uint32_t)cc, r);
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-            }
-            if (cc + 32 >= p.mma_n) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(tempty_bar(buf));
-            }
-            swap_finish<ACT, OUT>(p, v, n, ta * 128 + q * 32, m_tile0 + cc, min(32, p.M - (m_tile0 + cc)), lane);
-          }
-          continue;
-        }
-
-        // ---- split-K over a cluster of S CTAs, reduced as a reduce-scatter through shared
-        // memory: every CTA publishes its fp32 partial tile in its own shared memory; CTA r
-        // then sums all S partials (in rank order) for TMEM lanes [r·128/S, (r+1)·128/S) and
-        // finishes those output columns.
-        {
-          const uint32_t my_row = red_base + (uint32_t)(q * 32 + lane) * p.red_pitch;
+        if (S > 1) {
+#pragma unroll 1
           for (int cc = 0; cc < p.mma_n; cc += 32) {
             uint32_t r[32];
             if (have_acc) {
@@ -833,50 +809,109 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
             mbar_arrive(tempty_bar(buf));
             for (int rk = 0; rk < S; ++rk) mbar_arrive_remote(mapa_shared(red_ready_bar, (uint32_t)rk));
           }
-        }
-        if (!warp_wait_bounded(red_ready_bar, 0, p, lane, true)) ok = false;
-        if (ok) {
-          const int L = 128 / S;             // TMEM lanes this CTA finishes (S is 2 or 4)
-          const int groups = L / 32;         // 32-lane groups among them
-          const int g = ew % groups;
-          const int parts = kEpiWarps / groups;
-          const int part = ew / groups;
-          const int row = (int)rank * L + g * 32 + lane;
-          const int mcnt = p.mma_n / parts;  // a multiple of 8
-          const int mb = part * mcnt;
-          const uint32_t row_addr = red_base + (uint32_t)row * p.red_pitch;
-          for (int mc = mb; mc < mb + mcnt; mc += 32) {
-            const int cnt = min(32, mb + mcnt - mc);
-            // every rank's loads in flight together, then the sum in rank order
-            float v[32];
-            float4 f[4][8];
+          if (!warp_wait_bounded(red_ready_bar, 0, p, lane, true)) ok = false;
+          // sum the S partials of this thread's row (all ranks' loads in flight together,
+          // then the sum in rank order) and write it over this CTA's own copy of the row,
+          // which no peer reads
+          if (ok) {
+#pragma unroll 1
+            for (int mc = mb; mc < mb + mcnt; mc += 32) {
+              const int cnt = min(32, mb + mcnt - mc);
+              float4 f[4][8];
 #pragma unroll
-            for (int rk = 0; rk < 4; ++rk) {
-              const uint32_t a = mapa_shared(row_addr + (uint32_t)mc * 4u, (uint32_t)(rk < S ? rk : 0));
+              for (int rk = 0; rk < 4; ++rk) {
+                const uint32_t a = mapa_shared(sum_row + (uint32_t)mc * 4u, (uint32_t)(rk < S ? rk : 0));
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  f[rk][c] = make_float4(0.f, 0.f, 0.f, 0.f);
+                  if (rk < S && 4 * c < cnt) f[rk][c] = ld_shared_cluster_f4(a + 16u * c);
+                }
+              }
 #pragma unroll
               for (int c = 0; c < 8; ++c) {
-                f[rk][c] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (rk < S && 4 * c < cnt) f[rk][c] = ld_shared_cluster_f4(a + 16u * c);
+                float4 acc = f[0][c];
+#pragma unroll
+                for (int rk = 1; rk < 4; ++rk) {
+                  acc.x += f[rk][c].x;
+                  acc.y += f[rk][c].y;
+                  acc.z += f[rk][c].z;
+                  acc.w += f[rk][c].w;
+                }
+                if (4 * c < cnt) st_shared_f4(sum_row + (uint32_t)(mc + 4 * c) * 4u, acc);
               }
             }
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              float4 acc = f[0][c];
-#pragma unroll
-              for (int rk = 1; rk < 4; ++rk) {
-                acc.x += f[rk][c].x;
-                acc.y += f[rk][c].y;
-                acc.z += f[rk][c].z;
-                acc.w += f[rk][c].w;
-              }
-              v[4 * c] = acc.x;
-              v[4 * c + 1] = acc.y;
-              v[4 * c + 2] = acc.z;
-              v[4 * c + 3] = acc.w;
-            }
-            swap_finish<ACT, OUT>(p, v, ta * 128 + row, ta * 128 + (int)rank * L + g * 32, m_tile0 + mc,
-                                  min(cnt, p.M - (m_tile0 + mc)), lane);
           }
+        }
+
+        // ---- finish: rows in blocks of 32 (residual blocks double-buffered), four rows a trip
+        float bias_n = 0.0f;
+        if (has_bias && p.bias_axis == 0 && n_ok) bias_n = ldg_pinned(p.bias, n, p.bias_dtype);
+        const int res_es = (p.res_dtype == DT_F32) ? 4 : 2;
+        if (ok) {
+#pragma unroll 1
+          for (int bm = 0; bm < rows; bm += 32) {
+            const int cnt = min(32, rows - bm);
+            const uint32_t rcur = rst + (uint32_t)((bm >> 5) & 1) * p.res_blk_bytes;
+            if (res_async) {
+              if (bm + 32 < rows) {
+                stage_residual(p, rst + (uint32_t)(((bm >> 5) + 1) & 1) * p.res_blk_bytes, m_lo + bm + 32,
+                               min(32, rows - bm - 32), n_w0, lane);
+                cp_async_wait<1>();
+              } else {
+                cp_async_wait<0>();
+              }
+              __syncwarp();  // every lane's copies of the block have landed
+            }
+            // lane l holds the bias of row bm + l (bias along M), read back by shuffle
+            float bias_l = 0.0f;
+            if (has_bias && p.bias_axis == 1 && lane < cnt) bias_l = ldg_pinned(p.bias, m_lo + bm + lane, p.bias_dtype);
+#pragma unroll 1
+            for (int j = 0; j < cnt; j += 4) {
+              const int mc = mb + bm + j;  // accumulator column of row m_lo + bm + j
+              float x[4];
+              if (S > 1) {
+                const float4 v = ld_shared_f4(sum_row + (uint32_t)mc * 4u);
+                x[0] = v.x, x[1] = v.y, x[2] = v.z, x[3] = v.w;
+              } else if (have_acc) {
+                uint32_t r[4];
+                tmem_ld4(tacc + (uint32_t)mc, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 4; ++i) x[i] = __uint_as_float(r[i]);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) x[i] = 0.0f;
+              }
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int jj = j + i;
+                if (jj < cnt) {  // uniform across the warp
+                  const int m = m_lo + bm + jj;
+                  float xv = x[i];
+                  if (has_bias) xv += (p.bias_axis == 0) ? bias_n : __shfl_sync(0xffffffffu, bias_l, jj);
+                  float res = 0.0f;
+                  if (res_async) {
+                    const uint32_t ra = rcur + (uint32_t)(jj * 32 + lane) * (uint32_t)res_es;
+                    res = (p.res_dtype == DT_F32) ? __uint_as_float(ld_shared_u32(ra))
+                          : (p.res_dtype == DT_BF16)
+                              ? __uint_as_float((uint32_t)ld_shared_u16(ra) << 16)
+                              : __half2float(__ushort_as_half(ld_shared_u16(ra)));
+                  } else if (has_res && n_ok) {
+                    res = ldg_pinned(p.residual, (long long)m * p.ldr + n, p.res_dtype);
+                  }
+                  swap_store<ACT, OUT>(p, xv, res, m, n, n_ok, n_w0 >> 5, lane);
+                }
+              }
+            }
+            __syncwarp();  // the block's buffer is refilled two blocks later
+          }
+        }
+        if (S == 1) {
+          // this warp's TMEM reads of the buffer are done
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty_bar(buf));
+          continue;
         }
         // nobody leaves while a peer may still read its partial
         __syncwarp();
@@ -885,6 +920,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         if (!warp_wait_bounded(red_done_bar, 0, p, lane, true)) ok = false;
         break;  // a split-K cluster owns exactly one tile
       }
+      cp_async_wait<0>();  // no copy into shared memory outlives the loop
     }
     (void)ok;
     __syncwarp();
