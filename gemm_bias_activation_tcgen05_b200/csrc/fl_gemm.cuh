@@ -43,11 +43,11 @@ constexpr int kUmmaSteps = 4;                 // UMMA instructions per 128-byte 
 constexpr int kMaxSteps = 8;                  // at most two atoms per stage
 constexpr int kErrTimeout = 1;
 
-// Normal layout: 8 epilogue warps (two per TMEM lane quarter, one per column
-// half).  Swap-AB layout: 4 epilogue warps (one per lane quarter).
+// 8 epilogue warps, two per TMEM lane quarter (the normal layout gives each a
+// column half of the tile; the swap-AB layout a share of the rows).
 template <bool SWAP>
 struct Cfg {
-  static constexpr int kEpiWarps = SWAP ? 4 : 8;
+  static constexpr int kEpiWarps = 8;
   static constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
   static constexpr uint32_t kStagingBytes = SWAP ? 0u : kEpiWarps * kStagingBuf;
 };
@@ -309,19 +309,6 @@ __device__ __forceinline__ void stage_residual(const KParams& p, uint32_t dst, i
     cp_async_16(dst + (uint32_t)(r * 32 * es + k * 16), src, (uint32_t)bytes);
   }
   cp_async_commit();
-}
-
-// Swap-AB epilogue for one output element: lane = column n, row m, pre-activation
-// x (bias already added).  The mask word of row m is one ballot of the warp.
-template <int ACT, int OUT>
-__device__ __forceinline__ void swap_store(const KParams& p, float x, float res, int m, int n, bool n_ok, int wcol,
-                                           int lane) {
-  if (p.aux != nullptr) {
-    const uint32_t word = __ballot_sync(0xffffffffu, n_ok && x > 0.0f);
-    if (lane == 0 && (long long)wcol * 32 < p.N) p.aux[(long long)m * p.ld_aux + wcol] = word;
-  }
-  const float y = (activate<ACT>(x, 0.0f) + res) * p.scale;
-  if (n_ok) store_elem<OUT>(p.out, (long long)m * p.ldo + n, y);
 }
 
 // ------------------------------------------------------------------ kernel
@@ -754,29 +741,32 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
       // Split-K (S > 1): every CTA publishes its fp32 partial tile in its own shared
       // memory; CTA r then sums the S partials (in rank order) of TMEM lanes
       // [r·128/S, (r+1)·128/S) and finishes those output columns.  Warp ew owns 32
-      // of those lanes and a contiguous range of rows.  The finishing loop is kept
-      // rolled (four rows a trip): it runs once per CTA, so its instructions come
-      // from L2, and a short loop body keeps that fetch small.
+      // of those lanes and a range of rows.  The finishing loop stays rolled (eight
+      // independent rows a trip): it runs once per CTA, so its instructions come
+      // from L2, and a short body keeps that fetch small.
       const uint32_t red_base = smem_base + p.red_off;
       const int L = 128 / S;
       const int groups = L / 32;
-      const int g = (S == 1) ? q : ew % groups;          // S = 1: a warp finishes its own TMEM quarter
+      const int g = (S == 1) ? q : ew % groups;           // S = 1: a warp finishes a lane quarter it may read
       const int parts = kEpiWarps / groups;
-      const int part = (S == 1) ? 0 : ew / groups;
-      const int lrow = (int)rank * L + g * 32 + lane;    // TMEM lane = column within the tile
-      const int mcnt = p.mma_n / parts;                  // a multiple of 8
+      const int part = (S == 1) ? (ew >> 2) : ew / groups;
+      const int lrow = (int)rank * L + g * 32 + lane;     // TMEM lane = column within the tile
+      const int mcnt = ((p.mma_n + parts - 1) / parts + 7) & ~7;  // rows per warp, a multiple of 8
       const int mb = part * mcnt;
+      const int mlen = max(0, min(mcnt, p.mma_n - mb));   // accumulator columns of this warp
       const uint32_t my_row = red_base + (uint32_t)(q * 32 + lane) * p.red_pitch;  // published row
       const uint32_t sum_row = red_base + (uint32_t)lrow * p.red_pitch;            // finished row
       const uint32_t rst = smem_base + p.res_off + (uint32_t)ew * 2u * p.res_blk_bytes;
       const bool res_async = has_res && p.res_async;
+      const int res_es = (p.res_dtype == DT_F32) ? 4 : 2;
+      constexpr int eo = (OUT == DT_F32) ? 4 : 2;
       for (int t = cluster_id; t < total_tiles; t += num_clusters, ++local) {
         int ta, tb;
         tile_coords(t, p, ta, tb);
         const uint32_t buf = local & 1u;
         const uint32_t tph = (local >> 1) & 1u;
-        const int m_lo = tb * p.mma_n + mb;                // first output row of this warp
-        const int rows = max(0, min(mcnt, p.M - m_lo));
+        const int m_lo = tb * p.mma_n + mb;                 // first output row of this warp
+        const int rows = max(0, min(mlen, p.M - m_lo));
         const int n_w0 = ta * 128 + (int)rank * L + g * 32;
         const int n = n_w0 + lane;
         const bool n_ok = n < p.N;
@@ -787,8 +777,9 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
 
         if (S > 1) {
+          // the two warps of a lane quarter publish alternate 32-column chunks
 #pragma unroll 1
-          for (int cc = 0; cc < p.mma_n; cc += 32) {
+          for (int cc = (ew >> 2) * 32; cc < p.mma_n; cc += 64) {
             uint32_t r[32];
             if (have_acc) {
               tmem_ld32(tacc + (uint32_t)cc, r);
@@ -810,43 +801,53 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
             for (int rk = 0; rk < S; ++rk) mbar_arrive_remote(mapa_shared(red_ready_bar, (uint32_t)rk));
           }
           if (!warp_wait_bounded(red_ready_bar, 0, p, lane, true)) ok = false;
-          // sum the S partials of this thread's row (all ranks' loads in flight together,
-          // then the sum in rank order) and write it over this CTA's own copy of the row,
-          // which no peer reads
-          if (ok) {
+          // Sum the S partials of this CTA's slice (rows [rank·L, rank·L + L) of every CTA's
+          // buffer, contiguous) in rank order and write the sums over this CTA's own copy,
+          // which no peer reads.  The eight epilogue warps stream the slice in 16-byte
+          // pieces, so every warp-wide load from a peer is 512 contiguous bytes.
+          {
+            const uint32_t slice = red_base + (uint32_t)(rank * L) * p.red_pitch;
+            const uint32_t bytes = (uint32_t)L * p.red_pitch;
+            constexpr uint32_t kStep = kEpiWarps * 32u * 16u;
+            uint32_t peer[4];
+#pragma unroll
+            for (int rk = 0; rk < 4; ++rk) peer[rk] = mapa_shared(slice, (uint32_t)(rk < S ? rk : 0));
+            if (ok) {
 #pragma unroll 1
-            for (int mc = mb; mc < mb + mcnt; mc += 32) {
-              const int cnt = min(32, mb + mcnt - mc);
-              float4 f[4][8];
+              for (uint32_t o = (uint32_t)(ew * 32 + lane) * 16u; o < bytes; o += 4u * kStep) {
+                float4 f[4][4];
 #pragma unroll
-              for (int rk = 0; rk < 4; ++rk) {
-                const uint32_t a = mapa_shared(sum_row + (uint32_t)mc * 4u, (uint32_t)(rk < S ? rk : 0));
+                for (int u = 0; u < 4; ++u)
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                  f[rk][c] = make_float4(0.f, 0.f, 0.f, 0.f);
-                  if (rk < S && 4 * c < cnt) f[rk][c] = ld_shared_cluster_f4(a + 16u * c);
+                  for (int rk = 0; rk < 4; ++rk) {
+                    f[u][rk] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (rk < S && o + u * kStep < bytes) f[u][rk] = ld_shared_cluster_f4(peer[rk] + o + u * kStep);
+                  }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  float4 acc = f[u][0];
+#pragma unroll
+                  for (int rk = 1; rk < 4; ++rk) {
+                    acc.x += f[u][rk].x;
+                    acc.y += f[u][rk].y;
+                    acc.z += f[u][rk].z;
+                    acc.w += f[u][rk].w;
+                  }
+                  if (o + u * kStep < bytes) st_shared_f4(slice + o + u * kStep, acc);
                 }
-              }
-#pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                float4 acc = f[0][c];
-#pragma unroll
-                for (int rk = 1; rk < 4; ++rk) {
-                  acc.x += f[rk][c].x;
-                  acc.y += f[rk][c].y;
-                  acc.z += f[rk][c].z;
-                  acc.w += f[rk][c].w;
-                }
-                if (4 * c < cnt) st_shared_f4(sum_row + (uint32_t)(mc + 4 * c) * 4u, acc);
               }
             }
+            // every warp's sums are in place before any warp finishes rows
+            asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
           }
         }
 
-        // ---- finish: rows in blocks of 32 (residual blocks double-buffered), four rows a trip
+        // ---- finish: rows in blocks of 32 (residual blocks double-buffered), eight rows a
+        // trip.  Rows past the warp's count are computed from valid (stale) shared memory and
+        // never stored.
         float bias_n = 0.0f;
         if (has_bias && p.bias_axis == 0 && n_ok) bias_n = ldg_pinned(p.bias, n, p.bias_dtype);
-        const int res_es = (p.res_dtype == DT_F32) ? 4 : 2;
+        const float scale_v = p.scale;
         if (ok) {
 #pragma unroll 1
           for (int bm = 0; bm < rows; bm += 32) {
@@ -866,40 +867,64 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
             float bias_l = 0.0f;
             if (has_bias && p.bias_axis == 1 && lane < cnt) bias_l = ldg_pinned(p.bias, m_lo + bm + lane, p.bias_dtype);
 #pragma unroll 1
-            for (int j = 0; j < cnt; j += 4) {
+            for (int j = 0; j < cnt; j += 8) {
               const int mc = mb + bm + j;  // accumulator column of row m_lo + bm + j
-              float x[4];
+              float x[8];
               if (S > 1) {
-                const float4 v = ld_shared_f4(sum_row + (uint32_t)mc * 4u);
-                x[0] = v.x, x[1] = v.y, x[2] = v.z, x[3] = v.w;
+                const float4 v0 = ld_shared_f4(sum_row + (uint32_t)mc * 4u);
+                const float4 v1 = ld_shared_f4(sum_row + (uint32_t)mc * 4u + 16u);
+                x[0] = v0.x, x[1] = v0.y, x[2] = v0.z, x[3] = v0.w;
+                x[4] = v1.x, x[5] = v1.y, x[6] = v1.z, x[7] = v1.w;
               } else if (have_acc) {
-                uint32_t r[4];
-                tmem_ld4(tacc + (uint32_t)mc, r);
+                uint32_t r0[4], r1[4];
+                tmem_ld4(tacc + (uint32_t)mc, r0);
+                tmem_ld4(tacc + (uint32_t)mc + 4u, r1);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 4; ++i) x[i] = __uint_as_float(r[i]);
+                for (int i = 0; i < 4; ++i) x[i] = __uint_as_float(r0[i]), x[4 + i] = __uint_as_float(r1[i]);
               } else {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) x[i] = 0.0f;
+                for (int i = 0; i < 8; ++i) x[i] = 0.0f;
               }
+              float rv[8];
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int jj = j + i;
-                if (jj < cnt) {  // uniform across the warp
-                  const int m = m_lo + bm + jj;
-                  float xv = x[i];
-                  if (has_bias) xv += (p.bias_axis == 0) ? bias_n : __shfl_sync(0xffffffffu, bias_l, jj);
-                  float res = 0.0f;
-                  if (res_async) {
-                    const uint32_t ra = rcur + (uint32_t)(jj * 32 + lane) * (uint32_t)res_es;
-                    res = (p.res_dtype == DT_F32) ? __uint_as_float(ld_shared_u32(ra))
-                          : (p.res_dtype == DT_BF16)
-                              ? __uint_as_float((uint32_t)ld_shared_u16(ra) << 16)
-                              : __half2float(__ushort_as_half(ld_shared_u16(ra)));
-                  } else if (has_res && n_ok) {
-                    res = ldg_pinned(p.residual, (long long)m * p.ldr + n, p.res_dtype);
-                  }
-                  swap_store<ACT, OUT>(p, xv, res, m, n, n_ok, n_w0 >> 5, lane);
+              for (int i = 0; i < 8; ++i) rv[i] = 0.0f;
+              if (res_async) {
+                const uint32_t ra = rcur + (uint32_t)(j * 32 + lane) * (uint32_t)res_es;
+                if (res_es == 4) {
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) rv[i] = __uint_as_float(ld_shared_u32(ra + (uint32_t)i * 128u));
+                } else if (p.res_dtype == DT_BF16) {
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) rv[i] = __uint_as_float((uint32_t)ld_shared_u16(ra + (uint32_t)i * 64u) << 16);
+                } else {
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) rv[i] = __half2float(__ushort_as_half(ld_shared_u16(ra + (uint32_t)i * 64u)));
+                }
+              } else if (has_res && n_ok) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                  if (j + i < cnt) rv[i] = ldg_pinned(p.residual, (long long)(m_lo + bm + j + i) * p.ldr + n, p.res_dtype);
+              }
+              const long long row0 = (long long)(m_lo + bm + j);
+              char* orow = reinterpret_cast<char*>(p.out) + (row0 * p.ldo + n) * eo;
+              const long long ostep = p.ldo * eo;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                float xv = x[i];
+                if (has_bias) xv += (p.bias_axis == 0) ? bias_n : __shfl_sync(0xffffffffu, bias_l, (j + i) & 31);
+                if (has_aux) {
+                  const uint32_t word = __ballot_sync(0xffffffffu, n_ok && xv > 0.0f);
+                  const int wcol = n_w0 >> 5;
+                  if (lane == 0 && j + i < cnt && (long long)wcol * 32 < p.N)
+                    p.aux[(row0 + i) * p.ld_aux + wcol] = word;
+                }
+                const float y = (activate<ACT>(xv, 0.0f) + rv[i]) * scale_v;
+                if (n_ok && j + i < cnt) {
+                  char* dst = orow + i * ostep;
+                  if constexpr (OUT == DT_F32) *reinterpret_cast<float*>(dst) = y;
+                  else if constexpr (OUT == DT_BF16) *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(y);
+                  else *reinterpret_cast<__half*>(dst) = __float2half_rn(y);
                 }
               }
             }
