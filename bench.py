@@ -251,9 +251,11 @@ def run_ours(args):
     torch.cuda.synchronize()
     suite.check()
 
-    # ---- timed region: K steps, per-launch events on the launching stream.  The K
-    # steps are captured once as a CUDA graph (launches + event-record nodes), so
-    # the timed replay has no host enqueue gaps between the launches.
+    # ---- timed region: K steps captured once as a CUDA graph, so the replay has no
+    # host enqueue gaps between launches; the kernels are launched with programmatic
+    # dependent launch, so a kernel's prologue overlaps its predecessor's tail.
+    # Per-workload times come from a second graph with an event pair around every
+    # workload (an event node between two kernels serialises them fully).
     n_items = len(suite.items)
     use_graph = not args.no_graph
     ev = [[(torch.cuda.Event(enable_timing=True, external=use_graph),
@@ -261,18 +263,22 @@ def run_ours(args):
           for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-    def k_steps(stream_handle):
+    def k_steps(stream_handle, with_events):
         for s in range(args.steps):
             for i, it in enumerate(suite.items):
-                ev[s][i][0].record()
+                if with_events:
+                    ev[s][i][0].record()
                 suite.run_item(it, stream_handle)
-                ev[s][i][1].record()
+                if with_events:
+                    ev[s][i][1].record()
 
-    graph = None
+    graph = ev_graph = None
     if use_graph:
-        graph = torch.cuda.CUDAGraph()
+        graph, ev_graph = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
-            k_steps(torch.cuda.current_stream().cuda_stream)
+            k_steps(torch.cuda.current_stream().cuda_stream, False)
+        with torch.cuda.graph(ev_graph):
+            k_steps(torch.cuda.current_stream().cuda_stream, True)
         graph.replay()  # one untimed replay of the captured steps
         torch.cuda.synchronize()
     barrier(ws)
@@ -282,13 +288,19 @@ def run_ours(args):
         if graph is not None:
             graph.replay()
         else:
-            k_steps(sh)
+            k_steps(sh, False)
         t1.record(stream)
         torch.cuda.synchronize()
     barrier(ws)
     total_ms = max_over_ranks(t0.elapsed_time(t1), ws)
     suite.check()
     ms_step = total_ms / args.steps
+    # per-workload breakdown (outside the timed region)
+    if ev_graph is not None:
+        ev_graph.replay()
+    else:
+        k_steps(sh, True)
+    torch.cuda.synchronize()
     per_item = {}
     for i, it in enumerate(suite.items):
         times = [ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)]
@@ -344,7 +356,7 @@ def run_ours(args):
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph
+    del graph, ev_graph
     torch.cuda.synchronize()
     for it in suite.items:
         for p in it["plans"]:

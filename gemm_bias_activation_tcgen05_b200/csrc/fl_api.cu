@@ -510,6 +510,22 @@ struct GemmArgs {
   bool geglu_fused;
 };
 
+// Launch an elementwise kernel with programmatic dependent launch allowed.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 static fl_status launch_kernel(const fl_plan_s* p, const LaunchCache& c, cudaStream_t stream,
                                const void* kernel, bool swap) {
   cudaLaunchConfig_t cfg{};
@@ -517,15 +533,22 @@ static fl_status launch_kernel(const fl_plan_s* p, const LaunchCache& c, cudaStr
   cfg.blockDim = dim3(swap ? Cfg<true>::kThreads : Cfg<false>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)p->smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
+  unsigned na = 0;
+  // programmatic dependent launch: the kernel's prologue may overlap the tail of
+  // the previous kernel of the stream (the kernel waits before touching memory)
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
   if (p->split_k > 1 || p->pair) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = p->pair ? 2u : (unsigned)p->split_k;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = p->pair ? 2u : (unsigned)p->split_k;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
   }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
   cudaError_t err = cudaLaunchKernelEx(&cfg, reinterpret_cast<KernelFn>(const_cast<void*>(kernel)), c.tmA, c.tmB,
                                        c.tmB2, c.tmOut, c.k);
   if (err != cudaSuccess) return fail(FL_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(err));
@@ -666,7 +689,8 @@ static int grid_for(long long work, int num_sms) {
 template <int DT>
 static fl_status launch_ew_t(const EwParams& P, int num_sms, cudaStream_t s) {
   const long long work = P.M * ((P.N + 31) / 32);
-  fl_ew_step_kernel<DT><<<grid_for(work, num_sms), 256, 0, s>>>(P);
+  const cudaError_t err = launch_pdl(fl_ew_step_kernel<DT>, (unsigned)grid_for(work, num_sms), s, P);
+  if (err != cudaSuccess) return fail(FL_ERR_CUDA, "elementwise kernel launch: %s", cudaGetErrorString(err));
   return after_launch(s, "elementwise step kernel");
 }
 static fl_status launch_ew(int dt, const EwParams& P, int num_sms, cudaStream_t s) {
@@ -826,12 +850,17 @@ extern "C" fl_status fl_relu_backward(const void* grad, const uint32_t* aux, voi
   const long long work = M * words;
   const int grid = grid_for(work, sms);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+  cudaError_t err;
   if (dtype == FL_BF16)
-    fl_relu_backward_kernel<DT_BF16><<<grid, 256, 0, s>>>(grad, aux, dpre, M, N, ld_grad, ld_dpre, words, vec_ok);
+    err = launch_pdl(fl_relu_backward_kernel<DT_BF16>, (unsigned)grid, s, grad, aux, dpre, (long long)M, (long long)N,
+                     (long long)ld_grad, (long long)ld_dpre, words, vec_ok);
   else if (dtype == FL_F16)
-    fl_relu_backward_kernel<DT_F16><<<grid, 256, 0, s>>>(grad, aux, dpre, M, N, ld_grad, ld_dpre, words, vec_ok);
+    err = launch_pdl(fl_relu_backward_kernel<DT_F16>, (unsigned)grid, s, grad, aux, dpre, (long long)M, (long long)N,
+                     (long long)ld_grad, (long long)ld_dpre, words, vec_ok);
   else
-    fl_relu_backward_kernel<DT_F32><<<grid, 256, 0, s>>>(grad, aux, dpre, M, N, ld_grad, ld_dpre, words, vec_ok);
+    err = launch_pdl(fl_relu_backward_kernel<DT_F32>, (unsigned)grid, s, grad, aux, dpre, (long long)M, (long long)N,
+                     (long long)ld_grad, (long long)ld_dpre, words, vec_ok);
+  if (err != cudaSuccess) return fail(FL_ERR_CUDA, "dReLU kernel launch: %s", cudaGetErrorString(err));
   return after_launch(s, "dReLU kernel");
 }
 

@@ -40,6 +40,8 @@ __global__ void __launch_bounds__(256) fl_relu_backward_kernel(const void* __res
                                                                long long ldd, long long words,
                                                                int vec_ok) {
   using T = typename ElemT<DT>::T;
+  grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
   constexpr int ESZ = sizeof(T);
   constexpr int PER16 = 16 / ESZ;  // elements per 16-byte vector
   const T* grad = reinterpret_cast<const T*>(grad_);
@@ -144,6 +146,8 @@ __device__ __forceinline__ void ew_st(void* p, long long i, float v) {
 // Storage dtype DT for src/dst (the eager tensors); operands use their own dtype.
 template <int DT>
 __global__ void __launch_bounds__(256) fl_ew_step_kernel(const EwParams P) {
+  grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
   const long long words = (P.N + 31) / 32;
   const long long total = P.M * words;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;

@@ -388,6 +388,10 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (S > 1 || PAIR) cluster_sync_all();  // peers' barriers are initialised before any remote arrive
+  // Programmatic dependent launch: the prologue above may overlap the previous
+  // kernel of the stream; no global memory is touched before this wait.
+  grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(
       __cvta_shared_to_generic(tmem_slot));
 

@@ -257,6 +257,14 @@ __device__ __forceinline__ float tanh_approx(float x) {
 }
 
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Wait until every grid this one depends on has completed and its memory is
+// visible (returns at once when the launch has no such dependency).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel of the stream start its prologue; it still waits (above)
+// for this grid to complete before it touches memory.
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ cp.async (global -> shared)
 // 16-byte copy; only the first src_bytes (0..16) are read, the rest of the
 // 16 bytes is zero-filled.  Both addresses must be 16-byte aligned.
