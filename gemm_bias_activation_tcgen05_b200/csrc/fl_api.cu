@@ -122,6 +122,21 @@ static const void* pick_tf32(int out) {
   if (out == FL_F16) return reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, DT_F16, false, true>);
   return reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, DT_F32, false, true>);
 }
+template <int ACT>
+static const void* pick_tf32_pair(int out) {
+  if (out == FL_BF16) return reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, DT_BF16, false, true, true>);
+  if (out == FL_F16) return reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, DT_F16, false, true, true>);
+  return reinterpret_cast<const void*>(&fl_gemm_epi_tcgen05<ACT, DT_F32, false, true, true>);
+}
+static const void* pick_kernel_tf32_pair(int act, int out) {
+  switch (act) {
+    case ACT_NONE: return pick_tf32_pair<ACT_NONE>(out);
+    case ACT_RELU: return pick_tf32_pair<ACT_RELU>(out);
+    case ACT_GELU: return pick_tf32_pair<ACT_GELU>(out);
+    case ACT_GELU_TANH: return pick_tf32_pair<ACT_GELU_TANH>(out);
+    default: return nullptr;
+  }
+}
 static const void* pick_kernel_tf32(int act, int out) {
   switch (act) {
     case ACT_NONE: return pick_tf32<ACT_NONE>(out);
@@ -219,6 +234,7 @@ struct Layout {
   int stages;
 };
 
+constexpr int kMaxStages = 12;
 static Layout layout_for(const fl_plan_s* p, int mma_n, int b_boxes, int max_smem) {
   Layout L{};
   const int es = esize(p->dtype);
@@ -238,20 +254,25 @@ static Layout layout_for(const fl_plan_s* p, int mma_n, int b_boxes, int max_sme
   L.stride = (p->dtype == FL_F32) ? 2u * L.stage : L.stage;
   const uint32_t staging = p->swap ? Cfg<true>::kStagingBytes : Cfg<false>::kStagingBytes;
   const uint32_t bias = 0;
+  // Split-K partial tiles (swap-AB, S > 1): a split-K cluster owns one tile, so the
+  // partials are published after the last UMMA has read the last stage and can
+  // reuse the stage memory.
   const uint32_t red = (p->swap && p->split_k > 1) ? 128u * ((uint32_t)mma_n * 4u + 16u) : 0u;
   // swap-AB with a residual: two 32-row x 32-column residual blocks per epilogue warp
   L.res_blk = 32u * 32u * (uint32_t)esize(p->epi.residual_dtype);
   const uint32_t res = (p->swap && p->epi.has_residual) ? (uint32_t)Cfg<true>::kEpiWarps * 2u * L.res_blk : 0u;
-  const uint32_t bars = 8u * (3u * 8u + 8u);
-  const uint32_t budget = (uint32_t)max_smem - 1024u - staging - bias - red - res - bars;
+  const uint32_t bars = 8u * (3u * (uint32_t)kMaxStages + 8u);
+  const uint32_t budget = (uint32_t)max_smem - 1024u - staging - bias - res - bars;
   int st = (int)(budget / L.stride);
-  if (st > 8) st = 8;
+  if (st > kMaxStages) st = kMaxStages;
+  if (red > budget) st = 0;  // reported as "shared memory too small"
   L.stages = st;
-  L.staging_off = (uint32_t)st * L.stride;
+  const uint32_t stage_area = std::max((uint32_t)st * L.stride, red);
+  L.staging_off = stage_area;
   L.bias_off = L.staging_off + staging;
-  L.red_off = L.bias_off + bias;
+  L.red_off = 0;
   L.red_pitch = (uint32_t)mma_n * 4u + 16u;
-  L.res_off = L.red_off + red;
+  L.res_off = L.bias_off + bias;
   L.bar_off = L.res_off + res;
   L.total = L.bar_off + 8u * (3u * (uint32_t)st + 8u) + 1024u;
   return L;
@@ -271,7 +292,7 @@ static int grid_of(const fl_plan_s* p) {
   return std::min(tiles, p->num_sms);
 }
 static const void* kernel_of(const fl_plan_s* p, int act, int out) {
-  if (p->dtype == FL_F32) return pick_kernel_tf32(act, out);
+  if (p->dtype == FL_F32) return p->pair ? pick_kernel_tf32_pair(act, out) : pick_kernel_tf32(act, out);
   if (p->pair) return pick_kernel_pair(act, out);
   return pick_kernel(act, out, p->swap);
 }
@@ -284,10 +305,11 @@ static fl_status choose_config(fl_plan_s* p) {
   // Small M: put the weight on the 128-row side of the tensor core (swap-AB)
   // and split K across a cluster so that every SM streams a slice of W.
   p->swap = (M <= 128) && !geglu && !p->epi.b_major && p->dtype != FL_F32;
-  // CTA pairs take 128-deep K stages (two swizzle atoms, eight UMMA steps per
-  // barrier round trip); the other layouts keep one atom per stage.
-  p->pair = !p->swap && p->dtype != FL_F32 && M > 128;
-  p->k_atoms = p->pair ? 2 : 1;
+  // Beyond one 128-row tile: CTA pairs with 256-row UMMA tiles.  16-bit pairs take
+  // 128-deep K stages (two swizzle atoms, eight UMMA steps per barrier round trip);
+  // the other layouts keep one atom per stage (a 3xTF32 stage also holds lo halves).
+  p->pair = !p->swap && M > 128;
+  p->k_atoms = (p->pair && p->dtype != FL_F32) ? 2 : 1;
   p->num_kb = (int)cdiv(p->K, (int64_t)p->k_atoms * 128 / es);
   if (p->swap) {
     // The epilogue moves TMEM in 32-column chunks, so the activation tile is a multiple of 32.
@@ -303,15 +325,30 @@ static fl_status choose_config(fl_plan_s* p) {
     p->split_k = S;
   } else {
     p->split_k = 1;
-    // 16-bit operands beyond one 128-row tile: CTA pairs with 256-row UMMA tiles
     const int rows = p->pair ? 256 : 128;
     const int units = p->pair ? p->num_sms / 2 : p->num_sms;
     if (geglu) {
       p->mma_n = 256;
       p->out_tile_n = 128;
-    } else if (p->dtype == FL_F32) {
+    } else if (p->dtype == FL_F32 && !p->pair) {
       p->mma_n = 128;  // a 3xTF32 stage holds hi and lo tiles: 128 wide keeps three stages
       p->out_tile_n = 128;
+    } else if (p->dtype == FL_F32) {
+      // 3xTF32 pairs: the UMMA reads half of B from each CTA, halving the shared-memory
+      // operand traffic per FLOP, which bounds this path.  Each epilogue warp covers
+      // half the tile in chunks of 32 (fp32 out) or 64 (16-bit out) columns.
+      const bool narrow_ok = esize(p->epi.out_dtype) == 4;
+      int best = 256;
+      double best_cost = 1e300;
+      for (int bn : {256, 192, 128}) {
+        if (bn == 192 && !narrow_ok) continue;
+        const int64_t tiles = cdiv(M, rows) * cdiv(N, bn);
+        const double waves = (double)cdiv(tiles, units);
+        const double cost = waves * bn * (bn == 128 ? 1.3 : 1.0);
+        if (cost < best_cost) { best_cost = cost; best = bn; }
+      }
+      p->mma_n = best;
+      p->out_tile_n = best;
     } else {
       // Pick the N tile that minimises (waves x tile width) on this GPU.
       // Cost ~ (rounds of tiles per SM) x (tile width) x (relative cost per column):
@@ -439,7 +476,8 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
   if (epi->unfused) {
     // the bare GEMM kernels of both layouts may serve this plan's first step
     for (int sw = 0; sw < 3; ++sw) {
-      const void* kn = (dtype == FL_F32) ? pick_kernel_tf32(ACT_NONE, epi->out_dtype)
+      const void* kn = (dtype == FL_F32) ? (sw == 2 ? pick_kernel_tf32_pair(ACT_NONE, epi->out_dtype)
+                                                    : pick_kernel_tf32(ACT_NONE, epi->out_dtype))
                        : (sw == 2 ? pick_kernel_pair(ACT_NONE, epi->out_dtype)
                                   : pick_kernel(ACT_NONE, epi->out_dtype, sw == 1));
       if (cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, p->max_smem) != cudaSuccess) {

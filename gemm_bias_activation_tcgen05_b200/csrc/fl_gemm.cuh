@@ -365,8 +365,8 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
     // release covers the whole warp's shared-memory writes)
     mbar_init(red_ready_bar, kEpiWarps * S);
     mbar_init(red_done_bar, kEpiWarps * S);
-    if (TF32)
-      for (int s = 0; s < NS; ++s) mbar_init(conv_bar(s), kEpiWarps);
+    if (TF32)  // PAIR: both CTAs' converters arrive on the leader's barrier
+      for (int s = 0; s < NS; ++s) mbar_init(conv_bar(s), kEpiWarps * kCl);
     fence_mbarrier_init();
     if (p.num_kb > 0) {  // with K = 0 the operand maps are left unencoded and never used
       prefetch_tensormap(&tmA);
@@ -415,7 +415,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           const uint32_t sb = sa + p.a_stage_bytes;
           const int k0 = kb * p.bk;
           const int ae = p.bk / p.k_atoms;  // K elements of one 128-byte atom
-          if constexpr (PAIR) {
+          if constexpr (PAIR && !TF32) {
             // both CTAs' bytes complete on the leader's full barrier
             const uint32_t fb = mapa_shared(full_bar(s), 0);
             if (rank == 0) mbar_arrive_expect_tx(full_bar(s), 2u * p.stage_bytes);
@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
       // In the normal path these have all completed already.  A pair's peer
       // counts its bytes on the leader's barriers, which the leader waits for; the
       // final cluster barrier keeps the peer resident until then.
-      for (uint32_t s = 0; (!PAIR || rank == 0) && s < (uint32_t)NS && s < it; ++s) {
+      for (uint32_t s = 0; (!PAIR || TF32 || rank == 0) && s < (uint32_t)NS && s < it; ++s) {
         const uint32_t last = it - 1u - ((it - 1u - s) % (uint32_t)NS);
         (void)wait_bounded(full_bar((int)s), (last / (uint32_t)NS) & 1u, p);
       }
@@ -492,7 +492,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
           const int s = (int)(it % (uint32_t)NS);
           const uint32_t ph = (it / (uint32_t)NS) & 1u;
-          if (!wait_bounded(TF32 ? conv_bar(s) : full_bar(s), ph, p)) { ok = false; break; }
+          if (!wait_bounded(TF32 ? conv_bar(s) : full_bar(s), ph, p, TF32 && PAIR)) { ok = false; break; }
           tc_fence_after();
           const uint64_t da = da0 + (uint64_t)s * stage_step;
           const uint64_t db = db0 + (uint64_t)s * stage_step;
@@ -501,9 +501,15 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
             const uint64_t dbl = dbl0 + (uint64_t)s * stage_step;
 #pragma unroll
             for (int k = 0; k < kUmmaSteps; ++k) {
-              umma_tf32(d_tmem, dal + k * ak, db + k * bk, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
-              umma_tf32(d_tmem, da + k * ak, dbl + k * bk, idesc, 1u);
-              umma_tf32(d_tmem, da + k * ak, db + k * bk, idesc, 1u);
+              if constexpr (PAIR) {
+                umma_tf32_pair(d_tmem, dal + k * ak, db + k * bk, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
+                umma_tf32_pair(d_tmem, da + k * ak, dbl + k * bk, idesc, 1u);
+                umma_tf32_pair(d_tmem, da + k * ak, db + k * bk, idesc, 1u);
+              } else {
+                umma_tf32(d_tmem, dal + k * ak, db + k * bk, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
+                umma_tf32(d_tmem, da + k * ak, dbl + k * bk, idesc, 1u);
+                umma_tf32(d_tmem, da + k * ak, db + k * bk, idesc, 1u);
+              }
             }
           } else if constexpr (PAIR) {
 #pragma unroll
@@ -596,7 +602,11 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
             }
             fence_proxy_async_smem();  // the tensor core reads these through the async proxy
             __syncwarp();
-            if (lane == 0) mbar_arrive(conv_bar(s));
+            if (lane == 0) {
+              // a pair's UMMA is issued by the leader: both CTAs' halves must be split
+              if (PAIR && rank != 0) mbar_arrive_remote(mapa_shared(conv_bar(s), 0));
+              else mbar_arrive(conv_bar(s));
+            }
           }
           if (!ok) break;
         }

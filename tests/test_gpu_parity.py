@@ -175,6 +175,8 @@ def _run_workload_linear(fl, w, seed=0, rows=256):
 def test_fp32_operands_3xtf32(fl, M, N, K, epilogue, out_dtype):
     got = _linear_case(fl, M, N, K, dtype="f32", epilogue=epilogue, out_dtype=out_dtype, seed=13)
     assert got["info"]["swap_ab"] == 0
+    # beyond one 128-row tile the 3xTF32 UMMA runs on CTA pairs
+    assert got["info"]["cta_pair"] == (1 if M > 128 else 0)
 
 
 def test_fp32_residual_scale(fl):
