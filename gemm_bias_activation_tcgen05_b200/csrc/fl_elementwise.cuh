@@ -185,10 +185,10 @@ __global__ void __launch_bounds__(256) fl_ew_step_kernel(const EwParams P) {
           if (x > 0.0f) mask |= 1u << j;
           break;
         case EW_GELU: y = gelu_erf_f(x); break;
-        case EW_GELU_TANH: y = gelu_tanh_f(x); break;
+        case EW_GELU_TANH: y = gelu_tanh_f<DT != DT_F32>(x); break;
         case EW_RESIDUAL: y = x + opv; break;
         case EW_SCALE: y = x * P.scale; break;
-        default: y = gelu_tanh_f(x) * opv; break;
+        default: y = gelu_tanh_f<DT != DT_F32>(x) * opv; break;
       }
       const long long id = m * P.ldd + n;
       if (ew_in(id, P.dst_elems, P.err, code)) ew_st<DT>(P.dst, id, y);

@@ -144,20 +144,48 @@ __device__ __forceinline__ void store_elem(void* p, long long i, float v) {
   }
 }
 
-__device__ __forceinline__ float gelu_erf_f(float x) {
-  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+// erf by Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
+// with t = 1/(1 + p|x|), erf(|x|) = 1 - t(a1 + t(a2 + t(a3 + t(a4 + t·a5))))·e^(-x²),
+// absolute error at most 1.5e-7; erf is odd.  e^(-x²) and 1/(1 + p|x|) come from the
+// special-function unit (relative errors near 2^-22), which keeps the total error
+// near 2e-7, far inside the fp32 tolerance of the layer.
+__device__ __forceinline__ float erf_as(float x) {
+  const float ax = fabsf(x);
+  const float t = rcp_approx(fmaf(0.3275911f, ax, 1.0f));
+  float q = fmaf(1.061405429f, t, -1.453152027f);
+  q = fmaf(q, t, 1.421413741f);
+  q = fmaf(q, t, -0.284496736f);
+  q = fmaf(q, t, 0.254829592f);
+  q *= t;
+  const float e = ex2_approx(-(ax * ax) * 1.4426950408889634f);  // e^(-x²)
+  return copysignf(fmaf(-q, e, 1.0f), x);
 }
-__device__ __forceinline__ float gelu_tanh_f(float x) {
-  const float u = 0.79788456080286536f * (x + 0.044715f * x * x * x);
-  return 0.5f * x * (1.0f + tanhf(u));
+// tanh(u) = 1 - 2/(e^(2u) + 1): saturates to ±1 exactly (e^(2u) = inf or 0), absolute
+// error near 2^-22 elsewhere.
+__device__ __forceinline__ float tanh_ex2(float u) {
+  const float e = ex2_approx(u * 2.8853900817779268f);  // e^(2u)
+  return fmaf(-2.0f, rcp_approx(e + 1.0f), 1.0f);
 }
 
-template <int ACT>
+// GELU(x) = x·Φ(x) = x/2·(1 + erf(x/√2))
+__device__ __forceinline__ float gelu_erf_f(float x) {
+  return 0.5f * x * (1.0f + erf_as(x * 0.70710678118654752f));
+}
+// GELU-tanh(x) = x/2·(1 + tanh(√(2/π)·(x + 0.044715x³))).  LOWP (16-bit outputs,
+// relative precision 2^-8): tanh on the special-function unit (relative error
+// about 2^-11); otherwise the exp-based form above.
+template <bool LOWP>
+__device__ __forceinline__ float gelu_tanh_f(float x) {
+  const float u = 0.79788456080286536f * fmaf(0.044715f * x, x * x, x);
+  return 0.5f * x * (1.0f + (LOWP ? tanh_approx(u) : tanh_ex2(u)));
+}
+
+template <int ACT, bool LOWP = false>
 __device__ __forceinline__ float activate(float v, float u) {
   if constexpr (ACT == ACT_RELU) return fmaxf(v, 0.0f);
   if constexpr (ACT == ACT_GELU) return gelu_erf_f(v);
-  if constexpr (ACT == ACT_GELU_TANH) return gelu_tanh_f(v);
-  if constexpr (ACT == ACT_GEGLU) return gelu_tanh_f(v) * u;
+  if constexpr (ACT == ACT_GELU_TANH) return gelu_tanh_f<LOWP>(v);
+  if constexpr (ACT == ACT_GEGLU) return gelu_tanh_f<LOWP>(v) * u;
   return v;
 }
 
@@ -651,7 +679,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                  v[h * 32 + j] = activate<ACT>(__uint_as_float(rg[j]), __uint_as_float(ru[j]));
+                  v[h * 32 + j] = activate<ACT, OUT != DT_F32>(__uint_as_float(rg[j]), __uint_as_float(ru[j]));
               }
             } else {
               uint32_t ra[CH];
@@ -664,7 +692,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
             }
           } else {
 #pragma unroll
-            for (int j = 0; j < CH; ++j) v[j] = (ACT == ACT_GEGLU) ? activate<ACT>(0.0f, 0.0f) : 0.0f;
+            for (int j = 0; j < CH; ++j) v[j] = (ACT == ACT_GEGLU) ? activate<ACT, OUT != DT_F32>(0.0f, 0.0f) : 0.0f;
           }
           if (cc + CH >= c_end) {
             // this warp's TMEM reads of the tile are done: hand its share back to the MMA warp
@@ -696,7 +724,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           }
           if constexpr (ACT != ACT_GEGLU) {
 #pragma unroll
-            for (int j = 0; j < CH; ++j) v[j] = activate<ACT>(v[j], 0.0f);
+            for (int j = 0; j < CH; ++j) v[j] = activate<ACT, OUT != DT_F32>(v[j], 0.0f);
           }
           if (has_res && m_ok) {
 #pragma unroll
@@ -933,7 +961,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
                   if (lane == 0 && j + i < cnt && (long long)wcol * 32 < p.N)
                     p.aux[(row0 + i) * p.ld_aux + wcol] = word;
                 }
-                const float y = (activate<ACT>(xv, 0.0f) + rv[i]) * scale_v;
+                const float y = (activate<ACT, OUT != DT_F32>(xv, 0.0f) + rv[i]) * scale_v;
                 if (n_ok && j + i < cnt) {
                   char* dst = orow + i * ostep;
                   if constexpr (OUT == DT_F32) *reinterpret_cast<float*>(dst) = y;
