@@ -257,7 +257,11 @@ static Layout layout_for(const fl_plan_s* p, int mma_n, int b_boxes, int max_sme
   // Split-K partial tiles (swap-AB, S > 1): a split-K cluster owns one tile, so the
   // partials are published after the last UMMA has read the last stage and can
   // reuse the stage memory.
-  const uint32_t red = (p->swap && p->split_k > 1) ? 128u * ((uint32_t)mma_n * 4u + 16u) : 0u;
+  // (this CTA's partial, 128 rows, then S-1 received slices of 128/S rows each)
+  const uint32_t red = (p->swap && p->split_k > 1)
+                           ? (128u + (uint32_t)(p->split_k - 1) * (128u / (uint32_t)p->split_k)) *
+                                 ((uint32_t)mma_n * 4u + 16u)
+                           : 0u;
   // swap-AB with a residual: two 32-row x 32-column residual blocks per epilogue warp
   L.res_blk = 32u * 32u * (uint32_t)esize(p->epi.residual_dtype);
   const uint32_t res = (p->swap && p->epi.has_residual) ? (uint32_t)Cfg<true>::kEpiWarps * 2u * L.res_blk : 0u;

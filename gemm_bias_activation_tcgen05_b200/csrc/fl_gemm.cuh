@@ -230,17 +230,20 @@ __device__ __forceinline__ float ldg_pinned(const void* base, long long i, int d
 }
 
 // ------------------------------------------------------------------ 3xTF32 split
-// x = hi + lo with hi = x rounded to TF32 (nearest, ties away) and lo = x - hi
-// (exact in fp32) rounded to TF32 again, so that the tensor core reads both
-// halves exactly: x·y ≈ hi_x·hi_y + hi_x·lo_y + lo_x·hi_y.
+// x = hi + lo.  The tensor core reads a 32-bit operand word as TF32 by keeping its
+// top 19 bits (sign, exponent, 10 mantissa bits): the raw stage word therefore
+// serves as hi = trunc(x), and only lo = x - hi (exact in fp32, at most 13
+// significant bits) is written, rounded to TF32 so that the tensor core reads it
+// exactly.  x·y ≈ hi_x·hi_y + hi_x·lo_y + lo_x·hi_y.  (A reader that rounded
+// instead of truncating would leave errors near 2^-11 per product, which the
+// parity tests on inputs with all low bits set reject.)
 __device__ __forceinline__ uint32_t tf32_rna(float x) {
   uint32_t r;
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
   return r;
 }
-__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
-  hi = tf32_rna(x);
-  lo = tf32_rna(x - __uint_as_float(hi));
+__device__ __forceinline__ uint32_t tf32_lo(float x) {
+  return tf32_rna(x - __uint_as_float(__float_as_uint(x) & 0xFFFFE000u));
 }
 
 // ------------------------------------------------------------------ epilogue helpers
@@ -362,6 +365,9 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
   const uint32_t red_done_bar = bars + 8u * (2 * NS + 6);
   const uint32_t tmem_slot = bars + 8u * (2 * NS + 7);
   auto conv_bar = [&](int s) { return bars + 8u * (2 * NS + 8 + s); };  // 3xTF32: stage split done
+  // swap-AB split-K: the partial slices that the peers push (the slot of the first
+  // 3xTF32 barrier, which that layout does not use)
+  const uint32_t recv_bar = bars + 8u * (2 * NS + 8);
 
   // Clusters: split-K groups of S CTAs (swap layout), or CTA pairs that share one
   // 256-row UMMA (PAIR: rank 0 issues the UMMA for both, each CTA owns 128 rows).
@@ -392,7 +398,8 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
     // split-K hand-off: one arrive per epilogue warp (after __syncwarp, so the
     // release covers the whole warp's shared-memory writes)
     mbar_init(red_ready_bar, kEpiWarps * S);
-    mbar_init(red_done_bar, kEpiWarps * S);
+    mbar_init(red_done_bar, S - 1 > 0 ? S - 1 : 1);  // one arrival per peer that received our slices
+    if (SWAP && S > 1) mbar_init(recv_bar, 1);
     if (TF32)  // PAIR: both CTAs' converters arrive on the leader's barrier
       for (int s = 0; s < NS; ++s) mbar_init(conv_bar(s), kEpiWarps * kCl);
     fence_mbarrier_init();
@@ -601,8 +608,8 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         int ta, tb;
         tile_coords(t, p, ta, tb);
         if constexpr (TF32) {
-          // split every stage of this tile into hi (in place) and lo halves; the 256
-          // epilogue threads share the stage's 16-byte words
+          // write the TF32 lo half of every stage of this tile beside it (the raw words
+          // serve as hi); the 256 epilogue threads share the stage's 16-byte words
           const int et = (warp - kEpiWarp0) * 32 + lane;
           const uint32_t words = p.stage_bytes >> 4;
           for (int kb = kb_begin; ok && kb < kb_end; ++kb, ++cit) {
@@ -617,13 +624,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
                            : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w)
                            : "r"(a)
                            : "memory");
-              uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
-              split_tf32(x.x, h0, l0);
-              split_tf32(x.y, h1, l1);
-              split_tf32(x.z, h2, l2);
-              split_tf32(x.w, h3, l3);
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(h0), "r"(h1), "r"(h2), "r"(h3)
-                           : "memory");
+              const uint32_t l0 = tf32_lo(x.x), l1 = tf32_lo(x.y), l2 = tf32_lo(x.z), l3 = tf32_lo(x.w);
               asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a + p.stage_bytes), "r"(l0), "r"(l1),
                            "r"(l2), "r"(l3)
                            : "memory");
@@ -836,47 +837,63 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
                            "r"(r[4 * c]), "r"(r[4 * c + 1]), "r"(r[4 * c + 2]), "r"(r[4 * c + 3])
                            : "memory");
           }
+          // the copy engine reads these rows: generic writes before async-proxy reads
+          fence_proxy_async_smem();
           tc_fence_before();
           __syncwarp();
+          const uint32_t slice_bytes = (uint32_t)L * p.red_pitch;
+          const uint32_t recv = red_base + 128u * p.red_pitch;  // S-1 slots of one slice each
           if (lane == 0) {
             mbar_arrive(tempty_bar(buf));
+            // expect the peers' slices before telling anyone this CTA is ready for them
+            if (ew == 0) mbar_arrive_expect_tx(recv_bar, (uint32_t)(S - 1) * slice_bytes);
             for (int rk = 0; rk < S; ++rk) mbar_arrive_remote(mapa_shared(red_ready_bar, (uint32_t)rk));
           }
           if (!warp_wait_bounded(red_ready_bar, 0, p, lane, true)) ok = false;
-          // Sum the S partials of this CTA's slice (rows [rank·L, rank·L + L) of every CTA's
-          // buffer, contiguous) in rank order and write the sums over this CTA's own copy,
-          // which no peer reads.  The eight epilogue warps stream the slice in 16-byte
-          // pieces, so every warp-wide load from a peer is 512 contiguous bytes.
+          // Every CTA has published and its stages are dead: push slice k of this CTA's
+          // partial (rows [k·L, k·L + L), contiguous) into CTA k's receive slot for this
+          // rank, with the copy engine.
+          if (ok && ew == 0 && lane == 0) {
+            for (int k = 0; k < S; ++k) {
+              if (k == (int)rank) continue;
+              const int slot = ((int)rank < k) ? (int)rank : (int)rank - 1;
+              bulk_copy_to_peer(mapa_shared(recv + (uint32_t)slot * slice_bytes, (uint32_t)k),
+                                red_base + (uint32_t)(k * L) * p.red_pitch, slice_bytes,
+                                mapa_shared(recv_bar, (uint32_t)k));
+            }
+          }
+          // (waited even after a failed wait above: a peer that got through may be
+          // writing into this CTA, which must not leave before the bytes land)
+          if (!warp_wait_bounded(recv_bar, 0, p, lane, true)) ok = false;
+          // tell the sources their copies have landed (they stay resident until then)
+          if (ok && ew == 0 && lane == 0)
+            for (int k = 0; k < S; ++k)
+              if (k != (int)rank) mbar_arrive_remote(mapa_shared(red_done_bar, (uint32_t)k));
+          // Sum the S partials of this CTA's slice in rank order (this CTA's own rows and
+          // the received slots, all local) and write the sums over the own rows.
           {
             const uint32_t slice = red_base + (uint32_t)(rank * L) * p.red_pitch;
-            const uint32_t bytes = (uint32_t)L * p.red_pitch;
             constexpr uint32_t kStep = kEpiWarps * 32u * 16u;
-            uint32_t peer[4];
-#pragma unroll
-            for (int rk = 0; rk < 4; ++rk) peer[rk] = mapa_shared(slice, (uint32_t)(rk < S ? rk : 0));
             if (ok) {
 #pragma unroll 1
-              for (uint32_t o = (uint32_t)(ew * 32 + lane) * 16u; o < bytes; o += 4u * kStep) {
-                float4 f[4][4];
+              for (uint32_t o = (uint32_t)(ew * 32 + lane) * 16u; o < slice_bytes; o += kStep) {
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-#pragma unroll
-                  for (int rk = 0; rk < 4; ++rk) {
-                    f[u][rk] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (rk < S && o + u * kStep < bytes) f[u][rk] = ld_shared_cluster_f4(peer[rk] + o + u * kStep);
+                for (int k = 0; k < 4; ++k) {
+                  if (k >= S) break;
+                  const uint32_t a = (k == (int)rank) ? slice + o
+                                                      : recv + (uint32_t)(k < (int)rank ? k : k - 1) * slice_bytes + o;
+                  const float4 v = ld_shared_f4(a);
+                  if (k == 0) {
+                    acc = v;
+                  } else {
+                    acc.x += v.x;
+                    acc.y += v.y;
+                    acc.z += v.z;
+                    acc.w += v.w;
                   }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  float4 acc = f[u][0];
-#pragma unroll
-                  for (int rk = 1; rk < 4; ++rk) {
-                    acc.x += f[u][rk].x;
-                    acc.y += f[u][rk].y;
-                    acc.z += f[u][rk].z;
-                    acc.w += f[u][rk].w;
-                  }
-                  if (o + u * kStep < bytes) st_shared_f4(slice + o + u * kStep, acc);
                 }
+                st_shared_f4(slice + o, acc);
               }
             }
             // every warp's sums are in place before any warp finishes rows
@@ -980,11 +997,8 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           if (lane == 0) mbar_arrive(tempty_bar(buf));
           continue;
         }
-        // nobody leaves while a peer may still read its partial
-        __syncwarp();
-        if (lane == 0)
-          for (int rk = 0; rk < S; ++rk) mbar_arrive_remote(mapa_shared(red_done_bar, (uint32_t)rk));
-        if (!warp_wait_bounded(red_done_bar, 0, p, lane, true)) ok = false;
+        // nobody leaves while its copies into the peers may still be reading its rows
+        if (ew == 0 && !warp_wait_bounded(red_done_bar, 0, p, lane, true)) ok = false;
         break;  // a split-K cluster owns exactly one tile
       }
       cp_async_wait<0>();  // no copy into shared memory outlives the loop

@@ -179,6 +179,26 @@ def test_fp32_operands_3xtf32(fl, M, N, K, epilogue, out_dtype):
     assert got["info"]["cta_pair"] == (1 if M > 128 else 0)
 
 
+@pytest.mark.parametrize("M", [64, 130])
+def test_fp32_split_with_all_low_bits_set(fl, M):
+    # Every operand word has its 13 low mantissa bits set, where truncating and
+    # rounding an fp32 word to TF32 differ the most: the 3xTF32 split must still
+    # be exact to about 2^-21 per product.  (K is short so that one wrong hi word,
+    # an error near 2^-10 of a product, stands far above the bound.)
+    N, K = 200, 24
+    g = torch.Generator().manual_seed(M)
+
+    def words(rows, cols):
+        x = torch.randn(rows, cols, generator=g, dtype=torch.float32)
+        b = x.view(torch.int32) | 0x1FFF
+        return b.view(torch.float32).contiguous()
+
+    A, W = words(M, K), words(N, K)
+    got = P.run_linear(fl, M=M, N=N, K=K, dtype="f32", epilogue="NONE", out_dtype="f32", A=A, W=W)
+    y, _, _, absdot = P.oracle_linear(A=A, W=W, epilogue="NONE", out_dtype="f32", M=M, N=N, K=K)
+    P.check_close(got["out"], y, "f32", absdot, f"fp32 low bits M{M}")
+
+
 def test_fp32_residual_scale(fl):
     _linear_case(fl, 200, 264, 132, dtype="f32", epilogue="GELU_BIAS", out_dtype="f32", residual=True, scale=0.5)
 
