@@ -46,49 +46,62 @@ __global__ void __launch_bounds__(256) fl_relu_backward_kernel(const void* __res
   constexpr int PER16 = 16 / ESZ;  // elements per 16-byte vector
   const T* grad = reinterpret_cast<const T*>(grad_);
   T* dpre = reinterpret_cast<T*>(dpre_);
-  const long long total = M * words;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long m = i / words;
-    const long long w = i - m * words;
-    const uint32_t bits = __ldg(aux + m * words + w);
-    const long long n0 = w * 32;
-    const T* g = grad + m * ldg + n0;
-    T* d = dpre + m * ldd + n0;
-    if (vec_ok && n0 + 32 <= N) {
+  const int lane = threadIdx.x & 31;
+  // A warp takes a block of 32 mask words (32·32 elements) of one row.  In a full
+  // block lane l moves 16-byte vectors l, l+32, ... of the block, so every warp-wide
+  // access is 512 contiguous bytes, and reads its mask bits from the block's 32 words
+  // (one coalesced load) by shuffle.
+  const long long wblocks = (words + 31) / 32;
+  const long long total = M * wblocks;
+  const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long blk = warp0; blk < total; blk += nwarps) {
+    const long long m = blk / wblocks;
+    const long long w0 = (blk - m * wblocks) * 32;
+    const T* g = grad + m * ldg + w0 * 32;
+    T* d = dpre + m * ldd + w0 * 32;
+    const uint32_t myword = (w0 + lane < words) ? __ldg(aux + m * words + w0 + lane) : 0u;
+    if (vec_ok && w0 + 32 <= words && (w0 + 32) * 32 <= N) {
 #pragma unroll
-      for (int v = 0; v < 32 / PER16; ++v) {
-        uint4 x = __ldg(reinterpret_cast<const uint4*>(g) + v);
+      for (int v = 0; v < 32 * 32 / PER16 / 32; ++v) {
+        const int e0 = (v * 32 + lane) * PER16;  // first element of this lane's vector
+        const uint32_t bits = __shfl_sync(0xffffffffu, myword, e0 >> 5);
+        uint4 x = __ldg(reinterpret_cast<const uint4*>(g) + v * 32 + lane);
         uint32_t* xw = reinterpret_cast<uint32_t*>(&x);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           if constexpr (ESZ == 2) {
-            const int j = v * PER16 + e * 2;
+            const int j = (e0 & 31) + e * 2;
             // grad·0 keeps the sign of grad (IEEE): clear all but the sign bit
             const uint32_t lo_keep = ((bits >> j) & 1u) ? 0x0000FFFFu : 0x00008000u;
             const uint32_t hi_keep = ((bits >> (j + 1)) & 1u) ? 0xFFFF0000u : 0x80000000u;
             xw[e] &= (lo_keep | hi_keep);
           } else {
-            const int j = v * PER16 + e;
+            const int j = (e0 & 31) + e;
             xw[e] &= ((bits >> j) & 1u) ? 0xFFFFFFFFu : 0x80000000u;
           }
         }
-        reinterpret_cast<uint4*>(d)[v] = x;
+        reinterpret_cast<uint4*>(d)[v * 32 + lane] = x;
       }
     } else {
-      for (int j = 0; j < 32 && n0 + j < N; ++j) {
-        T x = g[j];
-        if (!((bits >> j) & 1u)) {
-          if constexpr (ESZ == 2) {
-            unsigned short b = *reinterpret_cast<unsigned short*>(&x);
-            b &= 0x8000u;
-            x = *reinterpret_cast<T*>(&b);
-          } else {
-            uint32_t b = __float_as_uint(x) & 0x80000000u;
-            x = __uint_as_float(b);
+      // ragged block: lane l finishes word w0 + l element by element
+      const long long w = w0 + lane;
+      if (w < words) {
+        const long long n0 = w * 32;
+        for (int j = 0; j < 32 && n0 + j < N; ++j) {
+          T x = g[lane * 32 + j];
+          if (!((myword >> j) & 1u)) {
+            if constexpr (ESZ == 2) {
+              unsigned short b = *reinterpret_cast<unsigned short*>(&x);
+              b &= 0x8000u;
+              x = *reinterpret_cast<T*>(&b);
+            } else {
+              uint32_t b = __float_as_uint(x) & 0x80000000u;
+              x = __uint_as_float(b);
+            }
           }
+          d[lane * 32 + j] = x;
         }
-        d[j] = x;
       }
     }
   }
