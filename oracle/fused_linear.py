@@ -78,7 +78,7 @@ def activation(v: np.ndarray, kind: str) -> np.ndarray:
         return v
     if kind in ("RELU_BIAS", "RELU_AUX_BIAS", "RELU"):
         return relu(v)
-    if kind in ("GELU_BIAS", "GELU"):
+    if kind in ("GELU_BIAS", "GELU_AUX_BIAS", "GELU"):
         return gelu_erf(v)
     if kind in ("GELU_TANH_BIAS", "GELU_TANH"):
         return gelu_tanh(v)
@@ -156,14 +156,20 @@ def fused_linear(A, W, bias=None, *, epilogue: str, out_dtype: str, bias_axis: i
 
     v = A·Wᵀ + bias (fp64, bias added before any rounding, as the [epilog] page
     describes the epilog acting on the FP32 result); a = act(v);
-    y = round_out((a + residual)·scale); aux = relu_aux_mask(v) for RELU_AUX_BIAS.
+    y = round_out((a + residual)·scale); aux = relu_aux_mask(v) for RELU_AUX_BIAS,
+    and for GELU_AUX_BIAS the pre-activation itself, rounded once to out_dtype
+    (the stored input of the GELU backward, see ``dgelu``).
     """
     v = gemm(A, W, b_major)
     if bias is not None and epilogue != "NONE":
         v = add_bias(v, bias, bias_axis)
     a = activation(v, epilogue)
     y = residual_scale(a, residual, scale)
-    aux = relu_aux_mask(v) if epilogue == "RELU_AUX_BIAS" else None
+    aux = None
+    if epilogue == "RELU_AUX_BIAS":
+        aux = relu_aux_mask(v)
+    elif epilogue == "GELU_AUX_BIAS":
+        aux = round_to(v, out_dtype)
     return round_to(y, out_dtype), aux, v
 
 
@@ -197,3 +203,41 @@ def drelu(grad, aux: np.ndarray, N: int, out_dtype: str = "bf16"):
     for n in range(N):
         bits[:, n] = ((aux[:, n // 32].astype(np.uint64) >> np.uint64(n % 32)) & np.uint64(1)).astype(np.float64)
     return round_to(grad[:, :N] * bits, out_dtype)
+
+
+# ---------------------------------------------------------------- backward of the fused layer
+# [epilog]: the RELU_AUX_BIAS epilog keeps a ReLU mask in the forward pass so that the
+# backward pass computes its gradient efficiently; [gelu] §2.2.1: when Linear+GELU is
+# rewritten into one fused operator, the backward gradient must be fused as well.  For
+# y = act(v), v = x·Wᵀ + b with b broadcast over the rows m, the chain rule gives
+#   dv[m,n] = dy[m,n] · act'(v[m,n])   and   db[n] = Σ_m dv[m,n].
+
+
+def bias_grad(dv: np.ndarray) -> np.ndarray:
+    """db[n] = Σ_m dv[m,n] in float64 (the bias is added to every row m of v)."""
+    return np.asarray(dv, dtype=np.float64).sum(axis=0)
+
+
+def drelu_bgrad(grad, aux: np.ndarray, N: int, out_dtype: str = "bf16"):
+    """(dv, db): dv = ``drelu`` (grad times the mask bit, exact) and db = Σ_m dv in float64."""
+    dv = drelu(grad, aux, N, out_dtype)
+    return dv, bias_grad(dv)
+
+
+def gelu_erf_grad(v: np.ndarray) -> np.ndarray:
+    """d/dv [v·Φ(v)] = Φ(v) + v·φ(v), φ(v) = e^(-v²/2)/√(2π) — the derivative of [gelu] §1's GELU."""
+    v = np.asarray(v, dtype=np.float64)
+    Phi = 0.5 * (1.0 + _erf(v / math.sqrt(2.0)))
+    phi = np.exp(-0.5 * v * v) / math.sqrt(2.0 * math.pi)
+    return Phi + v * phi
+
+
+def dgelu(grad, v, out_dtype: str = "bf16"):
+    """dv = grad · GELU'(v), rounded once to out_dtype; v is the stored pre-activation."""
+    return round_to(np.asarray(grad, dtype=np.float64) * gelu_erf_grad(v), out_dtype)
+
+
+def dgelu_bgrad(grad, v, out_dtype: str = "bf16"):
+    """(dv rounded to out_dtype, db = Σ_m grad·GELU'(v) in float64, before any rounding)."""
+    exact = np.asarray(grad, dtype=np.float64) * gelu_erf_grad(v)
+    return round_to(exact, out_dtype), bias_grad(exact)

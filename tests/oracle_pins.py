@@ -227,6 +227,80 @@ def pin_geglu_identity(o):
     assert np.array_equal(y, hh)
 
 
+def pin_bias_grad_brute_force(o):
+    r = _rng(11)
+    M, N = 7, 9
+    dv = r.standard_normal((M, N))
+    db = o.bias_grad(dv)
+    for n in range(N):
+        assert abs(db[n] - sum(dv[m, n] for m in range(M))) < 1e-12
+    assert np.array_equal(o.bias_grad(np.ones((5, 3))), np.full(3, 5.0))
+
+
+def pin_drelu_bgrad(o):
+    r = _rng(12)
+    M, N = 6, 45
+    v = r.standard_normal((M, N))
+    grad = o.round_to(r.standard_normal((M, N)), "bf16")
+    dv, db = o.drelu_bgrad(grad, o.relu_aux_mask(v), N, "bf16")
+    for n in range(N):
+        want = sum(grad[m, n] for m in range(M) if v[m, n] > 0)
+        assert abs(db[n] - want) < 1e-12, n
+    assert np.array_equal(dv, np.where(v > 0, grad, 0.0))
+
+
+def pin_gelu_grad_finite_difference(o):
+    """GELU' against a central difference of GELU (fp64, h = 1e-5: error ~1e-10)."""
+    v = np.linspace(-9.0, 9.0, 721)
+    h = 1e-5
+    fd = (o.gelu_erf(v + h) - o.gelu_erf(v - h)) / (2 * h)
+    assert np.max(np.abs(o.gelu_erf_grad(v) - fd)) < 1e-8
+
+
+def pin_gelu_grad_identities(o):
+    v = np.linspace(-6.0, 6.0, 241)
+    # Φ(v) + Φ(-v) = 1 and the v·φ(v) terms cancel: GELU'(v) + GELU'(-v) = 1
+    assert np.max(np.abs(o.gelu_erf_grad(v) + o.gelu_erf_grad(-v) - 1.0)) < 1e-14
+    assert o.gelu_erf_grad(np.array([0.0]))[0] == 0.5
+    assert abs(o.gelu_erf_grad(np.array([40.0]))[0] - 1.0) < 1e-15
+    assert abs(o.gelu_erf_grad(np.array([-40.0]))[0]) < 1e-15
+    # GELU' exceeds 1 just above zero (the maximum is near v = 1.4)
+    assert o.gelu_erf_grad(np.array([1.4]))[0] > 1.12
+
+
+def pin_dgelu_bgrad(o):
+    r = _rng(13)
+    M, N = 5, 33
+    v = o.round_to(r.standard_normal((M, N)) * 2, "bf16")
+    grad = o.round_to(r.standard_normal((M, N)), "bf16")
+    dv, db = o.dgelu_bgrad(grad, v, "bf16")
+    assert np.array_equal(dv, o.dgelu(grad, v, "bf16"))
+    for m in range(M):
+        for n in range(N):
+            x = v[m, n]
+            g = 0.5 * (1 + math.erf(x / math.sqrt(2.0))) + x * math.exp(-x * x / 2) / math.sqrt(2 * math.pi)
+            assert dv[m, n] == o.round_to(np.array([grad[m, n] * g]), "bf16")[0]
+    for n in range(N):
+        x = v[:, n]
+        want = sum(grad[m, n] * (0.5 * (1 + math.erf(x[m] / math.sqrt(2.0)))
+                                 + x[m] * math.exp(-x[m] ** 2 / 2) / math.sqrt(2 * math.pi)) for m in range(M))
+        assert abs(db[n] - want) < 1e-12
+
+
+def pin_gelu_aux_stores_preactivation(o):
+    r = _rng(14)
+    M, N, K = 4, 19, 6
+    A = r.standard_normal((M, K))
+    W = r.standard_normal((N, K))
+    b = r.standard_normal(N)
+    y, aux, v = o.fused_linear(A, W, b, epilogue="GELU_AUX_BIAS", out_dtype="bf16")
+    for m in range(M):
+        for n in range(N):
+            acc = sum(A[m, k] * W[n, k] for k in range(K)) + b[n]
+            assert aux[m, n] == o.round_to(np.array([acc]), "bf16")[0]
+            assert y[m, n] == o.round_to(np.array([0.5 * acc * (1 + math.erf(acc / math.sqrt(2.0)))]), "bf16")[0]
+
+
 # ---------------------------------------------------------------- rounding
 def pin_round_to(o):
     one = 1.0

@@ -29,7 +29,8 @@ def _namespace(**over):
         if hasattr(oracle, "__all__") else None
     if ns is None:
         names = ["gemm", "add_bias", "relu", "gelu_erf", "gelu_tanh", "activation", "relu_aux_mask",
-                 "residual_scale", "round_to", "fused_linear", "geglu_h", "geglu_mlp", "drelu"]
+                 "residual_scale", "round_to", "fused_linear", "geglu_h", "geglu_mlp", "drelu",
+                 "bias_grad", "drelu_bgrad", "gelu_erf_grad", "dgelu", "dgelu_bgrad"]
         ns = types.SimpleNamespace(**{k: getattr(oracle, k) for k in names})
     for k, v in over.items():
         setattr(ns, k, v)
@@ -42,7 +43,11 @@ def _namespace(**over):
             v = ns.add_bias(v, bias, bias_axis)
         a = ns.activation(v, epilogue)
         y = ns.residual_scale(a, residual, scale)
-        aux = ns.relu_aux_mask(v) if epilogue == "RELU_AUX_BIAS" else None
+        aux = None
+        if epilogue == "RELU_AUX_BIAS":
+            aux = ns.relu_aux_mask(v)
+        elif epilogue == "GELU_AUX_BIAS":
+            aux = ns.round_to(v, out_dtype)
         return ns.round_to(y, out_dtype), aux, v
 
     def activation(v, kind):
@@ -50,9 +55,20 @@ def _namespace(**over):
             return v
         if kind in ("RELU_BIAS", "RELU_AUX_BIAS", "RELU"):
             return ns.relu(v)
-        if kind in ("GELU_BIAS", "GELU"):
+        if kind in ("GELU_BIAS", "GELU_AUX_BIAS", "GELU"):
             return ns.gelu_erf(v)
         return ns.gelu_tanh(v)
+
+    def drelu_bgrad(grad, aux, N, out_dtype="bf16"):
+        dv = ns.drelu(grad, aux, N, out_dtype)
+        return dv, ns.bias_grad(dv)
+
+    def dgelu(grad, v, out_dtype="bf16"):
+        return ns.round_to(np.asarray(grad, float) * ns.gelu_erf_grad(v), out_dtype)
+
+    def dgelu_bgrad(grad, v, out_dtype="bf16"):
+        exact = np.asarray(grad, float) * ns.gelu_erf_grad(v)
+        return ns.round_to(exact, out_dtype), ns.bias_grad(exact)
 
     def geglu_h(x, Wg, Wu, out_dtype="bf16"):
         return ns.round_to(ns.gelu_tanh(ns.gemm(x, Wg)) * ns.gemm(x, Wu), out_dtype)
@@ -62,7 +78,8 @@ def _namespace(**over):
         return h, ns.round_to(ns.gemm(h, Wd), out_dtype)
 
     for name, f in [("fused_linear", fused_linear), ("activation", activation),
-                    ("geglu_h", geglu_h), ("geglu_mlp", geglu_mlp)]:
+                    ("geglu_h", geglu_h), ("geglu_mlp", geglu_mlp), ("drelu_bgrad", drelu_bgrad),
+                    ("dgelu", dgelu), ("dgelu_bgrad", dgelu_bgrad)]:
         if name not in over:
             setattr(ns, name, f)
     return ns
@@ -114,6 +131,15 @@ MUTANTS = {
     "residual_dropped": dict(residual_scale=lambda a, r, s: a * s),
     "round_truncates": dict(round_to=lambda x, d: (np.trunc(np.asarray(x, float) * 256) / 256) if d == "bf16"
                             else oracle.round_to(x, d)),
+    "bias_grad_over_columns": dict(bias_grad=lambda dv: np.asarray(dv, float).sum(axis=1)[:np.asarray(dv).shape[1]]
+                                   if np.asarray(dv).shape[0] >= np.asarray(dv).shape[1]
+                                   else np.resize(np.asarray(dv, float).sum(axis=1), np.asarray(dv).shape[1])),
+    "bias_grad_mean": dict(bias_grad=lambda dv: np.asarray(dv, float).mean(axis=0)),
+    "gelu_grad_drops_vphi": dict(gelu_erf_grad=lambda v: 0.5 * (1.0 + erf(np.asarray(v, float) / math.sqrt(2.0)))),
+    "gelu_grad_phi_sign": dict(gelu_erf_grad=lambda v: 0.5 * (1.0 + erf(np.asarray(v, float) / math.sqrt(2.0)))
+                               - np.asarray(v, float) * np.exp(-0.5 * np.asarray(v, float) ** 2) / math.sqrt(2 * math.pi)),
+    "gelu_grad_no_half_exponent": dict(gelu_erf_grad=lambda v: 0.5 * (1.0 + erf(np.asarray(v, float) / math.sqrt(2.0)))
+                                       + np.asarray(v, float) * np.exp(-np.asarray(v, float) ** 2) / math.sqrt(2 * math.pi)),
     "drelu_inverted": dict(drelu=lambda grad, aux, N, od="bf16": oracle.round_to(
         np.asarray(grad, float)[:, :N] - oracle.drelu(grad, aux, N, od), od)),
 }
