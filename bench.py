@@ -351,6 +351,7 @@ def run_ours(args):
         "roofline": roofline,
         "clocks": clk.summary(),
         "breakdown": breakdown,
+        "backward": time_backward(fl, pk),
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
@@ -380,6 +381,49 @@ def time_single_launch(suite, it, stream, sh, reps):
     torch.cuda.synchronize()
     del flush
     return sum(a.elapsed_time(b) for a, b in evs) / reps
+
+
+def time_backward(fl, pk, reps=10):
+    """The backward kernels with the fused bias gradient on the relu_aux_4096 shape
+    (4096 x 4096 bf16), each launch after a 256 MB L2 flush: us, achieved GB/s of the
+    algorithmic bytes, and the fraction of the measured HBM copy bandwidth."""
+    import torch
+    M = N = 4096
+    g = torch.Generator(device="cpu").manual_seed(5)
+    grad = torch.randn(M, N, generator=g).to(torch.bfloat16).cuda()
+    v = (torch.randn(M, N, generator=g) * 3).to(torch.bfloat16).cuda()
+    mask = torch.randint(-2 ** 31, 2 ** 31 - 1, (M, N // 32), generator=g, dtype=torch.int32).cuda()
+    dpre = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    dbias = torch.empty(N, dtype=torch.float32, device="cuda")
+    nbytes = fl.fl_bias_grad_workspace_size(M, N, "bf16")
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device="cuda")
+    sh = torch.cuda.current_stream().cuda_stream
+    runs = {
+        "drelu_bgrad_4096x4096_bf16": (lambda: fl.fl_drelu_bgrad(grad, mask, dpre, dbias, M, N, "bf16", ws, nbytes,
+                                                                 stream=sh),
+                                       2 * M * N * 2 + M * N // 8 + 4 * N),
+        "dgelu_bgrad_4096x4096_bf16": (lambda: fl.fl_dgelu_bgrad(grad, v, dpre, dbias, M, N, "bf16", ws, nbytes,
+                                                                 stream=sh),
+                                       3 * M * N * 2 + 4 * N),
+    }
+    out = {}
+    for name, (fn, algo_bytes) in runs.items():
+        fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in evs:
+            flush.zero_()
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in evs) / reps
+        gbs = algo_bytes / (ms * 1e-3) / 1e9
+        out[name] = {"us": round(ms * 1e3, 2), "algorithmic_bytes": algo_bytes, "gbs": round(gbs, 1),
+                     "frac_of_hbm": round(gbs / pk["hbm_gbs"], 3)}
+    del flush
+    return out
 
 
 def profiled_traffic():

@@ -8,7 +8,8 @@ without a B200.
 
 The entry points keep the C names: ``fl_plan``, ``fl_execute``, ``fl_free``,
 ``fl_relu_backward``, ``fl_check_status``, ``fl_get_plan_info``,
-``fl_last_error``, ``fl_set_wait_limit_ns``, ``fl_execute_noalloc``.  ``Plan`` is a small owner of one
+``fl_last_error``, ``fl_set_wait_limit_ns``, ``fl_execute_noalloc``, ``fl_bias_grad_workspace_size``,
+``fl_drelu_bgrad``, ``fl_dgelu_bgrad``.  ``Plan`` is a small owner of one
 plan handle (the cuBLASLt epilog page's Matmul → plan → execute → free).
 """
 from __future__ import annotations
@@ -28,12 +29,13 @@ STATUS_NAMES = {0: "FL_OK", 1: "FL_ERR_INVALID_ARG", 2: "FL_ERR_UNSUPPORTED", 3:
 FL_F16, FL_BF16, FL_F32 = 0, 1, 2
 FL_COMPUTE_32F, FL_COMPUTE_32F_3XTF32 = 0, 1
 EPILOGUES = {"NONE": 0, "BIAS": 1, "RELU_BIAS": 2, "RELU_AUX_BIAS": 3, "GELU_BIAS": 4,
-             "GELU_TANH_BIAS": 5, "GEGLU_TANH": 6}
+             "GELU_TANH_BIAS": 5, "GEGLU_TANH": 6, "GELU_AUX_BIAS": 7}
 DTYPES = {"f16": FL_F16, "bf16": FL_BF16, "f32": FL_F32}
 COMPUTES = {"32F": FL_COMPUTE_32F, "32F_3XTF32": FL_COMPUTE_32F_3XTF32}
 
 EXPORTED = ["fl_plan", "fl_execute", "fl_relu_backward", "fl_check_status", "fl_get_plan_info",
-            "fl_free", "fl_last_error", "fl_set_wait_limit_ns", "fl_execute_noalloc"]
+            "fl_free", "fl_last_error", "fl_set_wait_limit_ns", "fl_execute_noalloc",
+            "fl_bias_grad_workspace_size", "fl_drelu_bgrad", "fl_dgelu_bgrad"]
 
 
 class fl_epilogue_desc(ctypes.Structure):
@@ -78,6 +80,12 @@ def _load() -> ctypes.CDLL:
     lib.fl_execute_noalloc.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(fl_epilogue_desc),
                                        vp, vp, vp, vp, vp, vp, vp]
     lib.fl_execute_noalloc.restype = i32
+    lib.fl_bias_grad_workspace_size.argtypes = [i64, i64, i32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.fl_bias_grad_workspace_size.restype = i32
+    lib.fl_drelu_bgrad.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i32, vp, ctypes.c_size_t, vp]
+    lib.fl_drelu_bgrad.restype = i32
+    lib.fl_dgelu_bgrad.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, vp, ctypes.c_size_t, vp]
+    lib.fl_dgelu_bgrad.restype = i32
     return lib
 
 
@@ -166,6 +174,27 @@ def fl_relu_backward(grad, aux, dpre, M: int, N: int, dtype: str, ld_grad: int =
                      stream=None) -> None:
     _check(LIB.fl_relu_backward(_ptr(grad), _ptr(aux), _ptr(dpre), int(M), int(N), int(ld_grad),
                                 int(ld_dpre), DTYPES[dtype], _stream(stream)), "fl_relu_backward")
+
+
+def fl_bias_grad_workspace_size(M: int, N: int, dtype: str) -> int:
+    n = ctypes.c_size_t()
+    _check(LIB.fl_bias_grad_workspace_size(int(M), int(N), DTYPES[dtype], ctypes.byref(n)),
+           "fl_bias_grad_workspace_size")
+    return int(n.value)
+
+
+def fl_drelu_bgrad(grad, aux, dpre, dbias, M: int, N: int, dtype: str, workspace=None, workspace_bytes: int = 0,
+                   ld_grad: int = 0, ld_dpre: int = 0, stream=None) -> None:
+    _check(LIB.fl_drelu_bgrad(_ptr(grad), _ptr(aux), _ptr(dpre), _ptr(dbias), int(M), int(N), int(ld_grad),
+                              int(ld_dpre), DTYPES[dtype], _ptr(workspace), int(workspace_bytes), _stream(stream)),
+           "fl_drelu_bgrad")
+
+
+def fl_dgelu_bgrad(grad, v, dpre, dbias, M: int, N: int, dtype: str, workspace=None, workspace_bytes: int = 0,
+                   ld_grad: int = 0, ld_v: int = 0, ld_dpre: int = 0, stream=None) -> None:
+    _check(LIB.fl_dgelu_bgrad(_ptr(grad), _ptr(v), _ptr(dpre), _ptr(dbias), int(M), int(N), int(ld_grad),
+                              int(ld_v), int(ld_dpre), DTYPES[dtype], _ptr(workspace), int(workspace_bytes),
+                              _stream(stream)), "fl_dgelu_bgrad")
 
 
 def fl_check_status(plan: int, stream=None) -> int:

@@ -216,7 +216,8 @@ static int act_of(int kind) {
   switch (kind) {
     case FL_EPI_RELU_BIAS:
     case FL_EPI_RELU_AUX_BIAS: return ACT_RELU;
-    case FL_EPI_GELU_BIAS: return ACT_GELU;
+    case FL_EPI_GELU_BIAS:
+    case FL_EPI_GELU_AUX_BIAS: return ACT_GELU;
     case FL_EPI_GELU_TANH_BIAS: return ACT_GELU_TANH;
     case FL_EPI_GEGLU_TANH: return ACT_GEGLU;
     default: return ACT_NONE;
@@ -384,7 +385,7 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
                                            (long long)M, (long long)N, (long long)K);
   if (M > (1LL << 31) - 256 || N > (1LL << 30) || K > (1LL << 31) - 256)
     return fail(FL_ERR_INVALID_ARG, "fl_plan: dimension too large");
-  if (epi->kind < FL_EPI_NONE || epi->kind > FL_EPI_GEGLU_TANH)
+  if (epi->kind < FL_EPI_NONE || epi->kind > FL_EPI_GELU_AUX_BIAS)
     return fail(FL_ERR_INVALID_ARG, "fl_plan: unknown epilogue kind %d", epi->kind);
   for (int i = 0; i < 3; ++i)
     if (epi->reserved[i] != 0) return fail(FL_ERR_INVALID_ARG, "fl_plan: reserved fields must be 0");
@@ -410,6 +411,8 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
     return fail(FL_ERR_UNSUPPORTED, "fl_plan: GEGLU_TANH takes the stacked [2N,K] weight (b_major 0)");
   if (epi->kind == FL_EPI_GEGLU_TANH && epi->out_dtype == FL_F32)
     return fail(FL_ERR_UNSUPPORTED, "fl_plan: GEGLU_TANH writes h in f16/bf16");
+  if (epi->kind == FL_EPI_GELU_AUX_BIAS && epi->unfused)
+    return fail(FL_ERR_UNSUPPORTED, "fl_plan: the unfused twin has no GELU_AUX_BIAS step");
   if (epi->lda < 0 || epi->ldb < 0 || epi->ldo < 0 || epi->ldr < 0)
     return fail(FL_ERR_INVALID_ARG, "fl_plan: negative leading dimension");
 
@@ -419,7 +422,7 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
   if (p->epi.scale == 0.0f) p->epi.scale = 1.0f;
   p->act = act_of(epi->kind);
   p->has_bias = has_bias;
-  p->has_aux = epi->kind == FL_EPI_RELU_AUX_BIAS;
+  p->has_aux = epi->kind == FL_EPI_RELU_AUX_BIAS || epi->kind == FL_EPI_GELU_AUX_BIAS;
   // leading dimensions default to packed
   const int64_t a_cols = K, b_cols = epi->b_major ? N : K;
   if (p->epi.lda == 0) p->epi.lda = a_cols;
@@ -554,9 +557,9 @@ struct GemmArgs {
 
 // Launch an elementwise kernel with programmatic dependent launch allowed.
 template <typename... KArgs, typename... Args>
-static cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, cudaStream_t s, Args... args) {
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, cudaStream_t s, Args... args) {
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.gridDim = grid;
   cfg.blockDim = dim3(256, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
@@ -731,7 +734,7 @@ static int grid_for(long long work, int num_sms) {
 template <int DT>
 static fl_status launch_ew_t(const EwParams& P, int num_sms, cudaStream_t s) {
   const long long work = P.M * ((P.N + 31) / 32);
-  const cudaError_t err = launch_pdl(fl_ew_step_kernel<DT>, (unsigned)grid_for(work, num_sms), s, P);
+  const cudaError_t err = launch_pdl(fl_ew_step_kernel<DT>, dim3((unsigned)grid_for(work, num_sms)), s, P);
   if (err != cudaSuccess) return fail(FL_ERR_CUDA, "elementwise kernel launch: %s", cudaGetErrorString(err));
   return after_launch(s, "elementwise step kernel");
 }
@@ -742,16 +745,19 @@ static fl_status launch_ew(int dt, const EwParams& P, int num_sms, cudaStream_t 
 }
 
 // ------------------------------------------------------------------ execute
-extern "C" fl_status fl_execute(fl_plan_t p, const void* A, const void* W, const void* bias, uint32_t* aux,
+extern "C" fl_status fl_execute(fl_plan_t p, const void* A, const void* W, const void* bias, void* aux_,
                                 const void* residual, void* out, void* stream_) {
   g_err[0] = 0;
+  uint32_t* aux = static_cast<uint32_t*>(aux_);
   if (!p) return fail(FL_ERR_INVALID_ARG, "fl_execute: null plan");
   if (!out || (p->K > 0 && (!A || !W)))
     return fail(FL_ERR_INVALID_ARG, "fl_execute: A, W (when K > 0) and out are required");
   if (p->has_bias && !bias) return fail(FL_ERR_INVALID_ARG, "fl_execute: this epilogue needs a bias");
   if (!p->has_bias && bias) return fail(FL_ERR_INVALID_ARG, "fl_execute: this epilogue takes no bias");
-  if (p->has_aux && !aux) return fail(FL_ERR_INVALID_ARG, "fl_execute: RELU_AUX_BIAS needs the aux mask buffer");
-  if (!p->has_aux && aux) return fail(FL_ERR_INVALID_ARG, "fl_execute: only RELU_AUX_BIAS writes an aux mask");
+  if (p->has_aux && !aux) return fail(FL_ERR_INVALID_ARG, "fl_execute: RELU_AUX_BIAS / GELU_AUX_BIAS need the aux buffer");
+  if (!p->has_aux && aux) return fail(FL_ERR_INVALID_ARG, "fl_execute: only the AUX epilogues write an aux buffer");
+  if (aux && p->epi.kind == FL_EPI_GELU_AUX_BIAS && !aligned16(aux))
+    return fail(FL_ERR_ALIGNMENT, "fl_execute: the GELU_AUX_BIAS pre-activation buffer must be 16-byte aligned");
   if (p->epi.has_residual && !residual) return fail(FL_ERR_INVALID_ARG, "fl_execute: has_residual needs a residual");
   if (!p->epi.has_residual && residual) return fail(FL_ERR_INVALID_ARG, "fl_execute: residual given but not planned");
   if ((p->K > 0 && (!aligned16(A) || !aligned16(W))) || !aligned16(out) || (residual && !aligned16(residual)))
@@ -894,16 +900,130 @@ extern "C" fl_status fl_relu_backward(const void* grad, const uint32_t* aux, voi
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
   cudaError_t err;
   if (dtype == FL_BF16)
-    err = launch_pdl(fl_relu_backward_kernel<DT_BF16>, (unsigned)grid, s, grad, aux, dpre, (long long)M, (long long)N,
+    err = launch_pdl(fl_relu_backward_kernel<DT_BF16>, dim3((unsigned)grid), s, grad, aux, dpre, (long long)M, (long long)N,
                      (long long)ld_grad, (long long)ld_dpre, words, vec_ok);
   else if (dtype == FL_F16)
-    err = launch_pdl(fl_relu_backward_kernel<DT_F16>, (unsigned)grid, s, grad, aux, dpre, (long long)M, (long long)N,
+    err = launch_pdl(fl_relu_backward_kernel<DT_F16>, dim3((unsigned)grid), s, grad, aux, dpre, (long long)M, (long long)N,
                      (long long)ld_grad, (long long)ld_dpre, words, vec_ok);
   else
-    err = launch_pdl(fl_relu_backward_kernel<DT_F32>, (unsigned)grid, s, grad, aux, dpre, (long long)M, (long long)N,
+    err = launch_pdl(fl_relu_backward_kernel<DT_F32>, dim3((unsigned)grid), s, grad, aux, dpre, (long long)M, (long long)N,
                      (long long)ld_grad, (long long)ld_dpre, words, vec_ok);
   if (err != cudaSuccess) return fail(FL_ERR_CUDA, "dReLU kernel launch: %s", cudaGetErrorString(err));
   return after_launch(s, "dReLU kernel");
+}
+
+// ------------------------------------------------------------------ backward with bias gradient
+// Launch geometry of fl_bwd_bgrad_kernel: column strips of 32 16-byte vectors, and
+// row blocks enough for about four CTAs per SM.
+struct BwdGeom {
+  int strips, row_blocks, rows_per_block;
+  long long ws_ld;
+  size_t counters_bytes, bytes;
+};
+static fl_status bwd_geom(int64_t M, int64_t N, int dtype, BwdGeom* g) {
+  int dev = 0, sms = 148;
+  FL_CUDA(cudaGetDevice(&dev));
+  FL_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const int ve = 16 / esize(dtype);
+  g->strips = (int)std::max<int64_t>(1, cdiv(N, 32LL * ve));
+  int64_t rb = std::max<int64_t>(1, cdiv(4LL * sms, g->strips));
+  rb = std::min<int64_t>(rb, std::max<int64_t>(1, cdiv(M, 8)));
+  g->rows_per_block = (int)std::max<int64_t>(1, cdiv(M, rb));
+  g->row_blocks = (int)std::max<int64_t>(1, cdiv(M, g->rows_per_block));
+  g->ws_ld = (long long)g->strips * 32LL * ve;
+  g->counters_bytes = (size_t)cdiv((int64_t)g->strips * 4, 256) * 256;
+  g->bytes = g->counters_bytes + (size_t)g->row_blocks * (size_t)g->ws_ld * sizeof(float);
+  return FL_OK;
+}
+
+extern "C" fl_status fl_bias_grad_workspace_size(int64_t M, int64_t N, int32_t dtype, size_t* bytes) {
+  g_err[0] = 0;
+  if (!bytes) return fail(FL_ERR_INVALID_ARG, "fl_bias_grad_workspace_size: null pointer");
+  if (M < 0 || N < 0) return fail(FL_ERR_INVALID_ARG, "fl_bias_grad_workspace_size: negative size");
+  if (dtype != FL_F16 && dtype != FL_BF16 && dtype != FL_F32)
+    return fail(FL_ERR_INVALID_ARG, "fl_bias_grad_workspace_size: unknown dtype %d", dtype);
+  BwdGeom g;
+  fl_status st = bwd_geom(M, N, dtype, &g);
+  if (st) return st;
+  *bytes = g.bytes;
+  return FL_OK;
+}
+
+static fl_status bwd_bgrad(int mode, const char* who, const void* grad, const uint32_t* mask, const void* v, void* dpre,
+                           float* dbias, int64_t M, int64_t N, int64_t ld_grad, int64_t ld_v, int64_t ld_dpre,
+                           int32_t dtype, void* workspace, size_t workspace_bytes, void* stream_) {
+  g_err[0] = 0;
+  if (!grad || !dpre || (mode == BWD_DRELU ? !mask : !v)) return fail(FL_ERR_INVALID_ARG, "%s: null pointer", who);
+  if (M < 0 || N < 0) return fail(FL_ERR_INVALID_ARG, "%s: negative size", who);
+  if (dtype != FL_F16 && dtype != FL_BF16 && dtype != FL_F32)
+    return fail(FL_ERR_INVALID_ARG, "%s: unknown dtype %d", who, dtype);
+  if (ld_grad == 0) ld_grad = N;
+  if (ld_dpre == 0) ld_dpre = N;
+  if (ld_v == 0) ld_v = N;
+  if (ld_grad < N || ld_dpre < N || (mode == BWD_DGELU && ld_v < N))
+    return fail(FL_ERR_INVALID_ARG, "%s: leading dimension < N", who);
+  const int es = esize(dtype);
+  if (reinterpret_cast<uintptr_t>(grad) % es || reinterpret_cast<uintptr_t>(dpre) % es ||
+      (mask && reinterpret_cast<uintptr_t>(mask) % 4) || (v && reinterpret_cast<uintptr_t>(v) % es) ||
+      (dbias && reinterpret_cast<uintptr_t>(dbias) % 4))
+    return fail(FL_ERR_ALIGNMENT, "%s: misaligned pointer", who);
+  BwdGeom g;
+  fl_status st = bwd_geom(M, N, dtype, &g);
+  if (st) return st;
+  if (dbias && (!workspace || workspace_bytes < g.bytes || !aligned16(workspace)))
+    return fail(FL_ERR_INVALID_ARG, "%s: the bias gradient needs a 16-byte aligned, zero-initialised workspace of "
+                "%zu bytes (fl_bias_grad_workspace_size)", who, g.bytes);
+  if (M == 0 || N == 0) {
+    if (dbias && N > 0) FL_CUDA(cudaMemsetAsync(dbias, 0, (size_t)N * sizeof(float), (cudaStream_t)stream_));
+    return FL_OK;
+  }
+  BwdParams P{};
+  P.grad = grad;
+  P.mask = mask;
+  P.v = v;
+  P.dpre = dpre;
+  P.dbias = dbias;
+  P.counters = reinterpret_cast<int*>(workspace);
+  P.ws = dbias ? reinterpret_cast<float*>(static_cast<char*>(workspace) + g.counters_bytes) : nullptr;
+  P.M = M;
+  P.N = N;
+  P.ldg = ld_grad;
+  P.ldv = ld_v;
+  P.ldd = ld_dpre;
+  P.words = cdiv(N, 32);
+  P.ws_ld = g.ws_ld;
+  P.rows_per_block = g.rows_per_block;
+  P.row_blocks = g.row_blocks;
+  P.vec_ok = aligned16(grad) && aligned16(dpre) && (ld_grad * es) % 16 == 0 && (ld_dpre * es) % 16 == 0 &&
+             (mode == BWD_DRELU || (aligned16(v) && (ld_v * es) % 16 == 0));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+  const dim3 grid((unsigned)g.strips, (unsigned)g.row_blocks);
+  cudaError_t err;
+  if (mode == BWD_DRELU) {
+    err = dtype == FL_BF16 ? launch_pdl(fl_bwd_bgrad_kernel<DT_BF16, BWD_DRELU>, grid, s, P)
+        : dtype == FL_F16  ? launch_pdl(fl_bwd_bgrad_kernel<DT_F16, BWD_DRELU>, grid, s, P)
+                           : launch_pdl(fl_bwd_bgrad_kernel<DT_F32, BWD_DRELU>, grid, s, P);
+  } else {
+    err = dtype == FL_BF16 ? launch_pdl(fl_bwd_bgrad_kernel<DT_BF16, BWD_DGELU>, grid, s, P)
+        : dtype == FL_F16  ? launch_pdl(fl_bwd_bgrad_kernel<DT_F16, BWD_DGELU>, grid, s, P)
+                           : launch_pdl(fl_bwd_bgrad_kernel<DT_F32, BWD_DGELU>, grid, s, P);
+  }
+  if (err != cudaSuccess) return fail(FL_ERR_CUDA, "%s: kernel launch: %s", who, cudaGetErrorString(err));
+  return after_launch(s, who);
+}
+
+extern "C" fl_status fl_drelu_bgrad(const void* grad, const uint32_t* aux, void* dpre, float* dbias, int64_t M,
+                                    int64_t N, int64_t ld_grad, int64_t ld_dpre, int32_t dtype, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  return bwd_bgrad(BWD_DRELU, "fl_drelu_bgrad", grad, aux, nullptr, dpre, dbias, M, N, ld_grad, 0, ld_dpre, dtype,
+                   workspace, workspace_bytes, stream);
+}
+
+extern "C" fl_status fl_dgelu_bgrad(const void* grad, const void* v, void* dpre, float* dbias, int64_t M, int64_t N,
+                                    int64_t ld_grad, int64_t ld_v, int64_t ld_dpre, int32_t dtype, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  return bwd_bgrad(BWD_DGELU, "fl_dgelu_bgrad", grad, nullptr, v, dpre, dbias, M, N, ld_grad, ld_v, ld_dpre, dtype,
+                   workspace, workspace_bytes, stream);
 }
 
 // ------------------------------------------------------------------ status
@@ -957,15 +1077,16 @@ static fl_status noalloc_scratch(int dev, unsigned char** out) {
 
 extern "C" fl_status fl_execute_noalloc(int64_t M, int64_t N, int64_t K, int32_t dtype, int32_t compute,
                                         const fl_epilogue_desc* epi, const void* A, const void* W,
-                                        const void* bias, uint32_t* aux, const void* residual, void* out,
+                                        const void* bias, void* aux_, const void* residual, void* out,
                                         void* stream_) {
   g_err[0] = 0;
+  uint32_t* aux = static_cast<uint32_t*>(aux_);
   const char* who = "fl_execute_noalloc";
   if (!epi) return fail(FL_ERR_INVALID_ARG, "%s: null epilogue descriptor", who);
   if (M < 1 || N < 1 || K < 0) return fail(FL_ERR_INVALID_ARG, "%s: need M>=1, N>=1, K>=0", who);
   if (M > (1LL << 31) - 256 || N > (1LL << 30) || K > (1LL << 31) - 256)
     return fail(FL_ERR_INVALID_ARG, "%s: dimension too large", who);
-  if (epi->kind < FL_EPI_NONE || epi->kind > FL_EPI_GEGLU_TANH)
+  if (epi->kind < FL_EPI_NONE || epi->kind > FL_EPI_GELU_AUX_BIAS)
     return fail(FL_ERR_INVALID_ARG, "%s: unknown epilogue kind %d", who, epi->kind);
   for (int i = 0; i < 3; ++i)
     if (epi->reserved[i] != 0) return fail(FL_ERR_INVALID_ARG, "%s: reserved fields must be 0", who);
@@ -983,6 +1104,8 @@ extern "C" fl_status fl_execute_noalloc(int64_t M, int64_t N, int64_t K, int32_t
     return fail(FL_ERR_INVALID_ARG, "%s: unknown residual_dtype %d", who, epi->residual_dtype);
   if ((epi->bias_axis != 0 && epi->bias_axis != 1) || (epi->b_major != 0 && epi->b_major != 1))
     return fail(FL_ERR_INVALID_ARG, "%s: bias_axis and b_major must be 0 or 1", who);
+  if (epi->kind == FL_EPI_GELU_AUX_BIAS && epi->unfused)
+    return fail(FL_ERR_UNSUPPORTED, "%s: the unfused twin has no GELU_AUX_BIAS step", who);
   if (epi->kind == FL_EPI_GEGLU_TANH && (epi->b_major || epi->out_dtype == FL_F32))
     return fail(FL_ERR_UNSUPPORTED, "%s: GEGLU_TANH takes the stacked [2N,K] weight and writes f16/bf16", who);
   if (epi->lda < 0 || epi->ldb < 0 || epi->ldo < 0 || epi->ldr < 0)
@@ -995,7 +1118,7 @@ extern "C" fl_status fl_execute_noalloc(int64_t M, int64_t N, int64_t K, int32_t
   if (p.epi.scale == 0.0f) p.epi.scale = 1.0f;
   p.act = act_of(epi->kind);
   p.has_bias = has_bias;
-  p.has_aux = epi->kind == FL_EPI_RELU_AUX_BIAS;
+  p.has_aux = epi->kind == FL_EPI_RELU_AUX_BIAS || epi->kind == FL_EPI_GELU_AUX_BIAS;
   const int64_t a_cols = K, b_cols = epi->b_major ? N : K;
   if (p.epi.lda == 0) p.epi.lda = a_cols;
   if (p.epi.ldb == 0) p.epi.ldb = b_cols;

@@ -2,8 +2,11 @@
 //
 //   * fl_relu_backward_kernel: dpre = grad ⊙ bit(mask), the backward use of the
 //     RELU_AUX_BIAS mask (cuBLASLt epilog page: the aux ReLU mask serves the
-//     backward pass).  One thread per (row, 32-column mask word): one 4-byte
-//     mask load and 32 contiguous elements in 16-byte vectors.
+//     backward pass).  A warp per block of 32 mask words of a row.
+//   * fl_bwd_bgrad_kernel: the same step, or dpre = grad · GELU'(v) from the
+//     pre-activation a GELU_AUX_BIAS forward stored, fused with the bias
+//     gradient dbias[n] = Σ_m dpre[m,n] (Linear+GELU page §2.2.1: the backward
+//     gradient is fused as well).
 //   * fl_ew_step_kernel: ONE epilogue step per launch (bias, activation with
 //     optional mask, residual, scale, GeGLU product) over a row-major matrix —
 //     the unfused GEMM-then-elementwise design of the Linear+GELU page
@@ -30,6 +33,154 @@ template <>
 struct ElemT<DT_F16> { using T = __half; static constexpr uint32_t sign = 0x8000u; };
 template <>
 struct ElemT<DT_F32> { using T = float; static constexpr uint32_t sign = 0x80000000u; };
+
+// ---------------------------------------------------------------- backward with bias gradient
+enum BwdMode { BWD_DRELU = 0, BWD_DGELU = 1 };
+
+struct BwdParams {
+  const void* grad;      // [M, ldg] of DT
+  const uint32_t* mask;  // DRELU: [M, words] packed ReLU mask
+  const void* v;         // DGELU: [M, ldv] of DT, the stored pre-activation
+  void* dpre;            // [M, ldd] of DT
+  float* dbias;          // [N] fp32, or null (no bias gradient)
+  float* ws;             // row_blocks x ws_ld fp32 partial column sums
+  int* counters;         // per column strip: row blocks that have stored their partials
+  long long M, N, ldg, ldv, ldd, words, ws_ld;
+  int rows_per_block, row_blocks, vec_ok;
+};
+
+// GELU'(v) = Φ(v) + v·φ(v) in fp32, with erf as in the forward epilogue
+__device__ __forceinline__ float gelu_erf_grad_f(float v) {
+  const float Phi = 0.5f * (1.0f + erf_as(v * 0.70710678118654752f));
+  const float phi = ex2_approx(-0.5f * v * v * 1.4426950408889634f) * 0.39894228040143268f;  // e^(-v²/2)/√(2π)
+  return fmaf(v, phi, Phi);
+}
+
+// Grid (column strips of 32 16-byte vectors, row blocks).  Warp w of a CTA takes rows
+// r ≡ w (mod 8) of the block, lane l the l-th vector of the strip, so every warp-wide
+// access is 512 contiguous bytes of one row.  Each thread keeps fp32 column partials;
+// the CTA adds its eight warps' partials in warp order, stores them for its row block,
+// and the last row block of a strip to finish adds all row blocks in order: the result
+// does not depend on the schedule.
+template <int DT, int MODE>
+__global__ void __launch_bounds__(256, 4) fl_bwd_bgrad_kernel(const BwdParams P) {
+  using T = typename ElemT<DT>::T;
+  grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
+  constexpr int ESZ = sizeof(T);
+  constexpr int VE = 16 / ESZ;  // elements per 16-byte vector
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int strip = blockIdx.x, rb = blockIdx.y;
+  const long long c0 = (long long)strip * 32 * VE + (long long)lane * VE;
+  const long long r0 = (long long)rb * P.rows_per_block;
+  const long long r1 = min(P.M, r0 + P.rows_per_block);
+  const bool vec = P.vec_ok && c0 + VE <= P.N;
+  const T* grad = reinterpret_cast<const T*>(P.grad);
+  const T* vv = reinterpret_cast<const T*>(P.v);
+  T* dpre = reinterpret_cast<T*>(P.dpre);
+  float part[VE];
+#pragma unroll
+  for (int i = 0; i < VE; ++i) part[i] = 0.0f;
+  // four rows a trip (rows m, m+8, m+16, m+24 of this warp): every load of the trip is
+  // in flight before the first use; the vectors stay packed until then
+  constexpr int RU = 4;
+  for (long long mb = r0 + warp; mb < r1; mb += 8 * RU) {
+    uint4 gq[RU], vq[RU];
+    uint32_t word[RU];
+#pragma unroll
+    for (int u = 0; u < RU; ++u) {
+      const long long m = mb + 8 * u;
+      gq[u] = make_uint4(0u, 0u, 0u, 0u);
+      vq[u] = make_uint4(0u, 0u, 0u, 0u);
+      word[u] = 0u;
+      if (m >= r1) continue;
+      if (vec) {
+        gq[u] = __ldg(reinterpret_cast<const uint4*>(grad + m * P.ldg + c0));
+        if (MODE == BWD_DGELU) vq[u] = __ldg(reinterpret_cast<const uint4*>(vv + m * P.ldv + c0));
+      } else {
+        T* ge = reinterpret_cast<T*>(&gq[u]);
+        T* ve = reinterpret_cast<T*>(&vq[u]);
+#pragma unroll
+        for (int i = 0; i < VE; ++i) {
+          if (c0 + i < P.N) {
+            ge[i] = grad[m * P.ldg + c0 + i];
+            if (MODE == BWD_DGELU) ve[i] = vv[m * P.ldv + c0 + i];
+          }
+        }
+      }
+      // the VE columns lie in one mask word (VE divides 32)
+      if (MODE == BWD_DRELU && c0 < P.N) word[u] = __ldg(P.mask + m * P.words + (c0 >> 5));
+    }
+#pragma unroll
+    for (int u = 0; u < RU; ++u) {
+      const long long m = mb + 8 * u;
+      if (m >= r1) continue;
+      const T* ge = reinterpret_cast<const T*>(&gq[u]);
+      const T* ve = reinterpret_cast<const T*>(&vq[u]);
+      float d[VE];
+#pragma unroll
+      for (int i = 0; i < VE; ++i) {
+        const float gi = static_cast<float>(ge[i]);
+        if (MODE == BWD_DRELU) d[i] = ((word[u] >> ((c0 & 31) + i)) & 1u) ? gi : gi * 0.0f;  // keeps grad's sign
+        else d[i] = gi * gelu_erf_grad_f(static_cast<float>(ve[i]));
+      }
+      if (vec) {
+        uint4 q;
+        T* e = reinterpret_cast<T*>(&q);
+#pragma unroll
+        for (int i = 0; i < VE; ++i) e[i] = static_cast<T>(d[i]);
+        *reinterpret_cast<uint4*>(dpre + m * P.ldd + c0) = q;
+      } else {
+#pragma unroll
+        for (int i = 0; i < VE; ++i)
+          if (c0 + i < P.N) dpre[m * P.ldd + c0 + i] = static_cast<T>(d[i]);
+      }
+#pragma unroll
+      for (int i = 0; i < VE; ++i) part[i] += d[i];
+    }
+  }
+  if (P.dbias == nullptr) return;
+  // ---- bias gradient: the CTA's eight warps in warp order, then the row blocks in order
+  __shared__ float red[8][32 * 8];
+  __shared__ int last;
+#pragma unroll
+  for (int i = 0; i < VE; ++i) red[warp][lane * VE + i] = part[i];
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int i = 0; i < VE; ++i) {
+      float s = red[0][lane * VE + i];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) s += red[w][lane * VE + i];
+      if (c0 + i < P.N) P.ws[(long long)rb * P.ws_ld + c0 + i] = s;
+    }
+    __threadfence();  // this block's partials before its count
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) last = (atomicAdd(P.counters + strip, 1) == P.row_blocks - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  // every thread of the last block adds one column over the row blocks, in order
+  if (threadIdx.x < 32 * VE) {
+    const long long c = (long long)strip * 32 * VE + threadIdx.x;
+    if (c < P.N) {
+      const float* src = P.ws + c;
+      float s = 0.0f;
+      int b = 0;
+      for (; b + 8 <= P.row_blocks; b += 8) {
+        float t[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) t[k] = __ldcg(src + (long long)(b + k) * P.ws_ld);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) s += t[k];
+      }
+      for (; b < P.row_blocks; ++b) s += __ldcg(src + (long long)b * P.ws_ld);
+      P.dbias[c] = s;
+    }
+  }
+  if (threadIdx.x == 0) P.counters[strip] = 0;  // ready for the next launch
+}
 
 // ---------------------------------------------------------------- dReLU
 template <int DT>

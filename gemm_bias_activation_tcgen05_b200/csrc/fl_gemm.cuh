@@ -247,6 +247,31 @@ __device__ __forceinline__ uint32_t tf32_lo(float x) {
 }
 
 // ------------------------------------------------------------------ epilogue helpers
+// Store CH values of one row (first column nc0, element offset i0 of the row start)
+// in OUT type: 16-byte vectors when the whole chunk lies inside the N columns (the
+// caller's pitch and base are 16-byte aligned), else element by element up to N.
+template <int OUT, int CH>
+__device__ __forceinline__ void store_row_chunk(void* base, long long i0, int nc0, int N, const float (&v)[CH]) {
+  constexpr int ES = (OUT == DT_F32) ? 4 : 2;
+  if (nc0 + CH <= N) {
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<char*>(base) + i0 * ES);
+#pragma unroll
+    for (int c = 0; c < CH * ES / 16; ++c) {
+      uint32_t w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if constexpr (OUT == DT_F32) w[k] = __float_as_uint(v[4 * c + k]);
+        else w[k] = pack2<OUT>(v[8 * c + 2 * k], v[8 * c + 2 * k + 1]);
+      }
+      dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < CH; ++j)
+      if (nc0 + j < N) store_elem<OUT>(base, i0 + j, v[j]);
+  }
+}
+
 // Load CH consecutive elements of one row (16-byte vectors when the whole chunk
 // is in range, else guarded scalars) and widen them to fp32.
 template <int CH>
@@ -594,6 +619,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
     const bool has_bias = p.bias != nullptr;
     const bool has_res = p.residual != nullptr;
     const bool has_aux = p.aux != nullptr;
+    const bool has_mask = has_aux && ACT != ACT_GELU;  // the ReLU mask (GELU_AUX stores v instead)
     uint32_t local = 0;
     bool ok = true;
 
@@ -718,7 +744,11 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           uint32_t aux_word[CH / 32];
 #pragma unroll
           for (int h = 0; h < CH / 32; ++h) aux_word[h] = 0u;
-          if (has_aux) {
+          if constexpr (ACT == ACT_GELU) {
+            // GELU_AUX_BIAS: the pre-activation v, in the output type, for the backward pass
+            if (has_aux && m_ok) store_row_chunk<OUT, CH>(p.aux, (long long)m * p.ldo + nc0, nc0, p.N, v);
+          }
+          if (has_mask) {
 #pragma unroll
             for (int j = 0; j < CH; ++j)
               if (v[j] > 0.0f && (full_cols || nc0 + j < p.N)) aux_word[j >> 5] |= 1u << (j & 31);
@@ -735,7 +765,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
 #pragma unroll
             for (int j = 0; j < CH; ++j) v[j] *= scale;
           }
-          if (has_aux && m_ok) {
+          if (has_mask && m_ok) {
 #pragma unroll
             for (int h = 0; h < CH / 32; ++h) {
               const int w = (nc0 >> 5) + h;
@@ -972,7 +1002,11 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
               for (int i = 0; i < 8; ++i) {
                 float xv = x[i];
                 if (has_bias) xv += (p.bias_axis == 0) ? bias_n : __shfl_sync(0xffffffffu, bias_l, (j + i) & 31);
-                if (has_aux) {
+                if constexpr (ACT == ACT_GELU) {
+                  // GELU_AUX_BIAS: the pre-activation v, in the output type
+                  if (has_aux && n_ok && j + i < cnt) store_elem<OUT>(p.aux, (row0 + i) * p.ldo + n, xv);
+                }
+                if (has_mask) {
                   const uint32_t word = __ballot_sync(0xffffffffu, n_ok && xv > 0.0f);
                   const int wcol = n_w0 >> 5;
                   if (lane == 0 && j + i < cnt && (long long)wcol * 32 < p.N)

@@ -34,6 +34,7 @@
 #ifndef FUSED_LINEAR_H_
 #define FUSED_LINEAR_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -69,6 +70,9 @@ typedef enum { FL_COMPUTE_32F = 0, FL_COMPUTE_32F_3XTF32 = 1 } fl_compute;
  *   GELU_BIAS       y = gelu_erf(acc + bias)   = 0.5·v·(1 + erf(v/√2))
  *   GELU_TANH_BIAS  y = gelu_tanh(acc + bias)  = 0.5·v·(1 + tanh(√(2/π)(v + 0.044715 v³)))
  *   GEGLU_TANH      W is the stacked [2N, K] matrix [Wg; Wu]; y = gelu_tanh(A·Wgᵀ)·(A·Wuᵀ)
+ *   GELU_AUX_BIAS   as GELU_BIAS, and aux = v = acc + bias stored in the output type, the
+ *                   input of the GELU backward (fl_dgelu_bgrad); [epilog] keeps forward
+ *                   state for the backward pass, [gelu] §2.2.1 fuses the backward too
  * Every kind may add a residual and scale: y = (act(v) + residual)·scale. */
 typedef enum {
   FL_EPI_NONE = 0,
@@ -77,7 +81,8 @@ typedef enum {
   FL_EPI_RELU_AUX_BIAS = 3,
   FL_EPI_GELU_BIAS = 4,
   FL_EPI_GELU_TANH_BIAS = 5,
-  FL_EPI_GEGLU_TANH = 6
+  FL_EPI_GEGLU_TANH = 6,
+  FL_EPI_GELU_AUX_BIAS = 7
 } fl_epi_kind;
 
 /* The "epilog" argument of fl_plan.  Zero-initialise, then set fields. */
@@ -120,14 +125,15 @@ fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, int32_t dtype
  *   A        [M, lda] operand
  *   W        [N, ldb] weight (b_major 0), [K, ldb] (b_major 1) or [2N, ldb] (GEGLU)
  *   bias     length N (bias_axis 0) or M (bias_axis 1); required iff the kind has a bias
- *   aux      [M, ceil(N/32)] uint32, required iff RELU_AUX_BIAS, packed rows;
- *            bit j of word w of row m is column 32w+j, least significant bit first;
- *            bits of columns ≥ N are written as 0
+ *   aux      RELU_AUX_BIAS: [M, ceil(N/32)] uint32, packed rows; bit j of word w of
+ *            row m is column 32w+j, least significant bit first; bits of columns ≥ N
+ *            are written as 0.  GELU_AUX_BIAS: [M, ldo] in the output type (16-byte
+ *            aligned), the pre-activation v.  Null for every other kind
  *   residual [M, ldr], required iff has_residual
  *   out      [M, ldo] result
  * Errors: FL_ERR_INVALID_ARG (missing operand), FL_ERR_ALIGNMENT, FL_ERR_CUDA. */
 fl_status fl_execute(fl_plan_t plan, const void* A, const void* W, const void* bias,
-                     uint32_t* aux, const void* residual, void* out, void* stream);
+                     void* aux, const void* residual, void* out, void* stream);
 
 /* Backward of RELU_AUX_BIAS: dpre[m,n] = grad[m,n] · bit(m,n), with the mask
  * written by a RELU_AUX_BIAS forward ([epilog]: the aux ReLU mask serves the
@@ -137,6 +143,32 @@ fl_status fl_execute(fl_plan_t plan, const void* A, const void* W, const void* b
 fl_status fl_relu_backward(const void* grad, const uint32_t* aux, void* dpre, int64_t M,
                            int64_t N, int64_t ld_grad, int64_t ld_dpre, int32_t dtype,
                            void* stream);
+
+/* Backward of the fused layer with the bias gradient fused in (no counterpart API on
+ * the pages; [epilog] keeps the RELU_AUX mask for the backward pass and [gelu]
+ * §2.2.1 asks that the backward of Linear+GELU be fused as well).  For y = act(v),
+ * v = A·Wᵀ + bias with the bias broadcast over rows:
+ *   fl_drelu_bgrad  dpre[m,n] = grad[m,n] · bit(m,n)      (mask of RELU_AUX_BIAS)
+ *   fl_dgelu_bgrad  dpre[m,n] = grad[m,n] · GELU'(v[m,n])  (v of GELU_AUX_BIAS),
+ *                   GELU'(v) = Φ(v) + v·φ(v), evaluated in fp32
+ * and, when dbias is not null, dbias[n] = Σ_m dpre[m,n] in fp32 (of the fp32
+ * products, before dpre is rounded to dtype), summed in a fixed order so that the
+ * result does not depend on the schedule.
+ *   grad, v, dpre  [M, ld] of dtype (F16/BF16/F32); ld 0 = packed (N)
+ *   aux            [M, ceil(N/32)] uint32 packed mask (4-byte aligned)
+ *   dbias          [N] fp32, or null (then no workspace is needed)
+ *   workspace      fl_bias_grad_workspace_size bytes, 16-byte aligned, owned by the
+ *                  caller and zero-filled once before its first use; every call leaves
+ *                  it ready for the next.  Calls that overlap on the GPU must not share it.
+ * dpre may alias grad.  Errors: FL_ERR_INVALID_ARG (null operand, negative size, ld < N,
+ * workspace missing or too small), FL_ERR_ALIGNMENT, FL_ERR_CUDA. */
+fl_status fl_bias_grad_workspace_size(int64_t M, int64_t N, int32_t dtype, size_t* bytes);
+fl_status fl_drelu_bgrad(const void* grad, const uint32_t* aux, void* dpre, float* dbias, int64_t M,
+                         int64_t N, int64_t ld_grad, int64_t ld_dpre, int32_t dtype, void* workspace,
+                         size_t workspace_bytes, void* stream);
+fl_status fl_dgelu_bgrad(const void* grad, const void* v, void* dpre, float* dbias, int64_t M, int64_t N,
+                         int64_t ld_grad, int64_t ld_v, int64_t ld_dpre, int32_t dtype, void* workspace,
+                         size_t workspace_bytes, void* stream);
 
 /* Synchronise `stream` and read the plan's device error word.  Returns
  * FL_ERR_TIMEOUT if a bounded wait inside a kernel of this plan gave up
@@ -186,7 +218,7 @@ const char* fl_last_error(void);
  * Errors: as fl_plan and fl_execute. */
 fl_status fl_execute_noalloc(int64_t M, int64_t N, int64_t K, int32_t dtype, int32_t compute,
                              const fl_epilogue_desc* epi, const void* A, const void* W,
-                             const void* bias, uint32_t* aux, const void* residual, void* out,
+                             const void* bias, void* aux, const void* residual, void* out,
                              void* stream);
 
 /* Override the bound on every in-kernel wait for plans created afterwards

@@ -1,0 +1,158 @@
+"""GPU parity of the backward of the fused layer and of the GELU_AUX_BIAS forward.
+
+dReLU with the bias gradient, GELU' from the stored pre-activation, against the
+fp64 oracle.  Tolerances:
+  * dReLU's dpre is bit-exact (grad times 0 or 1); GELU's dpre within one unit in
+    the last place of its type (at least the subnormal quantum) plus the kernel's
+    GELU' error (4e-7·|grad|).
+  * dbias (fp32 sums in a fixed order) within 2^-24·(M + 16)·Σ_m|dpre| — the bound of
+    a sequential fp32 sum of M terms — plus 4e-7·Σ_m|grad| for GELU'.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+GELU_GRAD_ABS = 4e-7  # bound on |GELU'(v) in fp32 - GELU'(v)| (erf to ~2e-7, e^(-v²/2) to ~2^-22)
+# one unit in the last place at the bottom of each type's range (the subnormal quantum):
+# there a rounding of a value within GELU_GRAD_ABS of a midpoint moves by this much
+ULP_MIN = {"f16": 2.0 ** -24, "bf16": 2.0 ** -133, "f32": 2.0 ** -149}
+
+
+@pytest.fixture(scope="module")
+def fl():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import gemm_bias_activation_tcgen05_b200 as m
+    return m
+
+
+def _workspace(fl, M, N, dtype):
+    n = fl.fl_bias_grad_workspace_size(M, N, dtype)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device="cuda"), n
+
+
+def _check_dbias(got, want_exact, abs_terms, M, grad_abs=None, what=""):
+    tol = 2.0 ** -24 * (M + 16) * abs_terms + 1e-30
+    if grad_abs is not None:
+        tol = tol + GELU_GRAD_ABS * grad_abs
+    err = np.abs(got - want_exact)
+    assert np.all(err <= tol), f"{what}: dbias error {err.max():.3e} above its bound at {err.argmax()}"
+
+
+def _grad(M, N, dtype, seed, ld=None):
+    g = torch.Generator().manual_seed(seed)
+    ld = ld or N
+    return torch.randn(M, ld, generator=g, dtype=torch.float32).to(P.TD[dtype])
+
+
+@pytest.mark.parametrize("M,N,dtype", [(300, 520, "bf16"), (257, 77, "f16"), (64, 1000, "f32"), (5, 4096, "bf16"),
+                                       (1000, 24, "bf16")])
+def test_drelu_bgrad(fl, M, N, dtype):
+    g = torch.Generator().manual_seed(M + N)
+    v = torch.randn(M, N, generator=g, dtype=torch.float64).numpy()
+    v[0, :5] = 0.0  # ReLU'(0) = 0
+    mask = oracle.relu_aux_mask(v)
+    grad = _grad(M, N, dtype, M * 7 + N)
+    dmask = torch.from_numpy(mask.view(np.int32)).cuda()
+    dgrad = grad.cuda()
+    dpre = P.poison((M, N), dtype)
+    dbias = torch.full((N,), float("nan"), dtype=torch.float32, device="cuda")
+    ws, nbytes = _workspace(fl, M, N, dtype)
+    for rep in range(2):  # the workspace is left ready for the next call
+        fl.fl_drelu_bgrad(dgrad, dmask, dpre, dbias, M, N, dtype, ws, nbytes)
+        torch.cuda.synchronize()
+        dv, db = oracle.drelu_bgrad(P.to64(grad), mask, N, dtype)
+        assert np.array_equal(P.to64(dpre), dv), f"dpre differs (launch {rep})"
+        _check_dbias(P.to64(dbias), db, np.abs(dv).sum(axis=0), M, what=f"drelu_bgrad {M}x{N} {dtype} launch {rep}")
+
+
+def test_drelu_bgrad_without_bias_grad_and_aliasing(fl):
+    M, N = 130, 300
+    g = torch.Generator().manual_seed(3)
+    v = torch.randn(M, N, generator=g, dtype=torch.float64).numpy()
+    mask = oracle.relu_aux_mask(v)
+    grad = _grad(M, N, "bf16", 4)
+    buf = grad.cuda()
+    fl.fl_drelu_bgrad(buf, torch.from_numpy(mask.view(np.int32)).cuda(), buf, None, M, N, "bf16")  # dpre = grad
+    torch.cuda.synchronize()
+    assert np.array_equal(P.to64(buf), oracle.drelu(P.to64(grad), mask, N, "bf16"))
+
+
+def test_relu_aux_4096_backward_with_bias_grad(fl):
+    w = workloads.get("relu_aux_4096")
+    M, N = w.M, w.N
+    g = torch.Generator().manual_seed(11)
+    v = torch.randn(M, N, generator=g, dtype=torch.float32).numpy().astype(np.float64)
+    mask = oracle.relu_aux_mask(v)
+    grad = _grad(M, N, "bf16", 12)
+    dpre = P.poison((M, N), "bf16")
+    dbias = torch.empty(N, dtype=torch.float32, device="cuda")
+    ws, nbytes = _workspace(fl, M, N, "bf16")
+    fl.fl_drelu_bgrad(grad.cuda(), torch.from_numpy(mask.view(np.int32)).cuda(), dpre, dbias, M, N, "bf16", ws, nbytes)
+    torch.cuda.synchronize()
+    dv, db = oracle.drelu_bgrad(P.to64(grad), mask, N, "bf16")
+    assert np.array_equal(P.to64(dpre), dv)
+    _check_dbias(P.to64(dbias), db, np.abs(dv).sum(axis=0), M, what="drelu_bgrad 4096")
+
+
+@pytest.mark.parametrize("M,N,dtype", [(300, 520, "bf16"), (257, 77, "f16"), (64, 1000, "f32"), (2048, 4096, "bf16")])
+def test_dgelu_bgrad(fl, M, N, dtype):
+    g = torch.Generator().manual_seed(M * 3 + N)
+    v = (torch.randn(M, N, generator=g, dtype=torch.float32) * 3).to(P.TD[dtype])
+    grad = _grad(M, N, dtype, M + 5 * N)
+    dpre = P.poison((M, N), dtype)
+    dbias = torch.empty(N, dtype=torch.float32, device="cuda")
+    ws, nbytes = _workspace(fl, M, N, dtype)
+    fl.fl_dgelu_bgrad(grad.cuda(), v.cuda(), dpre, dbias, M, N, dtype, ws, nbytes)
+    torch.cuda.synchronize()
+    g64, v64 = P.to64(grad), P.to64(v)
+    dv, db = oracle.dgelu_bgrad(g64, v64, dtype)
+    err = np.abs(P.to64(dpre) - dv)
+    tol = P.ULP_REL[dtype] * np.abs(dv) + ULP_MIN[dtype] + 2 * GELU_GRAD_ABS * np.abs(g64)
+    assert np.all(err <= tol), f"dgelu dpre error {err.max():.3e}"
+    exact = g64 * oracle.gelu_erf_grad(v64)
+    _check_dbias(P.to64(dbias), db, np.abs(exact).sum(axis=0), M, np.abs(g64).sum(axis=0), f"dgelu_bgrad {M}x{N}")
+
+
+@pytest.mark.parametrize("M,N,K,out_dtype", [(300, 520, 200, "bf16"), (300, 520, 200, "f32"), (77, 1000, 1000, "bf16"),
+                                             (257, 136, 768, "f16")])
+def test_gelu_aux_forward_then_backward(fl, M, N, K, out_dtype):
+    """GELU_AUX_BIAS stores v; the GELU backward takes it as its input."""
+    inp = workloads.ragged_linear_inputs(M, N, K, "bf16", 31, bias_dtype="bf16")
+    ldo = -(-N // 8) * 8
+    out = P.poison((M, ldo), out_dtype)
+    vaux = P.poison((M, ldo), out_dtype)
+    plan = fl.Plan(M, N, K, kind="GELU_AUX_BIAS", out_dtype=out_dtype, lda=inp["A"].shape[1],
+                   ldb=inp["W"].shape[1], ldo=ldo)
+    try:
+        plan.execute(inp["A"].cuda(), inp["W"].cuda(), inp["bias"].cuda(), vaux, None, out)
+        assert plan.check() == fl.FL_OK, fl.fl_last_error()
+        info = plan.info()
+    finally:
+        plan.free()
+    y, aux, v, absdot = P.oracle_linear(A=inp["A"], W=inp["W"], bias=inp["bias"], epilogue="GELU_AUX_BIAS",
+                                        out_dtype=out_dtype, M=M, N=N, K=K)
+    P.check_close(P.to64(out[:, :N]), y, out_dtype, absdot, f"GELU_AUX out {info}")
+    P.check_close(P.to64(vaux[:, :N]), aux, out_dtype, absdot, f"GELU_AUX v {info}")
+    assert torch.isnan(vaux[:, N:].float()).all(), "pre-activation written into the row padding"
+    # backward from the stored v
+    grad = _grad(M, N, out_dtype, 41, ld=ldo).cuda()
+    dpre = P.poison((M, ldo), out_dtype)
+    dbias = torch.empty(N, dtype=torch.float32, device="cuda")
+    ws, nbytes = _workspace(fl, M, N, out_dtype)
+    fl.fl_dgelu_bgrad(grad, vaux, dpre, dbias, M, N, out_dtype, ws, nbytes, ld_grad=ldo, ld_v=ldo, ld_dpre=ldo)
+    torch.cuda.synchronize()
+    g64, v64 = P.to64(grad[:, :N]), P.to64(vaux[:, :N])
+    dv, db = oracle.dgelu_bgrad(g64, v64, out_dtype)
+    err = np.abs(P.to64(dpre[:, :N]) - dv)
+    assert np.all(err <= P.ULP_REL[out_dtype] * np.abs(dv) + ULP_MIN[out_dtype] + 2 * GELU_GRAD_ABS * np.abs(g64))
+    exact = g64 * oracle.gelu_erf_grad(v64)
+    _check_dbias(P.to64(dbias), db, np.abs(exact).sum(axis=0), M, np.abs(g64).sum(axis=0), "dgelu after GELU_AUX")
