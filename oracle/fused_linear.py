@@ -19,6 +19,8 @@ from scipy.special import erf as _erf
 GELU_TANH_C = math.sqrt(2.0 / math.pi)
 # [gelu] §2.2.2 and [mhc] §4.2: the cubic coefficient of the tanh form.
 GELU_TANH_A = 0.044715
+# [gelu] §2.2.2, "approximation 1": the sigmoid slope of x·σ(1.702x).
+GELU_SIGMOID_K = 1.702
 
 
 def gemm(A: np.ndarray, W: np.ndarray, b_major: int = 0) -> np.ndarray:
@@ -72,6 +74,13 @@ def gelu_tanh(v: np.ndarray) -> np.ndarray:
     return 0.5 * v * (1.0 + np.tanh(GELU_TANH_C * (v + GELU_TANH_A * v * v * v)))
 
 
+def gelu_sigmoid(v: np.ndarray) -> np.ndarray:
+    """Sigmoid form: x·σ(1.702·x) = x / (1 + e^(-1.702·x)) — [gelu] §2.2.2, approximation 1."""
+    v = np.asarray(v, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return v / (1.0 + np.exp(-GELU_SIGMOID_K * v))
+
+
 def activation(v: np.ndarray, kind: str) -> np.ndarray:
     """Apply the activation named by an epilogue kind (bias-only kinds are identity)."""
     if kind in ("NONE", "BIAS"):
@@ -82,6 +91,8 @@ def activation(v: np.ndarray, kind: str) -> np.ndarray:
         return gelu_erf(v)
     if kind in ("GELU_TANH_BIAS", "GELU_TANH"):
         return gelu_tanh(v)
+    if kind in ("GELU_SIGMOID_BIAS", "GELU_SIGMOID"):
+        return gelu_sigmoid(v)
     raise ValueError(kind)
 
 

@@ -227,6 +227,26 @@ def pin_geglu_identity(o):
     assert np.array_equal(y, hh)
 
 
+def pin_gelu_sigmoid_page_form(o):
+    """x·σ(1.702x) with the page's constant, per element against math.exp."""
+    k = _golden()["gelu_sigmoid_k"]["value"]
+    v = np.linspace(-20.0, 20.0, 161)
+    y = o.gelu_sigmoid(v)
+    for x, got in zip(v, y):
+        assert abs(got - x / (1.0 + math.exp(-k * x))) <= 1e-15 * max(1.0, abs(x))
+
+
+def pin_gelu_sigmoid_identities(o):
+    v = np.linspace(-8.0, 8.0, 161)
+    # σ(z) + σ(-z) = 1  ⇒  f(v) − f(−v) = v
+    assert np.max(np.abs(o.gelu_sigmoid(v) - o.gelu_sigmoid(-v) - v)) < 1e-14
+    assert o.gelu_sigmoid(np.array([0.0]))[0] == 0.0
+    assert abs(o.gelu_sigmoid(np.array([60.0]))[0] - 60.0) < 1e-12
+    assert abs(o.gelu_sigmoid(np.array([-60.0]))[0]) < 1e-40
+    # the activation kind routes to it
+    assert np.array_equal(o.activation(v, "GELU_SIGMOID_BIAS"), o.gelu_sigmoid(v))
+
+
 def pin_bias_grad_brute_force(o):
     r = _rng(11)
     M, N = 7, 9
@@ -337,6 +357,7 @@ def pin_fused_brute_force(o):
         "RELU_AUX_BIAS": lambda v: max(v, 0.0),
         "GELU_BIAS": lambda v: 0.5 * v * (1 + math.erf(v / math.sqrt(2.0))),
         "GELU_TANH_BIAS": lambda v: 0.5 * v * (1 + math.tanh(c * (v + 0.044715 * v ** 3))),
+        "GELU_SIGMOID_BIAS": lambda v: v / (1.0 + math.exp(-1.702 * v)),
     }
     for epi, f in acts.items():
         y, aux, v = o.fused_linear(A, W, b, epilogue=epi, out_dtype="f32", residual=res, scale=0.25)

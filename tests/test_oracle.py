@@ -30,7 +30,7 @@ def _namespace(**over):
     if ns is None:
         names = ["gemm", "add_bias", "relu", "gelu_erf", "gelu_tanh", "activation", "relu_aux_mask",
                  "residual_scale", "round_to", "fused_linear", "geglu_h", "geglu_mlp", "drelu",
-                 "bias_grad", "drelu_bgrad", "gelu_erf_grad", "dgelu", "dgelu_bgrad"]
+                 "bias_grad", "drelu_bgrad", "gelu_erf_grad", "dgelu", "dgelu_bgrad", "gelu_sigmoid"]
         ns = types.SimpleNamespace(**{k: getattr(oracle, k) for k in names})
     for k, v in over.items():
         setattr(ns, k, v)
@@ -57,6 +57,8 @@ def _namespace(**over):
             return ns.relu(v)
         if kind in ("GELU_BIAS", "GELU_AUX_BIAS", "GELU"):
             return ns.gelu_erf(v)
+        if kind in ("GELU_SIGMOID_BIAS", "GELU_SIGMOID"):
+            return ns.gelu_sigmoid(v)
         return ns.gelu_tanh(v)
 
     def drelu_bgrad(grad, aux, N, out_dtype="bf16"):
@@ -140,6 +142,8 @@ MUTANTS = {
                                - np.asarray(v, float) * np.exp(-0.5 * np.asarray(v, float) ** 2) / math.sqrt(2 * math.pi)),
     "gelu_grad_no_half_exponent": dict(gelu_erf_grad=lambda v: 0.5 * (1.0 + erf(np.asarray(v, float) / math.sqrt(2.0)))
                                        + np.asarray(v, float) * np.exp(-np.asarray(v, float) ** 2) / math.sqrt(2 * math.pi)),
+    "gelu_sigmoid_slope_one": dict(gelu_sigmoid=lambda v: np.asarray(v, float) / (1.0 + np.exp(-np.asarray(v, float)))),
+    "gelu_sigmoid_sign": dict(gelu_sigmoid=lambda v: np.asarray(v, float) / (1.0 + np.exp(1.702 * np.asarray(v, float)))),
     "drelu_inverted": dict(drelu=lambda grad, aux, N, od="bf16": oracle.round_to(
         np.asarray(grad, float)[:, :N] - oracle.drelu(grad, aux, N, od), od)),
 }
