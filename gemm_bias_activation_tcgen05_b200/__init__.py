@@ -29,7 +29,8 @@ STATUS_NAMES = {0: "FL_OK", 1: "FL_ERR_INVALID_ARG", 2: "FL_ERR_UNSUPPORTED", 3:
 FL_F16, FL_BF16, FL_F32 = 0, 1, 2
 FL_COMPUTE_32F, FL_COMPUTE_32F_3XTF32 = 0, 1
 EPILOGUES = {"NONE": 0, "BIAS": 1, "RELU_BIAS": 2, "RELU_AUX_BIAS": 3, "GELU_BIAS": 4,
-             "GELU_TANH_BIAS": 5, "GEGLU_TANH": 6, "GELU_AUX_BIAS": 7}
+             "GELU_TANH_BIAS": 5, "GEGLU_TANH": 6, "GELU_AUX_BIAS": 7,
+             "GELU_SIGMOID_BIAS": 8}
 DTYPES = {"f16": FL_F16, "bf16": FL_BF16, "f32": FL_F32}
 COMPUTES = {"32F": FL_COMPUTE_32F, "32F_3XTF32": FL_COMPUTE_32F_3XTF32}
 

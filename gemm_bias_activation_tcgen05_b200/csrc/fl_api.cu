@@ -134,6 +134,7 @@ static const void* pick_kernel_tf32_pair(int act, int out) {
     case ACT_RELU: return pick_tf32_pair<ACT_RELU>(out);
     case ACT_GELU: return pick_tf32_pair<ACT_GELU>(out);
     case ACT_GELU_TANH: return pick_tf32_pair<ACT_GELU_TANH>(out);
+    case ACT_GELU_SIGMOID: return pick_tf32_pair<ACT_GELU_SIGMOID>(out);
     default: return nullptr;
   }
 }
@@ -143,6 +144,7 @@ static const void* pick_kernel_tf32(int act, int out) {
     case ACT_RELU: return pick_tf32<ACT_RELU>(out);
     case ACT_GELU: return pick_tf32<ACT_GELU>(out);
     case ACT_GELU_TANH: return pick_tf32<ACT_GELU_TANH>(out);
+    case ACT_GELU_SIGMOID: return pick_tf32<ACT_GELU_SIGMOID>(out);
     default: return nullptr;
   }
 }
@@ -165,6 +167,7 @@ static const void* pick_kernel_pair(int act, int out) {
     case ACT_RELU: return pick_pair<ACT_RELU>(out);
     case ACT_GELU: return pick_pair<ACT_GELU>(out);
     case ACT_GELU_TANH: return pick_pair<ACT_GELU_TANH>(out);
+    case ACT_GELU_SIGMOID: return pick_pair<ACT_GELU_SIGMOID>(out);
     default: return pick_pair<ACT_GEGLU>(out);
   }
 }
@@ -174,6 +177,7 @@ static const void* pick_kernel(int act, int out, bool swap) {
     case ACT_RELU: return pick_out<ACT_RELU>(out, swap);
     case ACT_GELU: return pick_out<ACT_GELU>(out, swap);
     case ACT_GELU_TANH: return pick_out<ACT_GELU_TANH>(out, swap);
+    case ACT_GELU_SIGMOID: return pick_out<ACT_GELU_SIGMOID>(out, swap);
     default: return swap ? nullptr : pick_out<ACT_GEGLU>(out, false);
   }
 }
@@ -219,6 +223,7 @@ static int act_of(int kind) {
     case FL_EPI_GELU_BIAS:
     case FL_EPI_GELU_AUX_BIAS: return ACT_GELU;
     case FL_EPI_GELU_TANH_BIAS: return ACT_GELU_TANH;
+    case FL_EPI_GELU_SIGMOID_BIAS: return ACT_GELU_SIGMOID;
     case FL_EPI_GEGLU_TANH: return ACT_GEGLU;
     default: return ACT_NONE;
   }
@@ -385,7 +390,7 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
                                            (long long)M, (long long)N, (long long)K);
   if (M > (1LL << 31) - 256 || N > (1LL << 30) || K > (1LL << 31) - 256)
     return fail(FL_ERR_INVALID_ARG, "fl_plan: dimension too large");
-  if (epi->kind < FL_EPI_NONE || epi->kind > FL_EPI_GELU_AUX_BIAS)
+  if (epi->kind < FL_EPI_NONE || epi->kind > FL_EPI_GELU_SIGMOID_BIAS)
     return fail(FL_ERR_INVALID_ARG, "fl_plan: unknown epilogue kind %d", epi->kind);
   for (int i = 0; i < 3; ++i)
     if (epi->reserved[i] != 0) return fail(FL_ERR_INVALID_ARG, "fl_plan: reserved fields must be 0");
@@ -855,6 +860,8 @@ extern "C" fl_status fl_execute(fl_plan_t p, const void* A, const void* W, const
       st = step(EW_GELU, nullptr, 0, 0);
     } else if (p->act == ACT_GELU_TANH) {
       st = step(EW_GELU_TANH, nullptr, 0, 0);
+    } else if (p->act == ACT_GELU_SIGMOID) {
+      st = step(EW_GELU_SIGMOID, nullptr, 0, 0);
     }
     if (st) return st;
   }
@@ -1086,7 +1093,7 @@ extern "C" fl_status fl_execute_noalloc(int64_t M, int64_t N, int64_t K, int32_t
   if (M < 1 || N < 1 || K < 0) return fail(FL_ERR_INVALID_ARG, "%s: need M>=1, N>=1, K>=0", who);
   if (M > (1LL << 31) - 256 || N > (1LL << 30) || K > (1LL << 31) - 256)
     return fail(FL_ERR_INVALID_ARG, "%s: dimension too large", who);
-  if (epi->kind < FL_EPI_NONE || epi->kind > FL_EPI_GELU_AUX_BIAS)
+  if (epi->kind < FL_EPI_NONE || epi->kind > FL_EPI_GELU_SIGMOID_BIAS)
     return fail(FL_ERR_INVALID_ARG, "%s: unknown epilogue kind %d", who, epi->kind);
   for (int i = 0; i < 3; ++i)
     if (epi->reserved[i] != 0) return fail(FL_ERR_INVALID_ARG, "%s: reserved fields must be 0", who);

@@ -267,7 +267,8 @@ enum EwOp : int {
   EW_GELU_TANH = 4,
   EW_RESIDUAL = 5, // y = x + r[m,n]
   EW_SCALE = 6,    // y = x * s
-  EW_GEGLU_MUL = 7 // y[m,n] = gelu_tanh(x[m,n]) * u[m,n]  (u = operand)
+  EW_GEGLU_MUL = 7, // y[m,n] = gelu_tanh(x[m,n]) * u[m,n]  (u = operand)
+  EW_GELU_SIGMOID = 8
 };
 
 struct EwParams {
@@ -350,6 +351,7 @@ __global__ void __launch_bounds__(256) fl_ew_step_kernel(const EwParams P) {
           break;
         case EW_GELU: y = gelu_erf_f(x); break;
         case EW_GELU_TANH: y = gelu_tanh_f<DT != DT_F32>(x); break;
+        case EW_GELU_SIGMOID: y = gelu_sigmoid_f(x); break;
         case EW_RESIDUAL: y = x + opv; break;
         case EW_SCALE: y = x * P.scale; break;
         default: y = gelu_tanh_f<DT != DT_F32>(x) * opv; break;

@@ -34,7 +34,7 @@
 
 namespace fl {
 
-enum Act : int { ACT_NONE = 0, ACT_RELU = 1, ACT_GELU = 2, ACT_GELU_TANH = 3, ACT_GEGLU = 4 };
+enum Act : int { ACT_NONE = 0, ACT_RELU = 1, ACT_GELU = 2, ACT_GELU_TANH = 3, ACT_GEGLU = 4, ACT_GELU_SIGMOID = 5 };
 enum DType : int { DT_F16 = 0, DT_BF16 = 1, DT_F32 = 2 };
 
 constexpr int kEpiWarp0 = 2;                 // warps 0,1: TMA producer, UMMA issuer
@@ -180,12 +180,19 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
   return 0.5f * x * (1.0f + (LOWP ? tanh_approx(u) : tanh_ex2(u)));
 }
 
+// GELU's sigmoid form x·σ(1.702x) = x / (1 + 2^(-1.702·log2(e)·x)), reciprocal and
+// power of two on the special-function unit (relative error near 2^-22)
+__device__ __forceinline__ float gelu_sigmoid_f(float x) {
+  return x * rcp_approx(1.0f + ex2_approx(-1.702f * 1.4426950408889634f * x));
+}
+
 template <int ACT, bool LOWP = false>
 __device__ __forceinline__ float activate(float v, float u) {
   if constexpr (ACT == ACT_RELU) return fmaxf(v, 0.0f);
   if constexpr (ACT == ACT_GELU) return gelu_erf_f(v);
   if constexpr (ACT == ACT_GELU_TANH) return gelu_tanh_f<LOWP>(v);
   if constexpr (ACT == ACT_GEGLU) return gelu_tanh_f<LOWP>(v) * u;
+  if constexpr (ACT == ACT_GELU_SIGMOID) return gelu_sigmoid_f(v);
   return v;
 }
 

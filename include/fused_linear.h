@@ -70,6 +70,7 @@ typedef enum { FL_COMPUTE_32F = 0, FL_COMPUTE_32F_3XTF32 = 1 } fl_compute;
  *   GELU_BIAS       y = gelu_erf(acc + bias)   = 0.5·v·(1 + erf(v/√2))
  *   GELU_TANH_BIAS  y = gelu_tanh(acc + bias)  = 0.5·v·(1 + tanh(√(2/π)(v + 0.044715 v³)))
  *   GEGLU_TANH      W is the stacked [2N, K] matrix [Wg; Wu]; y = gelu_tanh(A·Wgᵀ)·(A·Wuᵀ)
+ *   GELU_SIGMOID_BIAS y = v·σ(1.702·v), the sigmoid approximation of GELU ([gelu] §2.2.2)
  *   GELU_AUX_BIAS   as GELU_BIAS, and aux = v = acc + bias stored in the output type, the
  *                   input of the GELU backward (fl_dgelu_bgrad); [epilog] keeps forward
  *                   state for the backward pass, [gelu] §2.2.1 fuses the backward too
@@ -82,7 +83,8 @@ typedef enum {
   FL_EPI_GELU_BIAS = 4,
   FL_EPI_GELU_TANH_BIAS = 5,
   FL_EPI_GEGLU_TANH = 6,
-  FL_EPI_GELU_AUX_BIAS = 7
+  FL_EPI_GELU_AUX_BIAS = 7,
+  FL_EPI_GELU_SIGMOID_BIAS = 8
 } fl_epi_kind;
 
 /* The "epilog" argument of fl_plan.  Zero-initialise, then set fields. */

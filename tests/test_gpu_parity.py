@@ -60,7 +60,8 @@ def test_multi_kblock_multi_tile(fl):
 
 
 @pytest.mark.parametrize("out_dtype", ["bf16", "f32", "f16"])
-@pytest.mark.parametrize("epilogue", ["NONE", "BIAS", "RELU_BIAS", "RELU_AUX_BIAS", "GELU_BIAS", "GELU_TANH_BIAS"])
+@pytest.mark.parametrize("epilogue", ["NONE", "BIAS", "RELU_BIAS", "RELU_AUX_BIAS", "GELU_BIAS", "GELU_TANH_BIAS",
+                                      "GELU_SIGMOID_BIAS"])
 def test_epilogues_ragged(fl, epilogue, out_dtype):
     # ragged in every dimension: M, N not tile multiples, K not a multiple of 64
     _linear_case(fl, 300, 520, 200, epilogue=epilogue, out_dtype=out_dtype, seed=11)
@@ -91,6 +92,13 @@ def test_small_m_swap_split_k(fl, M):
     assert got["info"]["swap_ab"] == 1
 
 
+@pytest.mark.parametrize("M,dtype", [(9, "bf16"), (100, "f16"), (200, "f32")])
+def test_sigmoid_gelu_layouts(fl, M, dtype):
+    # swap-AB (M <= 128, 16-bit), and the 3xTF32 pair path for fp32 operands
+    got = _linear_case(fl, M, 1000, 520, dtype=dtype, epilogue="GELU_SIGMOID_BIAS", out_dtype="f32", seed=M)
+    assert got["info"]["swap_ab"] == (1 if dtype != "f32" else 0)
+
+
 @pytest.mark.parametrize("M", [16, 100])
 def test_small_m_relu_aux(fl, M):
     _linear_case(fl, M, 520, 264, epilogue="RELU_AUX_BIAS", out_dtype="bf16", seed=3)
@@ -118,7 +126,7 @@ def test_geglu_dual(fl, M, N, K):
     P.check_close(got["out"], h, "bf16", absdot, f"geglu {M}x{N}x{K}")
 
 
-@pytest.mark.parametrize("epilogue", ["RELU_AUX_BIAS", "GELU_TANH_BIAS", "NONE"])
+@pytest.mark.parametrize("epilogue", ["RELU_AUX_BIAS", "GELU_TANH_BIAS", "NONE", "GELU_SIGMOID_BIAS"])
 def test_unfused_twin(fl, epilogue):
     got = _linear_case(fl, 256, 384, 192, epilogue=epilogue, out_dtype="bf16", unfused=True, seed=7)
     assert got["info"]["launches_per_execute"] >= 1
