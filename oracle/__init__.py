@@ -28,6 +28,6 @@ force, closed forms, identities or an independent library routine; none is
 from .fused_linear import (  # noqa: F401
     gemm, add_bias, relu, gelu_erf, gelu_tanh, activation, relu_aux_mask,
     residual_scale, round_to, fused_linear, geglu_h, geglu_mlp, drelu,
-    bias_grad, drelu_bgrad, gelu_erf_grad, dgelu, dgelu_bgrad, gelu_sigmoid,
+    bias_grad, drelu_bgrad, gelu_erf_grad, dgelu, dgelu_bgrad, gelu_sigmoid, layer_norm,
     GELU_TANH_C, GELU_TANH_A, GELU_SIGMOID_K,
 )

@@ -252,3 +252,18 @@ def dgelu_bgrad(grad, v, out_dtype: str = "bf16"):
     """(dv rounded to out_dtype, db = Σ_m grad·GELU'(v) in float64, before any rounding)."""
     exact = np.asarray(grad, dtype=np.float64) * gelu_erf_grad(v)
     return round_to(exact, out_dtype), bias_grad(exact)
+
+
+# ---------------------------------------------------------------- LayerNorm after the tail
+def layer_norm(x, gamma, beta, eps: float, out_dtype: str = "f32"):
+    """z = (x − μ)/√(σ² + ε)·γ + β over the last dimension, rounded once to out_dtype.
+
+    [mhc] §3.2: LayerNorm reduces a row to its mean and variance, then normalises
+    the row; the BERT tail (bias → GELU → + residual → × 0.5) is followed by it.
+    μ = mean over the row, σ² = mean((x − μ)²) (the population variance), in fp64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    z = (x - mu) / np.sqrt(var + float(eps)) * np.asarray(gamma, dtype=np.float64) + np.asarray(beta, dtype=np.float64)
+    return round_to(z, out_dtype)

@@ -247,6 +247,31 @@ def pin_gelu_sigmoid_identities(o):
     assert np.array_equal(o.activation(v, "GELU_SIGMOID_BIAS"), o.gelu_sigmoid(v))
 
 
+def pin_layer_norm(o):
+    r = _rng(15)
+    M, N = 6, 40
+    x = r.standard_normal((M, N)) * 3 + 1.5
+    g = r.standard_normal(N)
+    b = r.standard_normal(N)
+    z = o.layer_norm(x, g, b, 1e-5, "f32")
+    # per row against loops
+    for m in range(M):
+        mu = sum(x[m]) / N
+        var = sum((v - mu) ** 2 for v in x[m]) / N
+        for n in range(N):
+            ref = (x[m, n] - mu) / math.sqrt(var + 1e-5) * g[n] + b[n]
+            assert abs(z[m, n] - np.float32(ref)) <= 1e-6 * max(1.0, abs(ref))
+    # γ = 1, β = 0: each row has mean 0 and population variance var/(var + ε)
+    z1 = o.layer_norm(x, np.ones(N), np.zeros(N), 0.0, "f32")
+    assert np.max(np.abs(z1.mean(axis=1))) < 1e-6
+    assert np.max(np.abs(z1.var(axis=1) - 1.0)) < 1e-5
+    # against torch's layer_norm in fp64
+    zt = F.layer_norm(torch.from_numpy(x), (N,), torch.from_numpy(g), torch.from_numpy(b), eps=1e-12).numpy()
+    assert np.max(np.abs(o.layer_norm(x, g, b, 1e-12, "f32") - o.round_to(zt, "f32"))) < 1e-6
+    # invariant to shifting the row
+    assert np.max(np.abs(o.layer_norm(x + 100.0, g, b, 1e-5, "f32") - z)) < 1e-5
+
+
 def pin_bias_grad_brute_force(o):
     r = _rng(11)
     M, N = 7, 9

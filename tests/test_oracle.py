@@ -30,7 +30,7 @@ def _namespace(**over):
     if ns is None:
         names = ["gemm", "add_bias", "relu", "gelu_erf", "gelu_tanh", "activation", "relu_aux_mask",
                  "residual_scale", "round_to", "fused_linear", "geglu_h", "geglu_mlp", "drelu",
-                 "bias_grad", "drelu_bgrad", "gelu_erf_grad", "dgelu", "dgelu_bgrad", "gelu_sigmoid"]
+                 "bias_grad", "drelu_bgrad", "gelu_erf_grad", "dgelu", "dgelu_bgrad", "gelu_sigmoid", "layer_norm"]
         ns = types.SimpleNamespace(**{k: getattr(oracle, k) for k in names})
     for k, v in over.items():
         setattr(ns, k, v)
@@ -144,6 +144,15 @@ MUTANTS = {
                                        + np.asarray(v, float) * np.exp(-np.asarray(v, float) ** 2) / math.sqrt(2 * math.pi)),
     "gelu_sigmoid_slope_one": dict(gelu_sigmoid=lambda v: np.asarray(v, float) / (1.0 + np.exp(-np.asarray(v, float)))),
     "gelu_sigmoid_sign": dict(gelu_sigmoid=lambda v: np.asarray(v, float) / (1.0 + np.exp(1.702 * np.asarray(v, float)))),
+    "layer_norm_sample_variance": dict(layer_norm=lambda x, g, b, eps, od="f32": oracle.round_to(
+        (np.asarray(x, float) - np.asarray(x, float).mean(-1, keepdims=True))
+        / np.sqrt(np.asarray(x, float).var(-1, ddof=1, keepdims=True) + eps) * g + b, od)),
+    "layer_norm_eps_outside_sqrt": dict(layer_norm=lambda x, g, b, eps, od="f32": oracle.round_to(
+        (np.asarray(x, float) - np.asarray(x, float).mean(-1, keepdims=True))
+        / (np.sqrt(np.asarray(x, float).var(-1, keepdims=True)) + eps) * g + b, od)),
+    "layer_norm_no_beta": dict(layer_norm=lambda x, g, b, eps, od="f32": oracle.round_to(
+        (np.asarray(x, float) - np.asarray(x, float).mean(-1, keepdims=True))
+        / np.sqrt(np.asarray(x, float).var(-1, keepdims=True) + eps) * g, od)),
     "drelu_inverted": dict(drelu=lambda grad, aux, N, od="bf16": oracle.round_to(
         np.asarray(grad, float)[:, :N] - oracle.drelu(grad, aux, N, od), od)),
 }
