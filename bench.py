@@ -351,7 +351,8 @@ def run_ours(args):
         "roofline": roofline,
         "clocks": clk.summary(),
         "breakdown": breakdown,
-        "backward": time_backward(fl, pk),
+        "hbm_kernels": time_backward(fl, pk),
+        "gelu_sigmoid_1024x3072x768_bf16": time_gelu_sigmoid(fl, pk),
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
@@ -384,8 +385,9 @@ def time_single_launch(suite, it, stream, sh, reps):
 
 
 def time_backward(fl, pk, reps=10):
-    """The backward kernels with the fused bias gradient on the relu_aux_4096 shape
-    (4096 x 4096 bf16), each launch after a 256 MB L2 flush: us, achieved GB/s of the
+    """The HBM-bound kernels beside the fused layer: the backward with the fused bias
+    gradient on the relu_aux_4096 shape (4096 x 4096 bf16) and the LayerNorm of the
+    tail_m2048 output, each launch after a 256 MB L2 flush: us, achieved GB/s of the
     algorithmic bytes, and the fraction of the measured HBM copy bandwidth."""
     import torch
     M = N = 4096
@@ -407,6 +409,15 @@ def time_backward(fl, pk, reps=10):
                                                                  stream=sh),
                                        3 * M * N * 2 + 4 * N),
     }
+    # LayerNorm of the BERT-tail output rows (tail_m2048: [2048, 4096] fp32 -> bf16)
+    Ml, Nl = 2048, 4096
+    y = torch.randn(Ml, Nl, generator=g).cuda()
+    gam = torch.ones(Nl, device="cuda")
+    bet = torch.zeros(Nl, device="cuda")
+    zl = torch.empty(Ml, Nl, dtype=torch.bfloat16, device="cuda")
+    runs["layernorm_2048x4096_f32_to_bf16"] = (
+        lambda: fl.fl_layernorm(y, gam, bet, zl, Ml, Nl, "f32", "bf16", "f32", eps=1e-12, stream=sh),
+        Ml * Nl * (4 + 2) + 2 * 4 * Nl)
     out = {}
     for name, (fn, algo_bytes) in runs.items():
         fn()
@@ -424,6 +435,35 @@ def time_backward(fl, pk, reps=10):
                      "frac_of_hbm": round(gbs / pk["hbm_gbs"], 3)}
     del flush
     return out
+
+
+def time_gelu_sigmoid(fl, pk, reps=10):
+    """The GELU_SIGMOID_BIAS epilogue on the [gelu] unit-test shape (x [1024,768],
+    W [3072,768], bf16 out), each launch after a 256 MB L2 flush."""
+    import torch
+    import workloads
+    M, N, K = 1024, 3072, 768
+    inp = workloads.ragged_linear_inputs(M, N, K, "bf16", 3, bias_dtype="bf16", pad=1)
+    A, W, b = inp["A"].cuda(), inp["W"].cuda(), inp["bias"].cuda()
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    plan = fl.Plan(M, N, K, kind="GELU_SIGMOID_BIAS", out_dtype="bf16")
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device="cuda")
+    try:
+        plan.execute(A, W, b, out=out)
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, e in evs:
+            flush.zero_()
+            a.record()
+            plan.execute(A, W, b, out=out)
+            e.record()
+        torch.cuda.synchronize()
+        assert plan.check() == fl.FL_OK
+    finally:
+        plan.free()
+    ms = sum(a.elapsed_time(e) for a, e in evs) / reps
+    tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+    return {"us": round(ms * 1e3, 2), "tflops": round(tf, 1), "frac_of_bf16_burst": round(tf / pk["bf16_tflops"], 3)}
 
 
 def profiled_traffic():

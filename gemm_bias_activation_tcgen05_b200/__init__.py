@@ -9,7 +9,7 @@ without a B200.
 The entry points keep the C names: ``fl_plan``, ``fl_execute``, ``fl_free``,
 ``fl_relu_backward``, ``fl_check_status``, ``fl_get_plan_info``,
 ``fl_last_error``, ``fl_set_wait_limit_ns``, ``fl_execute_noalloc``, ``fl_bias_grad_workspace_size``,
-``fl_drelu_bgrad``, ``fl_dgelu_bgrad``.  ``Plan`` is a small owner of one
+``fl_drelu_bgrad``, ``fl_dgelu_bgrad``, ``fl_layernorm``.  ``Plan`` is a small owner of one
 plan handle (the cuBLASLt epilog page's Matmul → plan → execute → free).
 """
 from __future__ import annotations
@@ -36,7 +36,7 @@ COMPUTES = {"32F": FL_COMPUTE_32F, "32F_3XTF32": FL_COMPUTE_32F_3XTF32}
 
 EXPORTED = ["fl_plan", "fl_execute", "fl_relu_backward", "fl_check_status", "fl_get_plan_info",
             "fl_free", "fl_last_error", "fl_set_wait_limit_ns", "fl_execute_noalloc",
-            "fl_bias_grad_workspace_size", "fl_drelu_bgrad", "fl_dgelu_bgrad"]
+            "fl_bias_grad_workspace_size", "fl_drelu_bgrad", "fl_dgelu_bgrad", "fl_layernorm"]
 
 
 class fl_epilogue_desc(ctypes.Structure):
@@ -87,6 +87,8 @@ def _load() -> ctypes.CDLL:
     lib.fl_drelu_bgrad.restype = i32
     lib.fl_dgelu_bgrad.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, vp, ctypes.c_size_t, vp]
     lib.fl_dgelu_bgrad.restype = i32
+    lib.fl_layernorm.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i32, i32, i32, ctypes.c_float, vp]
+    lib.fl_layernorm.restype = i32
     return lib
 
 
@@ -196,6 +198,13 @@ def fl_dgelu_bgrad(grad, v, dpre, dbias, M: int, N: int, dtype: str, workspace=N
     _check(LIB.fl_dgelu_bgrad(_ptr(grad), _ptr(v), _ptr(dpre), _ptr(dbias), int(M), int(N), int(ld_grad),
                               int(ld_v), int(ld_dpre), DTYPES[dtype], _ptr(workspace), int(workspace_bytes),
                               _stream(stream)), "fl_dgelu_bgrad")
+
+
+def fl_layernorm(x, gamma, beta, z, M: int, N: int, x_dtype: str, z_dtype: str, param_dtype: str = "f32",
+                 eps: float = 1e-12, ld_x: int = 0, ld_z: int = 0, stream=None) -> None:
+    _check(LIB.fl_layernorm(_ptr(x), _ptr(gamma), _ptr(beta), _ptr(z), int(M), int(N), int(ld_x), int(ld_z),
+                            DTYPES[x_dtype], DTYPES[z_dtype], DTYPES[param_dtype], float(eps), _stream(stream)),
+           "fl_layernorm")
 
 
 def fl_check_status(plan: int, stream=None) -> int:

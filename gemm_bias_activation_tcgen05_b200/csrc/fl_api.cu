@@ -1033,6 +1033,53 @@ extern "C" fl_status fl_dgelu_bgrad(const void* grad, const void* v, void* dpre,
                    workspace, workspace_bytes, stream);
 }
 
+// ------------------------------------------------------------------ LayerNorm after the tail
+template <int XT>
+static cudaError_t launch_ln(int z_dtype, unsigned grid, cudaStream_t s, const LnParams& P) {
+  if (z_dtype == FL_BF16) return launch_pdl(fl_layernorm_kernel<XT, DT_BF16>, dim3(grid), s, P);
+  if (z_dtype == FL_F16) return launch_pdl(fl_layernorm_kernel<XT, DT_F16>, dim3(grid), s, P);
+  return launch_pdl(fl_layernorm_kernel<XT, DT_F32>, dim3(grid), s, P);
+}
+
+extern "C" fl_status fl_layernorm(const void* x, const void* gamma, const void* beta, void* z, int64_t M, int64_t N,
+                                  int64_t ld_x, int64_t ld_z, int32_t x_dtype, int32_t z_dtype, int32_t param_dtype,
+                                  float eps, void* stream_) {
+  g_err[0] = 0;
+  const char* who = "fl_layernorm";
+  if (!x || !z) return fail(FL_ERR_INVALID_ARG, "%s: null x or z", who);
+  if (M < 0 || N < 0) return fail(FL_ERR_INVALID_ARG, "%s: negative size", who);
+  for (int dt : {x_dtype, z_dtype, param_dtype})
+    if (dt != FL_F16 && dt != FL_BF16 && dt != FL_F32) return fail(FL_ERR_INVALID_ARG, "%s: unknown dtype %d", who, dt);
+  if (!(eps >= 0.0f)) return fail(FL_ERR_INVALID_ARG, "%s: eps must be >= 0", who);
+  if (M > 0x7fffffffLL) return fail(FL_ERR_INVALID_ARG, "%s: more than 2^31-1 rows", who);
+  if (ld_x == 0) ld_x = N;
+  if (ld_z == 0) ld_z = N;
+  if (ld_x < N || ld_z < N) return fail(FL_ERR_INVALID_ARG, "%s: leading dimension < N", who);
+  const int ex = esize(x_dtype), ez = esize(z_dtype), ep = esize(param_dtype);
+  if (reinterpret_cast<uintptr_t>(x) % ex || reinterpret_cast<uintptr_t>(z) % ez ||
+      (gamma && reinterpret_cast<uintptr_t>(gamma) % ep) || (beta && reinterpret_cast<uintptr_t>(beta) % ep))
+    return fail(FL_ERR_ALIGNMENT, "%s: misaligned pointer", who);
+  if (M == 0 || N == 0) return FL_OK;
+  LnParams P{};
+  P.x = x;
+  P.gamma = gamma;
+  P.beta = beta;
+  P.z = z;
+  P.M = M;
+  P.N = N;
+  P.ldx = ld_x;
+  P.ldz = ld_z;
+  P.param_dtype = param_dtype;
+  P.vec_ok = aligned16(x) && (ld_x * ex) % 16 == 0;
+  P.eps = eps;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+  cudaError_t err = x_dtype == FL_BF16 ? launch_ln<DT_BF16>(z_dtype, (unsigned)M, s, P)
+                    : x_dtype == FL_F16 ? launch_ln<DT_F16>(z_dtype, (unsigned)M, s, P)
+                                        : launch_ln<DT_F32>(z_dtype, (unsigned)M, s, P);
+  if (err != cudaSuccess) return fail(FL_ERR_CUDA, "%s: kernel launch: %s", who, cudaGetErrorString(err));
+  return after_launch(s, who);
+}
+
 // ------------------------------------------------------------------ status
 extern "C" fl_status fl_check_status(fl_plan_t p, void* stream_) {
   if (!p) return fail(FL_ERR_INVALID_ARG, "fl_check_status: null plan");

@@ -182,6 +182,128 @@ __global__ void __launch_bounds__(256, 4) fl_bwd_bgrad_kernel(const BwdParams P)
   if (threadIdx.x == 0) P.counters[strip] = 0;  // ready for the next launch
 }
 
+// ---------------------------------------------------------------- LayerNorm after the tail
+struct LnParams {
+  const void* x;      // [M, ldx] of XT
+  const void* gamma;  // [N] of param_dtype, or null (1)
+  const void* beta;   // [N] of param_dtype, or null (0)
+  void* z;            // [M, ldz] of ZT (may alias x)
+  long long M, N, ldx, ldz;
+  int param_dtype, vec_ok;
+  float eps;
+};
+
+// Sum of one value per thread over the 256 threads, in a fixed order (butterfly in
+// each warp, then the eight warp sums in warp order).
+__device__ __forceinline__ float block_sum256(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();  // red is free (a previous call has been read)
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float s = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) s += red[w];
+  return s;
+}
+
+// z = (x − μ)·rstd·γ + β over each row (mHC page §3.2: the mean and variance of the
+// row, then the normalisation, in one kernel: one read and one write of the row).
+// One CTA of 256 threads per row.  A row of up to 256·4 16-byte vectors stays in
+// registers across the three steps (mean, Σ(x − μ)², normalise); a longer row is
+// read again for the later steps.
+template <int XT, int ZT>
+__global__ void __launch_bounds__(256, 4) fl_layernorm_kernel(const LnParams P) {
+  using TX = typename ElemT<XT>::T;
+  grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
+  constexpr int VE = 16 / sizeof(TX);  // elements per 16-byte vector of x
+  constexpr int VMAX = 4;              // vectors a thread keeps in registers
+  __shared__ float red[8];
+  const long long m = blockIdx.x;
+  const TX* x = reinterpret_cast<const TX*>(P.x) + m * P.ldx;
+  const long long N = P.N;
+  const int t = threadIdx.x;
+  const bool in_regs = N <= 256LL * VMAX * VE;
+  auto load_vec = [&](long long c0, float (&v)[VE]) {
+    if (P.vec_ok && c0 + VE <= N) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(x + c0));
+      const TX* e = reinterpret_cast<const TX*>(&q);
+#pragma unroll
+      for (int i = 0; i < VE; ++i) v[i] = static_cast<float>(e[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < VE; ++i) v[i] = (c0 + i < N) ? static_cast<float>(x[c0 + i]) : 0.0f;
+    }
+  };
+  float xv[VMAX][VE];
+  float s = 0.0f;
+  if (in_regs) {
+#pragma unroll
+    for (int k = 0; k < VMAX; ++k) {
+      const long long c0 = ((long long)k * 256 + t) * VE;
+#pragma unroll
+      for (int i = 0; i < VE; ++i) xv[k][i] = 0.0f;
+      if (c0 < N) load_vec(c0, xv[k]);
+#pragma unroll
+      for (int i = 0; i < VE; ++i) s += xv[k][i];
+    }
+  } else {
+    for (long long c0 = (long long)t * VE; c0 < N; c0 += 256LL * VE) {
+      float v[VE];
+      load_vec(c0, v);
+#pragma unroll
+      for (int i = 0; i < VE; ++i) s += v[i];
+    }
+  }
+  const float mean = block_sum256(s, red) / (float)N;
+  float q = 0.0f;
+  if (in_regs) {
+#pragma unroll
+    for (int k = 0; k < VMAX; ++k) {
+      const long long c0 = ((long long)k * 256 + t) * VE;
+#pragma unroll
+      for (int i = 0; i < VE; ++i)
+        if (c0 + i < N) q += (xv[k][i] - mean) * (xv[k][i] - mean);
+    }
+  } else {
+    for (long long c0 = (long long)t * VE; c0 < N; c0 += 256LL * VE) {
+      float v[VE];
+      load_vec(c0, v);
+#pragma unroll
+      for (int i = 0; i < VE; ++i)
+        if (c0 + i < N) q += (v[i] - mean) * (v[i] - mean);
+    }
+  }
+  const float var = block_sum256(q, red) / (float)N;
+  const float rstd = 1.0f / sqrtf(var + P.eps);
+  auto finish = [&](long long c0, const float (&v)[VE]) {
+#pragma unroll
+    for (int i = 0; i < VE; ++i) {
+      const long long c = c0 + i;
+      if (c < N) {
+        const float g = P.gamma ? load_elem(P.gamma, c, P.param_dtype) : 1.0f;
+        const float b = P.beta ? load_elem(P.beta, c, P.param_dtype) : 0.0f;
+        store_elem<ZT>(P.z, m * P.ldz + c, (v[i] - mean) * rstd * g + b);
+      }
+    }
+  };
+  if (in_regs) {
+#pragma unroll
+    for (int k = 0; k < VMAX; ++k) {
+      const long long c0 = ((long long)k * 256 + t) * VE;
+      if (c0 < N) finish(c0, xv[k]);
+    }
+  } else {
+    for (long long c0 = (long long)t * VE; c0 < N; c0 += 256LL * VE) {
+      float v[VE];
+      load_vec(c0, v);
+      finish(c0, v);
+    }
+  }
+}
+
 // ---------------------------------------------------------------- dReLU
 template <int DT>
 __global__ void __launch_bounds__(256) fl_relu_backward_kernel(const void* __restrict__ grad_,

@@ -172,6 +172,18 @@ fl_status fl_dgelu_bgrad(const void* grad, const void* v, void* dpre, float* dbi
                          int64_t ld_grad, int64_t ld_v, int64_t ld_dpre, int32_t dtype, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/* LayerNorm of each row, the step after the residual tail ([mhc] §3.2: the row's mean
+ * and variance and the normalisation in one kernel, one read and one write):
+ *   z[m,n] = (x[m,n] − μ_m)/√(σ²_m + eps)·gamma[n] + beta[n],
+ *   μ_m = mean of row m, σ²_m = mean of (x − μ_m)² (population variance), in fp32.
+ *   x  [M, ld_x] of x_dtype; z [M, ld_z] of z_dtype (may alias x when the types match)
+ *   gamma, beta [N] of param_dtype; null gamma = 1, null beta = 0
+ * Errors: FL_ERR_INVALID_ARG (null x/z, negative size, ld < N, eps < 0, M ≥ 2^31),
+ * FL_ERR_ALIGNMENT, FL_ERR_CUDA. */
+fl_status fl_layernorm(const void* x, const void* gamma, const void* beta, void* z, int64_t M, int64_t N,
+                       int64_t ld_x, int64_t ld_z, int32_t x_dtype, int32_t z_dtype, int32_t param_dtype,
+                       float eps, void* stream);
+
 /* Synchronise `stream` and read the plan's device error word.  Returns
  * FL_ERR_TIMEOUT if a bounded wait inside a kernel of this plan gave up
  * (the error word is then cleared), FL_ERR_CUDA on a CUDA error, else FL_OK. */

@@ -156,3 +156,67 @@ def test_gelu_aux_forward_then_backward(fl, M, N, K, out_dtype):
     assert np.all(err <= P.ULP_REL[out_dtype] * np.abs(dv) + ULP_MIN[out_dtype] + 2 * GELU_GRAD_ABS * np.abs(g64))
     exact = g64 * oracle.gelu_erf_grad(v64)
     _check_dbias(P.to64(dbias), db, np.abs(exact).sum(axis=0), M, np.abs(g64).sum(axis=0), "dgelu after GELU_AUX")
+
+
+# ---------------------------------------------------------------- LayerNorm after the tail
+def _ln_check(got, x64, g64, b64, eps, out_dtype, what):
+    ref = oracle.layer_norm(x64, g64, b64, eps, out_dtype)
+    mu = x64.mean(axis=1, keepdims=True)
+    rstd = 1.0 / np.sqrt(((x64 - mu) ** 2).mean(axis=1, keepdims=True) + eps)
+    # fp32 mean and variance: |Δμ| ≲ 2^-20·max|x| of the row, |Δrstd|/rstd ≲ 2^-20
+    tol = (2.0 ** -20) * np.abs(g64) * rstd * (np.abs(x64).max(axis=1, keepdims=True) + np.abs(x64 - mu)) \
+        + 2 * P.ULP_REL[out_dtype] * np.abs(ref) + ULP_MIN[out_dtype]
+    err = np.abs(got - ref)
+    assert np.all(err <= tol), f"{what}: LayerNorm error {err.max():.3e} (bound there {tol.flat[err.argmax()]:.3e})"
+
+
+@pytest.mark.parametrize("M,N,x_dtype,z_dtype,p_dtype,eps", [
+    (300, 520, "f32", "f32", "f32", 1e-12), (64, 4096, "f32", "bf16", "bf16", 1e-5), (7, 77, "bf16", "bf16", "f32", 1e-5),
+    (33, 20000, "f32", "f32", "f32", 1e-12), (2048, 4096, "f32", "bf16", "f32", 1e-12), (5, 1000, "f16", "f16", "f16", 1e-5)])
+def test_layernorm(fl, M, N, x_dtype, z_dtype, p_dtype, eps):
+    g = torch.Generator().manual_seed(M + N)
+    x = (torch.randn(M, N, generator=g) * 2 + 0.7).to(P.TD[x_dtype])
+    gamma = (torch.rand(N, generator=g) + 0.5).to(P.TD[p_dtype])
+    beta = torch.randn(N, generator=g).to(P.TD[p_dtype])
+    z = P.poison((M, N), z_dtype)
+    fl.fl_layernorm(x.cuda(), gamma.cuda(), beta.cuda(), z, M, N, x_dtype, z_dtype, p_dtype, eps=eps)
+    torch.cuda.synchronize()
+    _ln_check(P.to64(z), P.to64(x), P.to64(gamma)[None, :], P.to64(beta)[None, :], eps, z_dtype,
+              f"LN {M}x{N} {x_dtype}->{z_dtype}")
+
+
+def test_layernorm_in_place_without_affine(fl):
+    M, N = 100, 3000
+    g = torch.Generator().manual_seed(9)
+    x = torch.randn(M, N, generator=g) * 5
+    buf = x.cuda()
+    fl.fl_layernorm(buf, None, None, buf, M, N, "f32", "f32")
+    torch.cuda.synchronize()
+    _ln_check(P.to64(buf), P.to64(x), np.ones((1, N)), np.zeros((1, N)), 1e-12, "f32", "LN in place")
+
+
+def test_bert_tail_then_layernorm(fl):
+    """bias -> GELU -> + residual -> x 0.5 in the fused layer, then LayerNorm of the rows."""
+    w = workloads.get("tail_m512")
+    inp = workloads.make_inputs(w, 0)
+    out = torch.empty(w.M, w.N, dtype=torch.float32, device="cuda")
+    plan = fl.Plan(w.M, w.N, w.K, kind=w.epilogue, out_dtype="f32", bias_dtype=w.bias_dtype, residual_dtype=w.dtype,
+                   has_residual=True, scale=w.scale)
+    try:
+        plan.execute(inp["A"].cuda(), inp["W"].cuda(), inp["bias"].cuda(), None, inp["residual"].cuda(), out)
+        assert plan.check() == fl.FL_OK, fl.fl_last_error()
+    finally:
+        plan.free()
+    gamma = torch.ones(w.N, dtype=torch.float32, device="cuda")
+    beta = torch.zeros(w.N, dtype=torch.float32, device="cuda")
+    z = P.poison((w.M, w.N), "bf16")
+    fl.fl_layernorm(out, gamma, beta, z, w.M, w.N, "f32", "bf16", "f32", eps=1e-12)
+    torch.cuda.synchronize()
+    sel = P.sample_rows(w.M, 64, 2)
+    y, _, _, absdot = P.oracle_linear(A=inp["A"], W=inp["W"], bias=inp["bias"], residual=inp["residual"],
+                                      scale=w.scale, epilogue=w.epilogue, out_dtype="f32", M=w.M, N=w.N, K=w.K,
+                                      rows=sel)
+    # the layer output against the oracle, then LayerNorm of the GPU's own rows
+    P.check_close(P.to64(out)[sel], y, "f32", absdot, "tail_m512 layer")
+    _ln_check(P.to64(z)[sel], P.to64(out)[sel], np.ones((1, w.N)), np.zeros((1, w.N)), 1e-12, "bf16",
+              "tail_m512 LayerNorm")
