@@ -9,7 +9,7 @@ without a B200.
 The entry points keep the C names: ``fl_plan``, ``fl_execute``, ``fl_free``,
 ``fl_relu_backward``, ``fl_check_status``, ``fl_get_plan_info``,
 ``fl_last_error``, ``fl_set_wait_limit_ns``, ``fl_execute_noalloc``, ``fl_bias_grad_workspace_size``,
-``fl_drelu_bgrad``, ``fl_dgelu_bgrad``, ``fl_layernorm``.  ``Plan`` is a small owner of one
+``fl_drelu_bgrad``, ``fl_dgelu_bgrad``, ``fl_layernorm``, ``fl_wait_selftest``.  ``Plan`` is a small owner of one
 plan handle (the cuBLASLt epilog page's Matmul → plan → execute → free).
 """
 from __future__ import annotations
@@ -36,7 +36,7 @@ COMPUTES = {"32F": FL_COMPUTE_32F, "32F_3XTF32": FL_COMPUTE_32F_3XTF32}
 
 EXPORTED = ["fl_plan", "fl_execute", "fl_relu_backward", "fl_check_status", "fl_get_plan_info",
             "fl_free", "fl_last_error", "fl_set_wait_limit_ns", "fl_execute_noalloc",
-            "fl_bias_grad_workspace_size", "fl_drelu_bgrad", "fl_dgelu_bgrad", "fl_layernorm"]
+            "fl_bias_grad_workspace_size", "fl_drelu_bgrad", "fl_dgelu_bgrad", "fl_layernorm", "fl_wait_selftest"]
 
 
 class fl_epilogue_desc(ctypes.Structure):
@@ -89,6 +89,8 @@ def _load() -> ctypes.CDLL:
     lib.fl_dgelu_bgrad.restype = i32
     lib.fl_layernorm.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i32, i32, i32, ctypes.c_float, vp]
     lib.fl_layernorm.restype = i32
+    lib.fl_wait_selftest.argtypes = [ctypes.c_uint64, vp]
+    lib.fl_wait_selftest.restype = i32
     return lib
 
 
@@ -205,6 +207,11 @@ def fl_layernorm(x, gamma, beta, z, M: int, N: int, x_dtype: str, z_dtype: str, 
     _check(LIB.fl_layernorm(_ptr(x), _ptr(gamma), _ptr(beta), _ptr(z), int(M), int(N), int(ld_x), int(ld_z),
                             DTYPES[x_dtype], DTYPES[z_dtype], DTYPES[param_dtype], float(eps), _stream(stream)),
            "fl_layernorm")
+
+
+def fl_wait_selftest(limit_ns: int, stream=None) -> int:
+    """Status of the bounded-wait failure-path self-test (FL_ERR_TIMEOUT when it works)."""
+    return LIB.fl_wait_selftest(int(limit_ns), _stream(stream))
 
 
 def fl_check_status(plan: int, stream=None) -> int:

@@ -1033,6 +1033,31 @@ extern "C" fl_status fl_dgelu_bgrad(const void* grad, const void* v, void* dpre,
                    workspace, workspace_bytes, stream);
 }
 
+// ------------------------------------------------------------------ failure-path self-test
+extern "C" fl_status fl_wait_selftest(uint64_t limit_ns, void* stream_) {
+  g_err[0] = 0;
+  if (limit_ns == 0 || limit_ns > 10000000000ull)
+    return fail(FL_ERR_INVALID_ARG, "fl_wait_selftest: limit must be in (0, 10 s]");
+  int* d_err = nullptr;
+  FL_CUDA(cudaMalloc(&d_err, sizeof(int)));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+  fl_status st = FL_OK;
+  if (cudaMemsetAsync(d_err, 0, sizeof(int), s) != cudaSuccess) st = fail(FL_ERR_CUDA, "fl_wait_selftest: memset");
+  if (!st) {
+    fl_wait_selftest_kernel<<<1, 32, 0, s>>>(d_err, (unsigned long long)limit_ns);
+    st = after_launch(s, "fl_wait_selftest");
+  }
+  int h = 0;
+  if (!st && cudaStreamSynchronize(s) != cudaSuccess) st = fail(FL_ERR_CUDA, "fl_wait_selftest: synchronize");
+  if (!st && cudaMemcpy(&h, d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    st = fail(FL_ERR_CUDA, "fl_wait_selftest: read back");
+  cudaFree(d_err);
+  if (st) return st;
+  // the wait must have given up: the bounded-wait failure path reports a timeout
+  if (h == 0) return fail(FL_ERR_CUDA, "fl_wait_selftest: the wait did not report its timeout");
+  return fail(FL_ERR_TIMEOUT, "fl_wait_selftest: the bounded wait gave up as designed (code %d)", h);
+}
+
 // ------------------------------------------------------------------ LayerNorm after the tail
 template <int XT>
 static cudaError_t launch_ln(int z_dtype, unsigned grid, cudaStream_t s, const LnParams& P) {

@@ -236,6 +236,22 @@ __device__ __forceinline__ float ldg_pinned(const void* base, long long i, int d
   return __half2float(__ushort_as_half(h));
 }
 
+// ------------------------------------------------------------------ failure-path self-test
+// One thread waits, with the same bounded wait as the kernels, on an mbarrier that
+// nothing arrives on: the wait gives up after `limit_ns`, records kErrTimeout in
+// *err and the kernel returns, leaving the context usable.
+__global__ void fl_wait_selftest_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  fence_mbarrier_init();
+  KParams p{};
+  p.err = err;
+  p.wait_limit_ns = limit_ns;
+  (void)wait_bounded(b, 0, p);
+}
+
 // ------------------------------------------------------------------ 3xTF32 split
 // x = hi + lo.  The tensor core reads a 32-bit operand word as TF32 by keeping its
 // top 19 bits (sign, exponent, 10 mantissa bits): the raw stage word therefore

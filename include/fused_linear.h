@@ -172,6 +172,14 @@ fl_status fl_dgelu_bgrad(const void* grad, const void* v, void* dpre, float* dbi
                          int64_t ld_grad, int64_t ld_v, int64_t ld_dpre, int32_t dtype, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/* Failure-path self-test (no counterpart on the pages): one thread of a tiny kernel
+ * waits, with the bounded wait every kernel of this library uses, on an mbarrier that
+ * nothing arrives on.  The wait gives up after limit_ns (0 < limit_ns ≤ 10 s) and the
+ * kernel records the timeout in a device word and returns; no trap, no fault, and the
+ * context stays usable.  Synchronises `stream`.  Returns FL_ERR_TIMEOUT when the failure
+ * path worked as designed, FL_ERR_CUDA otherwise, FL_ERR_INVALID_ARG for a bad limit. */
+fl_status fl_wait_selftest(uint64_t limit_ns, void* stream);
+
 /* LayerNorm of each row, the step after the residual tail ([mhc] §3.2: the row's mean
  * and variance and the normalisation in one kernel, one read and one write):
  *   z[m,n] = (x[m,n] − μ_m)/√(σ²_m + eps)·gamma[n] + beta[n],

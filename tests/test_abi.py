@@ -132,6 +132,32 @@ def test_relu_backward_validation(fl):
     assert fl.LIB.fl_relu_backward(16, 16, 16, 4, 4, 0, 0, 7, None) == fl.FL_ERR_INVALID_ARG
 
 
+def test_backward_and_layernorm_validation(fl):
+    # every argument check runs before the first CUDA call, so it works without a GPU
+    L = fl.LIB
+    INV, ALN = fl.FL_ERR_INVALID_ARG, fl.FL_ERR_ALIGNMENT
+    # fl_drelu_bgrad(grad, aux, dpre, dbias, M, N, ld_grad, ld_dpre, dtype, ws, ws_bytes, stream)
+    assert L.fl_drelu_bgrad(None, 16, 16, None, 4, 4, 0, 0, 1, None, 0, None) == INV
+    assert L.fl_drelu_bgrad(16, 16, 16, None, -1, 4, 0, 0, 1, None, 0, None) == INV
+    assert L.fl_drelu_bgrad(16, 16, 16, None, 4, 8, 4, 0, 1, None, 0, None) == INV   # ld < N
+    assert L.fl_drelu_bgrad(16, 16, 16, None, 4, 4, 0, 0, 9, None, 0, None) == INV   # dtype
+    assert L.fl_drelu_bgrad(16, 18, 16, None, 4, 4, 0, 0, 1, None, 0, None) == ALN   # mask not 4-byte aligned
+    # fl_dgelu_bgrad(grad, v, dpre, dbias, M, N, ld_grad, ld_v, ld_dpre, dtype, ws, ws_bytes, stream)
+    assert L.fl_dgelu_bgrad(16, None, 16, None, 4, 4, 0, 0, 0, 1, None, 0, None) == INV
+    assert L.fl_dgelu_bgrad(16, 17, 16, None, 4, 4, 0, 0, 0, 1, None, 0, None) == ALN
+    assert L.fl_dgelu_bgrad(16, 16, 16, 18, 4, 4, 0, 0, 0, 1, None, 0, None) == ALN  # dbias not 4-byte aligned
+    n = ctypes.c_size_t()
+    assert L.fl_bias_grad_workspace_size(-1, 4, 1, ctypes.byref(n)) == INV
+    assert L.fl_bias_grad_workspace_size(4, 4, 1, None) == INV
+    # fl_layernorm(x, gamma, beta, z, M, N, ld_x, ld_z, x_dtype, z_dtype, param_dtype, eps, stream)
+    assert L.fl_layernorm(None, None, None, 16, 4, 4, 0, 0, 2, 2, 2, 1e-5, None) == INV
+    assert L.fl_layernorm(16, None, None, 16, 4, 4, 0, 0, 2, 2, 2, -1.0, None) == INV   # eps < 0
+    assert L.fl_layernorm(16, None, None, 16, 4, 8, 4, 0, 2, 2, 2, 1e-5, None) == INV   # ld < N
+    assert L.fl_layernorm(18, None, None, 16, 4, 4, 0, 0, 2, 2, 2, 1e-5, None) == ALN   # x not 4-byte aligned
+    assert L.fl_layernorm(16, None, None, 16, 4, 4, 0, 0, 2, 2, 5, 1e-5, None) == INV   # param dtype
+    assert L.fl_wait_selftest(0, None) == INV
+
+
 SOURCES = [os.path.join(ROOT, "gemm_bias_activation_tcgen05_b200", "csrc", f)
            for f in ("fl_api.cu", "fl_gemm.cuh", "fl_ptx.cuh", "fl_elementwise.cuh")]
 

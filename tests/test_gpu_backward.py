@@ -220,3 +220,22 @@ def test_bert_tail_then_layernorm(fl):
     P.check_close(P.to64(out)[sel], y, "f32", absdot, "tail_m512 layer")
     _ln_check(P.to64(z)[sel], P.to64(out)[sel], np.ones((1, w.N)), np.zeros((1, w.N)), 1e-12, "bf16",
               "tail_m512 LayerNorm")
+
+
+def test_bounded_wait_failure_path(fl):
+    """A wait that nothing satisfies gives up after its limit and reports FL_ERR_TIMEOUT;
+    the context stays usable (a layer runs and matches the oracle right after)."""
+    import time
+    t0 = time.perf_counter()
+    assert fl.fl_wait_selftest(20_000_000) == fl.FL_ERR_TIMEOUT, fl.fl_last_error()
+    assert time.perf_counter() - t0 < 5.0
+    got = P.run_linear(fl, M=130, N=200, K=64, dtype="bf16", epilogue="RELU_BIAS", out_dtype="bf16",
+                       **_small_layer_inputs())
+    y, _, _, absdot = P.oracle_linear(epilogue="RELU_BIAS", out_dtype="bf16", M=130, N=200, K=64,
+                                      **{k: v for k, v in _small_layer_inputs().items() if k in ("A", "W", "bias")})
+    P.check_close(got["out"], y, "bf16", absdot, "layer after the self-test")
+
+
+def _small_layer_inputs():
+    inp = workloads.ragged_linear_inputs(130, 200, 64, "bf16", 77, bias_dtype="bf16")
+    return {"A": inp["A"], "W": inp["W"], "bias": inp["bias"]}
