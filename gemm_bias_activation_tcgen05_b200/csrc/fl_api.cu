@@ -1096,6 +1096,9 @@ extern "C" fl_status fl_layernorm(const void* x, const void* gamma, const void* 
   P.ldz = ld_z;
   P.param_dtype = param_dtype;
   P.vec_ok = aligned16(x) && (ld_x * ex) % 16 == 0;
+  P.pvec = (!gamma || aligned16(gamma)) && (!beta || aligned16(beta));
+  // a thread's VE outputs (VE = 16 bytes of x) start on a multiple of their own size
+  P.zvec = aligned16(z) && (ld_z * ez) % 16 == 0 && P.vec_ok;
   P.eps = eps;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
   cudaError_t err = x_dtype == FL_BF16 ? launch_ln<DT_BF16>(z_dtype, (unsigned)M, s, P)

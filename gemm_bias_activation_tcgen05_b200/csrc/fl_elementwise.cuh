@@ -190,8 +190,42 @@ struct LnParams {
   void* z;            // [M, ldz] of ZT (may alias x)
   long long M, N, ldx, ldz;
   int param_dtype, vec_ok;
+  int pvec;  // gamma/beta 16-byte aligned: loaded as vectors
+  int zvec;  // z base and pitch allow vector stores of a thread's VE outputs
   float eps;
 };
+
+// VE consecutive parameters from c0 (16-byte vector loads), or `dflt` for a null pointer
+template <int VE>
+__device__ __forceinline__ void load_params_vec(const void* p, long long c0, int dt, float dflt, float (&o)[VE]) {
+  if (p == nullptr) {
+#pragma unroll
+    for (int i = 0; i < VE; ++i) o[i] = dflt;
+    return;
+  }
+  if (dt == DT_F32) {
+#pragma unroll
+    for (int j = 0; j < VE / 4; ++j) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p) + c0) + j);
+      o[4 * j] = f.x, o[4 * j + 1] = f.y, o[4 * j + 2] = f.z, o[4 * j + 3] = f.w;
+    }
+  } else {
+    // 16-bit parameters: VE = 4 reads 8 bytes, VE = 8 reads 16 bytes
+    uint32_t w[VE / 2];
+    if constexpr (VE == 8) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p) + c0));
+      w[0] = q.x, w[1] = q.y, w[2] = q.z, w[3] = q.w;
+    } else {
+      const uint2 q = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(p) + c0));
+      w[0] = q.x, w[1] = q.y;
+    }
+#pragma unroll
+    for (int i = 0; i < VE; ++i) {
+      const uint16_t h = (uint16_t)(w[i >> 1] >> (16 * (i & 1)));
+      o[i] = (dt == DT_BF16) ? __uint_as_float((uint32_t)h << 16) : __half2float(__ushort_as_half(h));
+    }
+  }
+}
 
 // Sum of one value per thread over the 256 threads, in a fixed order (butterfly in
 // each warp, then the eight warp sums in warp order).
@@ -279,6 +313,27 @@ __global__ void __launch_bounds__(256, 4) fl_layernorm_kernel(const LnParams P) 
   const float var = block_sum256(q, red) / (float)N;
   const float rstd = 1.0f / sqrtf(var + P.eps);
   auto finish = [&](long long c0, const float (&v)[VE]) {
+    if (c0 + VE <= N && P.pvec && P.zvec) {
+      // whole vector: parameters by 16-byte loads, the VE outputs by one or two vector stores
+      float g[VE], b[VE], o[VE];
+      load_params_vec<VE>(P.gamma, c0, P.param_dtype, 1.0f, g);
+      load_params_vec<VE>(P.beta, c0, P.param_dtype, 0.0f, b);
+#pragma unroll
+      for (int i = 0; i < VE; ++i) o[i] = (v[i] - mean) * rstd * g[i] + b[i];
+      char* dst = reinterpret_cast<char*>(P.z) + (m * P.ldz + c0) * (ZT == DT_F32 ? 4 : 2);
+      if constexpr (ZT == DT_F32) {
+#pragma unroll
+        for (int j = 0; j < VE / 4; ++j)
+          reinterpret_cast<float4*>(dst)[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+      } else {
+        uint32_t w[VE / 2];
+#pragma unroll
+        for (int j = 0; j < VE / 2; ++j) w[j] = pack2<ZT>(o[2 * j], o[2 * j + 1]);
+        if constexpr (VE == 8) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        else *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+      }
+      return;
+    }
 #pragma unroll
     for (int i = 0; i < VE; ++i) {
       const long long c = c0 + i;

@@ -195,6 +195,24 @@ def test_layernorm_in_place_without_affine(fl):
     _ln_check(P.to64(buf), P.to64(x), np.ones((1, N)), np.zeros((1, N)), 1e-12, "f32", "LN in place")
 
 
+@pytest.mark.parametrize("ldx_pad,ldz_pad,param_off", [(0, 0, 1), (3, 0, 0), (0, 5, 0), (4, 4, 4)])
+def test_layernorm_pitches_and_parameter_alignment(fl, ldx_pad, ldz_pad, param_off):
+    """Row pitches and parameter offsets that switch between the vector and the element paths."""
+    M, N = 37, 1032
+    g = torch.Generator().manual_seed(ldx_pad * 100 + ldz_pad * 10 + param_off)
+    x = torch.randn(M, N + ldx_pad, generator=g) * 3 - 1
+    gfull = torch.rand(N + param_off, generator=g) + 0.5
+    bfull = torch.randn(N + param_off, generator=g)
+    gamma, beta = gfull.cuda()[param_off:], bfull.cuda()[param_off:]
+    z = P.poison((M, N + ldz_pad), "bf16")
+    fl.fl_layernorm(x.cuda(), gamma, beta, z, M, N, "f32", "bf16", "f32", eps=1e-5, ld_x=N + ldx_pad, ld_z=N + ldz_pad)
+    torch.cuda.synchronize()
+    _ln_check(P.to64(z)[:, :N], P.to64(x)[:, :N], P.to64(gfull[param_off:])[None, :],
+              P.to64(bfull[param_off:])[None, :], 1e-5, "bf16", f"LN pitches {ldx_pad},{ldz_pad},{param_off}")
+    if ldz_pad:
+        assert torch.isnan(z[:, N:]).all(), "LN wrote the pitch pad"
+
+
 def test_bert_tail_then_layernorm(fl):
     """bias -> GELU -> + residual -> x 0.5 in the fused layer, then LayerNorm of the rows."""
     w = workloads.get("tail_m512")
