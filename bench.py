@@ -407,11 +407,11 @@ def time_single_launch(suite, it, stream, sh, reps):
     return sum(a.elapsed_time(b) for a, b in evs) / reps
 
 
-def time_backward(fl, pk, reps=10):
-    """The HBM-bound kernels beside the fused layer: the backward with the fused bias
-    gradient on the relu_aux_4096 shape (4096 x 4096 bf16) and the LayerNorm of the
-    tail_m2048 output, each launch after a 256 MB L2 flush: us, achieved GB/s of the
-    algorithmic bytes, and the fraction of the measured HBM copy bandwidth."""
+def hbm_runs(fl, sh):
+    """The HBM-bound kernels beside the fused layer, on resident synthetic inputs: the
+    backward with and without the fused bias gradient on the relu_aux_4096 shape
+    (4096 x 4096 bf16) and the LayerNorm of the tail_m2048 output.  Returns
+    {name: (launch, algorithmic bytes)}."""
     import torch
     M = N = 4096
     g = torch.Generator(device="cpu").manual_seed(5)
@@ -422,8 +422,6 @@ def time_backward(fl, pk, reps=10):
     dbias = torch.empty(N, dtype=torch.float32, device="cuda")
     nbytes = fl.fl_bias_grad_workspace_size(M, N, "bf16")
     ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
-    flush = L2Flush()
-    sh = torch.cuda.current_stream().cuda_stream
     runs = {
         "drelu_bgrad_4096x4096_bf16": (lambda: fl.fl_drelu_bgrad(grad, mask, dpre, dbias, M, N, "bf16", ws, nbytes,
                                                                  stream=sh),
@@ -446,6 +444,20 @@ def time_backward(fl, pk, reps=10):
     runs["layernorm_2048x4096_f32_to_bf16"] = (
         lambda: fl.fl_layernorm(y, gam, bet, zl, Ml, Nl, "f32", "bf16", "f32", eps=1e-12, stream=sh),
         Ml * Nl * (4 + 2) + 2 * 4 * Nl)
+    return runs
+
+
+HBM_KERNELS = ("drelu_bgrad_4096x4096_bf16", "dgelu_bgrad_4096x4096_bf16", "drelu_4096x4096_bf16",
+               "relu_backward_4096x4096_bf16", "layernorm_2048x4096_f32_to_bf16")
+
+
+def time_backward(fl, pk, reps=10):
+    """Each HBM-bound kernel of hbm_runs() after a 256 MB L2 flush: us, achieved GB/s of
+    the algorithmic bytes, and the fraction of the measured HBM copy bandwidth."""
+    import torch
+    sh = torch.cuda.current_stream().cuda_stream
+    runs = hbm_runs(fl, sh)
+    flush = L2Flush()
     out = {}
     for name, (fn, algo_bytes) in runs.items():
         fn()
@@ -667,10 +679,17 @@ def run_reference(args):
 
 
 def run_profile(args):
-    """Launch one workload warm-up + steps times and exit: a small, fixed program for ncu."""
+    """Launch one workload (or one HBM-bound kernel of hbm_runs) warm-up + steps times and
+    exit: a small, fixed program for ncu."""
     import torch
     import gemm_bias_activation_tcgen05_b200 as fl
     torch.cuda.set_device(0)
+    if args.profile in HBM_KERNELS:
+        fn, _ = hbm_runs(fl, torch.cuda.current_stream().cuda_stream)[args.profile]
+        for _ in range(args.warmup + args.steps):
+            fn()
+        torch.cuda.synchronize()
+        return
     global SUITE
     SUITE = [args.profile]
     suite = Suite(fl, seed=0)

@@ -562,10 +562,10 @@ struct GemmArgs {
 
 // Launch an elementwise kernel with programmatic dependent launch allowed.
 template <typename... KArgs, typename... Args>
-static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, cudaStream_t s, Args... args) {
+static cudaError_t launch_pdl_b(void (*kern)(KArgs...), dim3 grid, unsigned block, cudaStream_t s, Args... args) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(256, 1, 1);
+  cfg.blockDim = dim3(block, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -574,6 +574,11 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, cudaStream_t s,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, cudaStream_t s, Args... args) {
+  return launch_pdl_b(kern, grid, 256u, s, args...);
 }
 
 static fl_status launch_kernel(const fl_plan_s* p, const LaunchCache& c, cudaStream_t stream,
@@ -734,6 +739,22 @@ static int grid_for(long long work, int num_sms) {
   if (b > cap) b = cap;
   if (b < 1) b = 1;
   return (int)b;
+}
+
+// One wave of resident 256-thread CTAs for a grid-stride kernel whose warps take `units`
+// work units in turn.  A grid larger than one wave leaves a partial second wave of CTAs; a
+// grid of exactly one wave can leave some warps a unit more than the rest.  So: the fewest
+// rounds of units one wave needs, then the fewest warps that finish in that many rounds.
+static int resident_grid(const void* kernel, long long units, int num_sms) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess || per_sm < 1) {
+    (void)cudaGetLastError();
+    per_sm = 1;
+  }
+  const long long slots = (long long)num_sms * per_sm * 8;
+  const long long rounds = std::max<long long>(1, (units + slots - 1) / slots);
+  const long long warps = (units + rounds - 1) / rounds;
+  return (int)std::max<long long>(1, (warps + 7) / 8);
 }
 
 template <int DT>
@@ -902,8 +923,11 @@ extern "C" fl_status fl_relu_backward(const void* grad, const uint32_t* aux, voi
   FL_CUDA(cudaGetDevice(&dev));
   FL_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   const long long words = cdiv(N, 32);
-  const long long work = M * words;
-  const int grid = grid_for(work, sms);
+  const long long units = M * cdiv(words, 32);  // a warp takes 32 mask words of a row per round
+  const void* kern = dtype == FL_BF16 ? (const void*)fl_relu_backward_kernel<DT_BF16>
+                   : dtype == FL_F16  ? (const void*)fl_relu_backward_kernel<DT_F16>
+                                      : (const void*)fl_relu_backward_kernel<DT_F32>;
+  const int grid = resident_grid(kern, units, sms);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
   cudaError_t err;
   if (dtype == FL_BF16)
@@ -1059,11 +1083,36 @@ extern "C" fl_status fl_wait_selftest(uint64_t limit_ns, void* stream_) {
 }
 
 // ------------------------------------------------------------------ LayerNorm after the tail
+template <int XT, int ZT, int TPB>
+static void (*ln_kernel(bool vec))(LnParams) {
+  return vec ? fl_layernorm_vec_kernel<XT, ZT, TPB> : fl_layernorm_kernel<XT, ZT, TPB>;
+}
+
+// 128 threads per row when the row fits their registers (32 elements a thread).  The
+// kernel loops over rows: the grid is one resident wave, or M CTAs if fewer.
+template <int XT, int TPB>
+static cudaError_t launch_ln_w(int z_dtype, cudaStream_t s, const LnParams& P) {
+  int dev = 0, sms = 148, per_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  // whole-vector layout: every access of the row, the parameters and z is a 16-byte vector
+  constexpr long long ve = 16 / (XT == DT_F32 ? 4 : 2);
+  constexpr long long vmax = TPB == 128 ? 32 / ve : 4;
+  const bool vec = P.vec_ok && P.pvec && P.zvec && P.N % ve == 0 && P.N <= TPB * vmax * ve;
+  void (*k)(LnParams) = z_dtype == FL_BF16 ? ln_kernel<XT, DT_BF16, TPB>(vec)
+                      : z_dtype == FL_F16  ? ln_kernel<XT, DT_F16, TPB>(vec)
+                                           : ln_kernel<XT, DT_F32, TPB>(vec);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, (const void*)k, TPB, 0);
+  if (e != cudaSuccess) return e;
+  const long long wave = (long long)std::max(1, per_sm) * sms;
+  return launch_pdl_b(k, dim3((unsigned)std::min<long long>(P.M, wave)), TPB, s, P);
+}
+
 template <int XT>
-static cudaError_t launch_ln(int z_dtype, unsigned grid, cudaStream_t s, const LnParams& P) {
-  if (z_dtype == FL_BF16) return launch_pdl(fl_layernorm_kernel<XT, DT_BF16>, dim3(grid), s, P);
-  if (z_dtype == FL_F16) return launch_pdl(fl_layernorm_kernel<XT, DT_F16>, dim3(grid), s, P);
-  return launch_pdl(fl_layernorm_kernel<XT, DT_F32>, dim3(grid), s, P);
+static cudaError_t launch_ln(int z_dtype, cudaStream_t s, const LnParams& P) {
+  if (P.N <= 128 * 32) return launch_ln_w<XT, 128>(z_dtype, s, P);
+  return launch_ln_w<XT, 256>(z_dtype, s, P);
 }
 
 extern "C" fl_status fl_layernorm(const void* x, const void* gamma, const void* beta, void* z, int64_t M, int64_t N,
@@ -1101,9 +1150,9 @@ extern "C" fl_status fl_layernorm(const void* x, const void* gamma, const void* 
   P.zvec = aligned16(z) && (ld_z * ez) % 16 == 0 && P.vec_ok;
   P.eps = eps;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
-  cudaError_t err = x_dtype == FL_BF16 ? launch_ln<DT_BF16>(z_dtype, (unsigned)M, s, P)
-                    : x_dtype == FL_F16 ? launch_ln<DT_F16>(z_dtype, (unsigned)M, s, P)
-                                        : launch_ln<DT_F32>(z_dtype, (unsigned)M, s, P);
+  cudaError_t err = x_dtype == FL_BF16 ? launch_ln<DT_BF16>(z_dtype, s, P)
+                    : x_dtype == FL_F16 ? launch_ln<DT_F16>(z_dtype, s, P)
+                                        : launch_ln<DT_F32>(z_dtype, s, P);
   if (err != cudaSuccess) return fail(FL_ERR_CUDA, "%s: kernel launch: %s", who, cudaGetErrorString(err));
   return after_launch(s, who);
 }

@@ -227,9 +227,10 @@ __device__ __forceinline__ void load_params_vec(const void* p, long long c0, int
   }
 }
 
-// Sum of one value per thread over the 256 threads, in a fixed order (butterfly in
-// each warp, then the eight warp sums in warp order).
-__device__ __forceinline__ float block_sum256(float v, float* red) {
+// Sum of one value per thread over the NW warps of the CTA, in a fixed order (butterfly
+// in each warp, then the warp sums in warp order).
+template <int NW>
+__device__ __forceinline__ float block_sum(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -238,89 +239,243 @@ __device__ __forceinline__ float block_sum256(float v, float* red) {
   __syncthreads();
   float s = red[0];
 #pragma unroll
-  for (int w = 1; w < 8; ++w) s += red[w];
+  for (int w = 1; w < NW; ++w) s += red[w];
   return s;
 }
 
 // z = (x − μ)·rstd·γ + β over each row (mHC page §3.2: the mean and variance of the
 // row, then the normalisation, in one kernel: one read and one write of the row).
-// One CTA of 256 threads per row.  A row of up to 256·4 16-byte vectors stays in
-// registers across the three steps (mean, Σ(x − μ)², normalise); a longer row is
-// read again for the later steps.
-template <int XT, int ZT>
-__global__ void __launch_bounds__(256, 4) fl_layernorm_kernel(const LnParams P) {
+// A CTA of TPB threads normalises rows blockIdx.x, blockIdx.x + gridDim.x, ... (one
+// resident wave).  A row of up to TPB·VMAX 16-byte vectors stays in registers across
+// the three steps (mean, Σ(x − μ)², normalise).  When rows are 16-byte aligned, each
+// thread copies its vectors of the CTA's NEXT row into shared memory (cp.async) as
+// soon as it has taken the current row into registers, so that row's read runs while
+// this one is reduced and stored; each thread reads back only the slots it copied.
+// A longer row is read again for the later steps.  Rows of up to 4096 elements take
+// 128-thread CTAs keeping 32 elements a thread; longer rows take 256 threads.
+template <int XT, int ZT, int TPB>
+__global__ void __launch_bounds__(TPB, TPB == 128 ? 6 : 3) fl_layernorm_kernel(const LnParams P) {
   using TX = typename ElemT<XT>::T;
   grid_dependency_wait();
   if (threadIdx.x == 0) grid_launch_dependents();
-  constexpr int VE = 16 / sizeof(TX);  // elements per 16-byte vector of x
-  constexpr int VMAX = 4;              // vectors a thread keeps in registers
-  __shared__ float red[8];
-  const long long m = blockIdx.x;
-  const TX* x = reinterpret_cast<const TX*>(P.x) + m * P.ldx;
+  constexpr int VE = 16 / sizeof(TX);             // elements per 16-byte vector of x
+  constexpr int VMAX = TPB == 128 ? 32 / VE : 4;  // vectors a thread keeps in registers
+  constexpr int NW = TPB / 32;
+  __shared__ float red[NW];
+  __shared__ __align__(16) uint4 stage[VMAX * TPB];  // the next row, slot k·TPB + t for thread t
   const long long N = P.N;
   const int t = threadIdx.x;
-  const bool in_regs = N <= 256LL * VMAX * VE;
-  auto load_vec = [&](long long c0, float (&v)[VE]) {
-    if (P.vec_ok && c0 + VE <= N) {
-      const uint4 q = __ldg(reinterpret_cast<const uint4*>(x + c0));
-      const TX* e = reinterpret_cast<const TX*>(&q);
-#pragma unroll
-      for (int i = 0; i < VE; ++i) v[i] = static_cast<float>(e[i]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < VE; ++i) v[i] = (c0 + i < N) ? static_cast<float>(x[c0 + i]) : 0.0f;
-    }
-  };
-  float xv[VMAX][VE];
-  float s = 0.0f;
-  if (in_regs) {
+  const bool in_regs = N <= (long long)TPB * VMAX * VE;
+  const bool pipelined = in_regs && P.vec_ok;
+  const uint32_t stage_base = (uint32_t)__cvta_generic_to_shared(stage);
+  auto row_ptr = [&](long long m) { return reinterpret_cast<const TX*>(P.x) + m * P.ldx; };
+  // copy this thread's whole vectors of row m into its stage slots
+  auto prefetch = [&](long long m) {
+    const TX* x = row_ptr(m);
 #pragma unroll
     for (int k = 0; k < VMAX; ++k) {
-      const long long c0 = ((long long)k * 256 + t) * VE;
+      const long long c0 = ((long long)k * TPB + t) * VE;
+      if (c0 + VE <= N) cp_async_16(stage_base + (uint32_t)(k * TPB + t) * 16u, x + c0, 16u);
+    }
+    cp_async_commit();
+  };
+  if (pipelined && blockIdx.x < P.M) prefetch(blockIdx.x);
+  for (long long m = blockIdx.x; m < P.M; m += gridDim.x) {
+    const TX* x = row_ptr(m);
+    auto load_vec = [&](long long c0, float (&v)[VE]) {
+      if (P.vec_ok && c0 + VE <= N) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(x + c0));
+        const TX* e = reinterpret_cast<const TX*>(&q);
 #pragma unroll
-      for (int i = 0; i < VE; ++i) xv[k][i] = 0.0f;
-      if (c0 < N) load_vec(c0, xv[k]);
+        for (int i = 0; i < VE; ++i) v[i] = static_cast<float>(e[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < VE; ++i) v[i] = (c0 + i < N) ? static_cast<float>(x[c0 + i]) : 0.0f;
+      }
+    };
+    float xv[VMAX][VE];
+    float s = 0.0f;
+    if (pipelined) {
+      cp_async_wait<0>();  // this thread's copies of row m have landed
+#pragma unroll
+      for (int k = 0; k < VMAX; ++k) {
+        const long long c0 = ((long long)k * TPB + t) * VE;
+#pragma unroll
+        for (int i = 0; i < VE; ++i) xv[k][i] = 0.0f;
+        if (c0 + VE <= N) {
+          const uint4 q = *reinterpret_cast<const uint4*>(&stage[k * TPB + t]);
+          const TX* e = reinterpret_cast<const TX*>(&q);
+#pragma unroll
+          for (int i = 0; i < VE; ++i) xv[k][i] = static_cast<float>(e[i]);
+        } else if (c0 < N) {
+          load_vec(c0, xv[k]);  // the row's partial last vector
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < VMAX; ++k)
+#pragma unroll
+        for (int i = 0; i < VE; ++i) s += xv[k][i];
+      // the slots are free once their values have been used (the sum above)
+      if (m + gridDim.x < P.M) prefetch(m + gridDim.x);
+    } else if (in_regs) {
+      // every load of the row is issued before the first use, so their latencies overlap
+#pragma unroll
+      for (int k = 0; k < VMAX; ++k) {
+        const long long c0 = ((long long)k * TPB + t) * VE;
+#pragma unroll
+        for (int i = 0; i < VE; ++i) xv[k][i] = 0.0f;
+        if (c0 < N) load_vec(c0, xv[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < VMAX; ++k)
+#pragma unroll
+        for (int i = 0; i < VE; ++i) s += xv[k][i];
+    } else {
+      for (long long c0 = (long long)t * VE; c0 < N; c0 += (long long)TPB * VE) {
+        float v[VE];
+        load_vec(c0, v);
+#pragma unroll
+        for (int i = 0; i < VE; ++i) s += v[i];
+      }
+    }
+    const float mean = block_sum<NW>(s, red) / (float)N;
+    float q = 0.0f;
+    if (in_regs) {
+#pragma unroll
+      for (int k = 0; k < VMAX; ++k) {
+        const long long c0 = ((long long)k * TPB + t) * VE;
+#pragma unroll
+        for (int i = 0; i < VE; ++i)
+          if (c0 + i < N) q += (xv[k][i] - mean) * (xv[k][i] - mean);
+      }
+    } else {
+      for (long long c0 = (long long)t * VE; c0 < N; c0 += (long long)TPB * VE) {
+        float v[VE];
+        load_vec(c0, v);
+#pragma unroll
+        for (int i = 0; i < VE; ++i)
+          if (c0 + i < N) q += (v[i] - mean) * (v[i] - mean);
+      }
+    }
+    const float var = block_sum<NW>(q, red) / (float)N;
+    const float rstd = 1.0f / sqrtf(var + P.eps);
+    auto finish = [&](long long c0, const float (&v)[VE]) {
+      if (c0 + VE <= N && P.pvec && P.zvec) {
+        // whole vector: parameters by 16-byte loads, the VE outputs by one or two vector stores
+        float g[VE], b[VE], o[VE];
+        load_params_vec<VE>(P.gamma, c0, P.param_dtype, 1.0f, g);
+        load_params_vec<VE>(P.beta, c0, P.param_dtype, 0.0f, b);
+#pragma unroll
+        for (int i = 0; i < VE; ++i) o[i] = (v[i] - mean) * rstd * g[i] + b[i];
+        char* dst = reinterpret_cast<char*>(P.z) + (m * P.ldz + c0) * (ZT == DT_F32 ? 4 : 2);
+        if constexpr (ZT == DT_F32) {
+#pragma unroll
+          for (int j = 0; j < VE / 4; ++j)
+            reinterpret_cast<float4*>(dst)[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+        } else {
+          uint32_t w[VE / 2];
+#pragma unroll
+          for (int j = 0; j < VE / 2; ++j) w[j] = pack2<ZT>(o[2 * j], o[2 * j + 1]);
+          if constexpr (VE == 8) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+          else *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+        }
+        return;
+      }
+#pragma unroll
+      for (int i = 0; i < VE; ++i) {
+        const long long c = c0 + i;
+        if (c < N) {
+          const float g = P.gamma ? load_elem(P.gamma, c, P.param_dtype) : 1.0f;
+          const float b = P.beta ? load_elem(P.beta, c, P.param_dtype) : 0.0f;
+          store_elem<ZT>(P.z, m * P.ldz + c, (v[i] - mean) * rstd * g + b);
+        }
+      }
+    };
+    if (in_regs) {
+#pragma unroll
+      for (int k = 0; k < VMAX; ++k) {
+        const long long c0 = ((long long)k * TPB + t) * VE;
+        if (c0 < N) finish(c0, xv[k]);
+      }
+    } else {
+      for (long long c0 = (long long)t * VE; c0 < N; c0 += (long long)TPB * VE) {
+        float v[VE];
+        load_vec(c0, v);
+        finish(c0, v);
+      }
+    }
+  }
+  cp_async_wait<0>();  // no copy of this CTA is still in flight when it exits
+}
+
+// The same normalisation for the common layout: x, z and the parameters 16-byte aligned
+// with 16-byte row pitches, N a multiple of the vector width and at most TPB·VMAX
+// vectors.  Column offsets are 32-bit, the validity of each of a thread's vectors is
+// fixed for the whole launch, and every access is a whole vector, which keeps the
+// instruction count per element small.  Rows are prefetched as in fl_layernorm_kernel.
+template <int XT, int ZT, int TPB>
+__global__ void __launch_bounds__(TPB, TPB == 128 ? 6 : 3) fl_layernorm_vec_kernel(const LnParams P) {
+  using TX = typename ElemT<XT>::T;
+  grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
+  constexpr int VE = 16 / sizeof(TX);
+  constexpr int VMAX = TPB == 128 ? 32 / VE : 4;
+  constexpr int NW = TPB / 32;
+  constexpr int EZ = (ZT == DT_F32) ? 4 : 2;
+  __shared__ float red[NW];
+  __shared__ __align__(16) uint4 stage[VMAX * TPB];
+  const int t = threadIdx.x;
+  const int nvec = (int)(P.N / VE);
+  const float inv_n = 1.0f / (float)P.N;
+  const uint32_t stage_base = (uint32_t)__cvta_generic_to_shared(stage);
+  auto prefetch = [&](long long m) {
+    const uint4* x = reinterpret_cast<const uint4*>(reinterpret_cast<const TX*>(P.x) + m * P.ldx);
+#pragma unroll
+    for (int k = 0; k < VMAX; ++k)
+      if (k * TPB + t < nvec) cp_async_16(stage_base + (uint32_t)(k * TPB + t) * 16u, x + k * TPB + t, 16u);
+    cp_async_commit();
+  };
+  if (blockIdx.x < P.M) prefetch(blockIdx.x);
+  for (long long m = blockIdx.x; m < P.M; m += gridDim.x) {
+    float xv[VMAX][VE];
+    cp_async_wait<0>();
+    float s = 0.0f;
+#pragma unroll
+    for (int k = 0; k < VMAX; ++k) {
+      if (k * TPB + t < nvec) {
+        const uint4 q = stage[k * TPB + t];
+        const TX* e = reinterpret_cast<const TX*>(&q);
+#pragma unroll
+        for (int i = 0; i < VE; ++i) xv[k][i] = static_cast<float>(e[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < VE; ++i) xv[k][i] = 0.0f;
+      }
 #pragma unroll
       for (int i = 0; i < VE; ++i) s += xv[k][i];
     }
-  } else {
-    for (long long c0 = (long long)t * VE; c0 < N; c0 += 256LL * VE) {
-      float v[VE];
-      load_vec(c0, v);
-#pragma unroll
-      for (int i = 0; i < VE; ++i) s += v[i];
-    }
-  }
-  const float mean = block_sum256(s, red) / (float)N;
-  float q = 0.0f;
-  if (in_regs) {
+    if (m + gridDim.x < P.M) prefetch(m + gridDim.x);  // the slots' values are used above
+    const float mean = block_sum<NW>(s, red) * inv_n;
+    float q = 0.0f;
 #pragma unroll
     for (int k = 0; k < VMAX; ++k) {
-      const long long c0 = ((long long)k * 256 + t) * VE;
+      if (k * TPB + t < nvec) {
 #pragma unroll
-      for (int i = 0; i < VE; ++i)
-        if (c0 + i < N) q += (xv[k][i] - mean) * (xv[k][i] - mean);
+        for (int i = 0; i < VE; ++i) q += (xv[k][i] - mean) * (xv[k][i] - mean);
+      }
     }
-  } else {
-    for (long long c0 = (long long)t * VE; c0 < N; c0 += 256LL * VE) {
-      float v[VE];
-      load_vec(c0, v);
+    const float rstd = 1.0f / sqrtf(block_sum<NW>(q, red) * inv_n + P.eps);
+    char* zrow = reinterpret_cast<char*>(P.z) + m * P.ldz * EZ;
 #pragma unroll
-      for (int i = 0; i < VE; ++i)
-        if (c0 + i < N) q += (v[i] - mean) * (v[i] - mean);
-    }
-  }
-  const float var = block_sum256(q, red) / (float)N;
-  const float rstd = 1.0f / sqrtf(var + P.eps);
-  auto finish = [&](long long c0, const float (&v)[VE]) {
-    if (c0 + VE <= N && P.pvec && P.zvec) {
-      // whole vector: parameters by 16-byte loads, the VE outputs by one or two vector stores
+    for (int k = 0; k < VMAX; ++k) {
+      const int v = k * TPB + t;
+      if (v >= nvec) continue;
       float g[VE], b[VE], o[VE];
-      load_params_vec<VE>(P.gamma, c0, P.param_dtype, 1.0f, g);
-      load_params_vec<VE>(P.beta, c0, P.param_dtype, 0.0f, b);
+      load_params_vec<VE>(P.gamma, (long long)v * VE, P.param_dtype, 1.0f, g);
+      load_params_vec<VE>(P.beta, (long long)v * VE, P.param_dtype, 0.0f, b);
 #pragma unroll
-      for (int i = 0; i < VE; ++i) o[i] = (v[i] - mean) * rstd * g[i] + b[i];
-      char* dst = reinterpret_cast<char*>(P.z) + (m * P.ldz + c0) * (ZT == DT_F32 ? 4 : 2);
+      for (int i = 0; i < VE; ++i) o[i] = (xv[k][i] - mean) * rstd * g[i] + b[i];
+      char* dst = zrow + (size_t)v * VE * EZ;
       if constexpr (ZT == DT_F32) {
 #pragma unroll
         for (int j = 0; j < VE / 4; ++j)
@@ -332,36 +487,14 @@ __global__ void __launch_bounds__(256, 4) fl_layernorm_kernel(const LnParams P) 
         if constexpr (VE == 8) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
         else *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
       }
-      return;
-    }
-#pragma unroll
-    for (int i = 0; i < VE; ++i) {
-      const long long c = c0 + i;
-      if (c < N) {
-        const float g = P.gamma ? load_elem(P.gamma, c, P.param_dtype) : 1.0f;
-        const float b = P.beta ? load_elem(P.beta, c, P.param_dtype) : 0.0f;
-        store_elem<ZT>(P.z, m * P.ldz + c, (v[i] - mean) * rstd * g + b);
-      }
-    }
-  };
-  if (in_regs) {
-#pragma unroll
-    for (int k = 0; k < VMAX; ++k) {
-      const long long c0 = ((long long)k * 256 + t) * VE;
-      if (c0 < N) finish(c0, xv[k]);
-    }
-  } else {
-    for (long long c0 = (long long)t * VE; c0 < N; c0 += 256LL * VE) {
-      float v[VE];
-      load_vec(c0, v);
-      finish(c0, v);
     }
   }
+  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------- dReLU
 template <int DT>
-__global__ void __launch_bounds__(256) fl_relu_backward_kernel(const void* __restrict__ grad_,
+__global__ void __launch_bounds__(256, 4) fl_relu_backward_kernel(const void* __restrict__ grad_,
                                                                const uint32_t* __restrict__ aux,
                                                                void* __restrict__ dpre_, long long M,
                                                                long long N, long long ldg,
@@ -371,64 +504,90 @@ __global__ void __launch_bounds__(256) fl_relu_backward_kernel(const void* __res
   grid_dependency_wait();
   if (threadIdx.x == 0) grid_launch_dependents();
   constexpr int ESZ = sizeof(T);
-  constexpr int PER16 = 16 / ESZ;  // elements per 16-byte vector
+  constexpr int PER16 = 16 / ESZ;             // elements per 16-byte vector
+  constexpr int V = 32 * 32 / PER16 / 32;     // vectors per lane in a block of 32 words
+  constexpr int U = (ESZ == 2) ? 2 : 1;       // blocks a trip (16-bit: 8 vectors a lane in flight)
   const T* grad = reinterpret_cast<const T*>(grad_);
   T* dpre = reinterpret_cast<T*>(dpre_);
   const int lane = threadIdx.x & 31;
-  // A warp takes a block of 32 mask words (32·32 elements) of one row.  In a full
-  // block lane l moves 16-byte vectors l, l+32, ... of the block, so every warp-wide
-  // access is 512 contiguous bytes, and reads its mask bits from the block's 32 words
-  // (one coalesced load) by shuffle.
+  // A warp takes blocks of 32 mask words (32·32 elements) of one row, U blocks a trip.
+  // In a full block lane l moves 16-byte vectors l, l+32, ... of the block, so every
+  // warp-wide access is 512 contiguous bytes, and reads its mask bits from the block's
+  // 32 words (one coalesced load) by shuffle.  Every load of a trip (mask words and
+  // gradient vectors) is issued before the first use.
   const long long wblocks = (words + 31) / 32;
   const long long total = M * wblocks;
   const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-  for (long long blk = warp0; blk < total; blk += nwarps) {
-    const long long m = blk / wblocks;
-    const long long w0 = (blk - m * wblocks) * 32;
-    const T* g = grad + m * ldg + w0 * 32;
-    T* d = dpre + m * ldd + w0 * 32;
-    const uint32_t myword = (w0 + lane < words) ? __ldg(aux + m * words + w0 + lane) : 0u;
-    if (vec_ok && w0 + 32 <= words && (w0 + 32) * 32 <= N) {
+  for (long long blk0 = warp0; blk0 < total; blk0 += U * nwarps) {
+    uint32_t myword[U];
+    uint4 x[U][V];
+    bool full[U];
+    long long base_g[U], base_d[U];
 #pragma unroll
-      for (int v = 0; v < 32 * 32 / PER16 / 32; ++v) {
-        const int e0 = (v * 32 + lane) * PER16;  // first element of this lane's vector
-        const uint32_t bits = __shfl_sync(0xffffffffu, myword, e0 >> 5);
-        uint4 x = __ldg(reinterpret_cast<const uint4*>(g) + v * 32 + lane);
-        uint32_t* xw = reinterpret_cast<uint32_t*>(&x);
+    for (int j = 0; j < U; ++j) {
+      const long long blk = blk0 + j * nwarps;
+      full[j] = false;
+      myword[j] = 0u;
+      base_g[j] = base_d[j] = 0;
+      if (blk >= total) continue;
+      const long long m = blk / wblocks;
+      const long long w0 = (blk - m * wblocks) * 32;
+      base_g[j] = m * ldg + w0 * 32;
+      base_d[j] = m * ldd + w0 * 32;
+      if (w0 + lane < words) myword[j] = __ldg(aux + m * words + w0 + lane);
+      full[j] = vec_ok && w0 + 32 <= words && (w0 + 32) * 32 <= N;
+      if (full[j]) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if constexpr (ESZ == 2) {
-            const int j = (e0 & 31) + e * 2;
-            // grad·0 keeps the sign of grad (IEEE): clear all but the sign bit
-            const uint32_t lo_keep = ((bits >> j) & 1u) ? 0x0000FFFFu : 0x00008000u;
-            const uint32_t hi_keep = ((bits >> (j + 1)) & 1u) ? 0xFFFF0000u : 0x80000000u;
-            xw[e] &= (lo_keep | hi_keep);
-          } else {
-            const int j = (e0 & 31) + e;
-            xw[e] &= ((bits >> j) & 1u) ? 0xFFFFFFFFu : 0x80000000u;
-          }
-        }
-        reinterpret_cast<uint4*>(d)[v * 32 + lane] = x;
+        for (int v = 0; v < V; ++v) x[j][v] = __ldg(reinterpret_cast<const uint4*>(grad + base_g[j]) + v * 32 + lane);
       }
-    } else {
-      // ragged block: lane l finishes word w0 + l element by element
-      const long long w = w0 + lane;
-      if (w < words) {
-        const long long n0 = w * 32;
-        for (int j = 0; j < 32 && n0 + j < N; ++j) {
-          T x = g[lane * 32 + j];
-          if (!((myword >> j) & 1u)) {
+    }
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const long long blk = blk0 + j * nwarps;
+      if (blk >= total) continue;
+      const T* g = grad + base_g[j];
+      T* d = dpre + base_d[j];
+      if (full[j]) {
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+          const int e0 = (v * 32 + lane) * PER16;  // first element of this lane's vector
+          const uint32_t bits = __shfl_sync(0xffffffffu, myword[j], e0 >> 5);
+          uint32_t* xw = reinterpret_cast<uint32_t*>(&x[j][v]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
             if constexpr (ESZ == 2) {
-              unsigned short b = *reinterpret_cast<unsigned short*>(&x);
-              b &= 0x8000u;
-              x = *reinterpret_cast<T*>(&b);
+              const int b = (e0 & 31) + e * 2;
+              // grad·0 keeps the sign of grad (IEEE): clear all but the sign bit
+              const uint32_t lo_keep = ((bits >> b) & 1u) ? 0x0000FFFFu : 0x00008000u;
+              const uint32_t hi_keep = ((bits >> (b + 1)) & 1u) ? 0xFFFF0000u : 0x80000000u;
+              xw[e] &= (lo_keep | hi_keep);
             } else {
-              uint32_t b = __float_as_uint(x) & 0x80000000u;
-              x = __uint_as_float(b);
+              const int b = (e0 & 31) + e;
+              xw[e] &= ((bits >> b) & 1u) ? 0xFFFFFFFFu : 0x80000000u;
             }
           }
-          d[lane * 32 + j] = x;
+          reinterpret_cast<uint4*>(d)[v * 32 + lane] = x[j][v];
+        }
+      } else {
+        // ragged block: lane l finishes word w0 + l element by element
+        const long long w = (blk - (blk / wblocks) * wblocks) * 32 + lane;
+        if (w < words) {
+          const long long n0 = w * 32;
+          for (int b = 0; b < 32 && n0 + b < N; ++b) {
+            T xe = g[lane * 32 + b];
+            if (!((myword[j] >> b) & 1u)) {
+              if constexpr (ESZ == 2) {
+                unsigned short h = *reinterpret_cast<unsigned short*>(&xe);
+                h &= 0x8000u;
+                xe = *reinterpret_cast<T*>(&h);
+              } else {
+                uint32_t h = __float_as_uint(xe) & 0x80000000u;
+                xe = __uint_as_float(h);
+              }
+            }
+            d[lane * 32 + b] = xe;
+          }
         }
       }
     }

@@ -172,7 +172,11 @@ def _ln_check(got, x64, g64, b64, eps, out_dtype, what):
 
 @pytest.mark.parametrize("M,N,x_dtype,z_dtype,p_dtype,eps", [
     (300, 520, "f32", "f32", "f32", 1e-12), (64, 4096, "f32", "bf16", "bf16", 1e-5), (7, 77, "bf16", "bf16", "f32", 1e-5),
-    (33, 20000, "f32", "f32", "f32", 1e-12), (2048, 4096, "f32", "bf16", "f32", 1e-12), (5, 1000, "f16", "f16", "f16", 1e-5)])
+    (33, 20000, "f32", "f32", "f32", 1e-12), (2048, 4096, "f32", "bf16", "f32", 1e-12), (5, 1000, "f16", "f16", "f16", 1e-5),
+    (16, 6000, "bf16", "f32", "bf16", 1e-5), (9, 5000, "f32", "f16", "f32", 1e-5), (3, 4097, "f32", "f32", "f32", 1e-5),
+    # more rows than one resident wave: CTAs loop over rows (prefetching the next when aligned)
+    (3000, 1032, "bf16", "f16", "f32", 1e-5), (4000, 300, "bf16", "bf16", "bf16", 1e-5),
+    (1200, 4100, "f32", "f32", "f32", 1e-5), (2000, 6000, "bf16", "bf16", "f32", 1e-5)])
 def test_layernorm(fl, M, N, x_dtype, z_dtype, p_dtype, eps):
     g = torch.Generator().manual_seed(M + N)
     x = (torch.randn(M, N, generator=g) * 2 + 0.7).to(P.TD[x_dtype])
