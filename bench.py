@@ -43,7 +43,7 @@ DOMINANT = "relu_aux_4096"   # the largest single fused launch of the step
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -87,24 +87,40 @@ def barrier(ws):
 
 
 def max_over_ranks(x, ws):
+    """The largest of the ranks' values (each rank's device time): the job ends with its
+    slowest replica.  A one-element all-reduce, on the GPU under NCCL, on the host under gloo."""
     if ws == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
+def job_tflops(ws, flops_per_step, steps, total_ms):
+    """Whole-job throughput of N replicas (weak scaling): every rank runs `steps` steps of
+    `flops_per_step`, and the job takes the slowest rank's `total_ms`."""
+    return ws * flops_per_step * steps / (total_ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples every 200 ms while the context is open; summary() keeps the
+    samples taken after mark() (the warm pass and the timed region, both under load)."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index):
         self.idx = gpu_index
         self.proc = None
+        self.t_mark = None
+
+    def mark(self):
+        import datetime
+        self.t_mark = datetime.datetime.now()
 
     def __enter__(self):
         try:
@@ -128,25 +144,32 @@ class ClockSampler:
             self.lines = [l for l in out.splitlines() if l.strip()]
 
     def summary(self):
+        import datetime
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for l in getattr(self, "lines", []):
             f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
+            if self.t_mark is not None:
+                try:
+                    ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f")
+                    if ts < self.t_mark - datetime.timedelta(milliseconds=50):
+                        continue  # taken while the GPU idled before the warm pass
+                except ValueError:
+                    pass
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                sm.append(float(f[2]))
+                mx = float(f[3])
             except ValueError:
                 continue
-            for name, val in zip(names, f[5:9]):
+            for name, val in zip(names, f[6:10]):
                 if val.lower().startswith("active"):
                     reasons.add(name)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
-        loaded = [s for s in sm if mx and s > 0.5 * mx] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "window": "warm pass + timed region"}
 
 
 # ---------------------------------------------------------------- our arm
@@ -258,13 +281,14 @@ def run_ours(args):
     # workload (an event node between two kernels serialises them fully).
     n_items = len(suite.items)
     use_graph = not args.no_graph
+    n_ev = min(args.steps, 20)  # steps of the per-workload breakdown graph
     ev = [[(torch.cuda.Event(enable_timing=True, external=use_graph),
             torch.cuda.Event(enable_timing=True, external=use_graph)) for _ in range(n_items)]
-          for _ in range(args.steps)]
+          for _ in range(n_ev)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
     def k_steps(stream_handle, with_events):
-        for s in range(args.steps):
+        for s in range(n_ev if with_events else args.steps):
             for i, it in enumerate(suite.items):
                 if with_events:
                     ev[s][i][0].record()
@@ -284,6 +308,7 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         # the sampler's start leaves the GPU idle for a moment: one more untimed pass of the
         # K steps brings the clocks back up before the barrier that opens the timed region
+        clk.mark()
         if graph is not None:
             graph.replay()
         else:
@@ -310,14 +335,14 @@ def run_ours(args):
     torch.cuda.synchronize()
     per_item = {}
     for i, it in enumerate(suite.items):
-        times = [ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)]
+        times = [ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(n_ev)]
         per_item[it["w"].name] = {"ms_mean": sum(times) / len(times), "ms_median": statistics.median(times)}
 
     # ---- e2e through the public API with host buffers: pinned H2D of every operand,
     # the launches, D2H of every result, all inside the timed region
     e2e = e2e_measure(suite, stream, sh, args, ws)
 
-    value = ws * suite.flops * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_tflops(ws, suite.flops, args.steps, total_ms)
     breakdown = {}
     for it in suite.items:
         w = it["w"]
@@ -331,7 +356,7 @@ def run_ours(args):
     dom_w = dom["w"]
     # the dominant fused GEMM launch alone (its dReLU follows inside the same event pair,
     # so the forward is timed separately below on the same stream)
-    fwd_ms = time_single_launch(suite, dom, stream, sh, reps=max(10, args.steps // 2))
+    fwd_ms = time_single_launch(suite, dom, stream, sh, reps=max(10, min(100, args.steps // 2)))
     achieved = dom_w.flops / (fwd_ms * 1e-3) / 1e12
     peak = pk["bf16_tflops_sustained"]
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
@@ -657,7 +682,7 @@ def run_reference(args):
     if rank != 0:
         return
     # steps x warmup of bounded oracle samples; the whole run stays within minutes
-    per_step = max(0.25, min(6.0, 60.0 / max(1, args.steps + args.warmup)))
+    per_step = max(0.05, min(6.0, 60.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         _oracle_sample(per_step / 4)
     tot_f, tot_t, cores, desc = 0.0, 0.0, 1, ""
