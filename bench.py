@@ -409,7 +409,7 @@ class L2Flush:
         import torch
         n = 256 * 1024 * 1024 // 4
         self.w = torch.empty(n, dtype=torch.int32, device="cuda")
-        self.r = torch.zeros(n, dtype=torch.int32, device="cuda")
+        self.r = torch.zeros(n, dtype=torch.float32, device="cuda")  # fp32: sum() reads it without a cast copy
 
     def __call__(self):
         self.w.zero_()
