@@ -187,7 +187,7 @@ struct LnParams {
   const void* x;      // [M, ldx] of XT
   const void* gamma;  // [N] of param_dtype, or null (1)
   const void* beta;   // [N] of param_dtype, or null (0)
-  void* z;            // [M, ldz] of ZT (may alias x)
+  void* z;            // [M, ldz] of ZT (may be x itself, with ldz == ldx)
   long long M, N, ldx, ldz;
   int param_dtype, vec_ok;
   int pvec;  // gamma/beta 16-byte aligned: loaded as vectors

@@ -184,7 +184,8 @@ fl_status fl_wait_selftest(uint64_t limit_ns, void* stream);
  * and variance and the normalisation in one kernel, one read and one write):
  *   z[m,n] = (x[m,n] − μ_m)/√(σ²_m + eps)·gamma[n] + beta[n],
  *   μ_m = mean of row m, σ²_m = mean of (x − μ_m)² (population variance), in fp32.
- *   x  [M, ld_x] of x_dtype; z [M, ld_z] of z_dtype (may alias x when the types match)
+ *   x  [M, ld_x] of x_dtype; z [M, ld_z] of z_dtype.  In place: z == x with the same
+ *   type and ld_z == ld_x (each row is read before it is written; other overlaps race)
  *   gamma, beta [N] of param_dtype; null gamma = 1, null beta = 0
  * Errors: FL_ERR_INVALID_ARG (null x/z, negative size, ld < N, eps < 0, M ≥ 2^31),
  * FL_ERR_ALIGNMENT, FL_ERR_CUDA. */
