@@ -9,8 +9,8 @@ without a B200.
 The entry points keep the C names: ``fl_plan``, ``fl_execute``, ``fl_free``,
 ``fl_relu_backward``, ``fl_check_status``, ``fl_get_plan_info``,
 ``fl_last_error``, ``fl_set_wait_limit_ns``, ``fl_execute_noalloc``, ``fl_bias_grad_workspace_size``,
-``fl_drelu_bgrad``, ``fl_dgelu_bgrad``, ``fl_layernorm``, ``fl_wait_selftest``.  ``Plan`` is a small owner of one
-plan handle (the cuBLASLt epilog page's Matmul → plan → execute → free).
+``fl_drelu_bgrad``, ``fl_dgelu_bgrad``, ``fl_layernorm``, ``fl_wait_selftest``, ``fl_plan_preview``.
+``Plan`` is a small owner of one plan handle (the cuBLASLt epilog page's Matmul → plan → execute → free).
 """
 from __future__ import annotations
 
@@ -36,7 +36,8 @@ COMPUTES = {"32F": FL_COMPUTE_32F, "32F_3XTF32": FL_COMPUTE_32F_3XTF32}
 
 EXPORTED = ["fl_plan", "fl_execute", "fl_relu_backward", "fl_check_status", "fl_get_plan_info",
             "fl_free", "fl_last_error", "fl_set_wait_limit_ns", "fl_execute_noalloc",
-            "fl_bias_grad_workspace_size", "fl_drelu_bgrad", "fl_dgelu_bgrad", "fl_layernorm", "fl_wait_selftest"]
+            "fl_bias_grad_workspace_size", "fl_drelu_bgrad", "fl_dgelu_bgrad", "fl_layernorm", "fl_wait_selftest",
+            "fl_plan_preview"]
 
 
 class fl_epilogue_desc(ctypes.Structure):
@@ -72,6 +73,9 @@ def _load() -> ctypes.CDLL:
     lib.fl_check_status.restype = i32
     lib.fl_get_plan_info.argtypes = [vp, ctypes.POINTER(fl_plan_info)]
     lib.fl_get_plan_info.restype = i32
+    lib.fl_plan_preview.argtypes = [i64, i64, i64, i32, i32, ctypes.POINTER(fl_epilogue_desc), i32, i32,
+                                    ctypes.POINTER(fl_plan_info)]
+    lib.fl_plan_preview.restype = i32
     lib.fl_free.argtypes = [vp]
     lib.fl_free.restype = i32
     lib.fl_last_error.argtypes = []
@@ -221,6 +225,17 @@ def fl_check_status(plan: int, stream=None) -> int:
 def fl_get_plan_info(plan: int) -> dict:
     info = fl_plan_info()
     _check(LIB.fl_get_plan_info(plan, ctypes.byref(info)), "fl_get_plan_info")
+    return {k: getattr(info, k) for k, _ in fl_plan_info._fields_ if k != "reserved"}
+
+
+def fl_plan_preview(M: int, N: int, K: int, dtype: str = "bf16", compute: str = "32F", *, num_sms: int = 148,
+                    max_smem_per_block: int = 232448, **epi) -> dict:
+    """The configuration fl_plan would choose on a device with `num_sms` SMs and that much
+    opt-in shared memory per block, computed on the host (no device needed)."""
+    info = fl_plan_info()
+    e = make_epilogue(**epi)
+    _check(LIB.fl_plan_preview(int(M), int(N), int(K), DTYPES[dtype], COMPUTES[compute], ctypes.byref(e),
+                               int(num_sms), int(max_smem_per_block), ctypes.byref(info)), "fl_plan_preview")
     return {k: getattr(info, k) for k, _ in fl_plan_info._fields_ if k != "reserved"}
 
 

@@ -381,10 +381,20 @@ static fl_status choose_config(fl_plan_s* p) {
   return FL_OK;
 }
 
-extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, int32_t dtype,
-                             int32_t compute, const fl_epilogue_desc* epi) {
-  g_err[0] = 0;
-  if (!out || !epi) return fail(FL_ERR_INVALID_ARG, "fl_plan: null out or epilogue descriptor");
+// Launches of one unfused execute: the bare GEMM, then one elementwise kernel per step.
+static int unfused_launches(const fl_plan_s* p) {
+  int steps = 0;
+  if (p->epi.kind == FL_EPI_GEGLU_TANH) steps += 1;
+  else steps += (p->has_bias ? 1 : 0) + (p->act != ACT_NONE ? 1 : 0);
+  steps += (p->epi.has_residual ? 1 : 0) + (p->epi.scale != 1.0f ? 1 : 0);
+  return 1 + steps;
+}
+
+// Everything fl_plan checks and records before it touches the device: the shape, the
+// types, the epilogue descriptor and the row pitches.  On success *out is a new host
+// plan (no device state yet) that the caller owns.
+static fl_status plan_host_part(fl_plan_s** out, int64_t M, int64_t N, int64_t K, int32_t dtype, int32_t compute,
+                                const fl_epilogue_desc* epi) {
   *out = nullptr;
   if (M < 1 || N < 1 || K < 0) return fail(FL_ERR_INVALID_ARG, "fl_plan: need M>=1, N>=1, K>=0 (got %lld %lld %lld)",
                                            (long long)M, (long long)N, (long long)K);
@@ -444,6 +454,21 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
     delete p;
     return fail(FL_ERR_ALIGNMENT, "fl_plan: every row pitch must be a multiple of 16 bytes");
   }
+  *out = p;
+  return FL_OK;
+}
+
+extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, int32_t dtype,
+                             int32_t compute, const fl_epilogue_desc* epi) {
+  g_err[0] = 0;
+  if (!out || !epi) return fail(FL_ERR_INVALID_ARG, "fl_plan: null out or epilogue descriptor");
+  *out = nullptr;
+  fl_plan_s* p = nullptr;
+  {
+    const fl_status st0 = plan_host_part(&p, M, N, K, dtype, compute, epi);
+    if (st0 != FL_OK) return st0;
+  }
+  const int eo = esize(epi->out_dtype);
 
   if (cudaGetDevice(&p->device) != cudaSuccess) { delete p; return fail(FL_ERR_DEVICE, "fl_plan: no CUDA device"); }
   cudaDeviceProp prop;
@@ -498,11 +523,7 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
         return fail(FL_ERR_CUDA, "cudaFuncSetAttribute (unfused GEMM)");
       }
     }
-    int steps = 0;
-    if (epi->kind == FL_EPI_GEGLU_TANH) steps += 1;
-    else steps += (has_bias ? 1 : 0) + (p->act != ACT_NONE ? 1 : 0);
-    steps += (epi->has_residual ? 1 : 0) + (p->epi.scale != 1.0f ? 1 : 0);
-    p->launches = 1 + steps;
+    p->launches = unfused_launches(p);
     // GEMM into a plan-owned intermediate (the [M, N] or [M, 2N] result), then one
     // elementwise kernel per epilogue step.
     const int64_t cols = (epi->kind == FL_EPI_GEGLU_TANH) ? 2 * N : N;
@@ -516,6 +537,43 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
   }
   *out = p;
   return FL_OK;
+}
+
+// The configuration fl_plan would choose on a device with `num_sms` SMs and
+// `max_smem_per_block` bytes of opt-in shared memory per block, without touching any
+// device: the same checks, the same choice, nothing allocated.
+extern "C" fl_status fl_plan_preview(int64_t M, int64_t N, int64_t K, int32_t dtype, int32_t compute,
+                                     const fl_epilogue_desc* epi, int32_t num_sms, int32_t max_smem_per_block,
+                                     fl_plan_info* info) {
+  g_err[0] = 0;
+  if (!epi || !info) return fail(FL_ERR_INVALID_ARG, "fl_plan_preview: null epilogue descriptor or info");
+  if (num_sms < 2 || num_sms > 4096 || max_smem_per_block < 16384)
+    return fail(FL_ERR_INVALID_ARG, "fl_plan_preview: implausible device (%d SMs, %d bytes of shared memory)",
+                num_sms, max_smem_per_block);
+  fl_plan_s* p = nullptr;
+  const fl_status st = plan_host_part(&p, M, N, K, dtype, compute, epi);
+  if (st != FL_OK) return st;
+  p->num_sms = num_sms;
+  p->max_smem = max_smem_per_block;
+  choose_config(p);
+  const int b_boxes = b_boxes_of(p, p->epi.kind == FL_EPI_GEGLU_TANH);
+  const Layout L = layout_for(p, p->mma_n, b_boxes, p->max_smem);
+  fl_status r = FL_OK;
+  if (L.stages < 2) {
+    r = fail(FL_ERR_UNSUPPORTED, "fl_plan_preview: shared memory too small");
+  } else {
+    p->stages = L.stages;
+    p->smem = (int)L.total;
+    p->grid = grid_of(p);
+    if (!kernel_of(p, p->act, p->epi.out_dtype)) {
+      r = fail(FL_ERR_UNSUPPORTED, "fl_plan_preview: no kernel for this combination");
+    } else {
+      p->launches = p->epi.unfused ? unfused_launches(p) : 1;
+      r = fl_get_plan_info(p, info);
+    }
+  }
+  delete p;
+  return r;
 }
 
 extern "C" fl_status fl_get_plan_info(fl_plan_t p, fl_plan_info* info) {

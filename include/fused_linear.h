@@ -213,6 +213,18 @@ typedef struct {
 } fl_plan_info;
 fl_status fl_get_plan_info(fl_plan_t plan, fl_plan_info* info);
 
+/* The configuration fl_plan would choose for these arguments on a device with
+ * num_sms SMs and max_smem_per_block bytes of opt-in shared memory per block (B200:
+ * 148 and 232448), computed on the host alone: the same argument checks and the same
+ * choice as fl_plan, no device call, nothing allocated.  Lets a caller (or a test
+ * without a GPU) inspect the layout, split-K and grid fl_plan will use.
+ * Errors: those of fl_plan's argument checks; FL_ERR_INVALID_ARG for a null pointer or
+ * an implausible device (num_sms outside [2, 4096], max_smem_per_block < 16384);
+ * FL_ERR_UNSUPPORTED when no configuration fits. */
+fl_status fl_plan_preview(int64_t M, int64_t N, int64_t K, int32_t dtype, int32_t compute,
+                          const fl_epilogue_desc* epi, int32_t num_sms, int32_t max_smem_per_block,
+                          fl_plan_info* info);
+
 /* Release a plan and its workspace ([epilog] free()).  NULL is accepted.
  * Synchronises nothing: the caller must not free a plan with work in flight. */
 fl_status fl_free(fl_plan_t plan);
