@@ -385,6 +385,7 @@ def run_ours(args):
         "breakdown": breakdown,
         "hbm_kernels": time_backward(fl, pk),
         "gelu_sigmoid_1024x3072x768_bf16": time_gelu_sigmoid(fl, pk),
+        "fusion": time_fusion(suite, fl),
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
@@ -529,6 +530,87 @@ def time_gelu_sigmoid(fl, pk, reps=10):
     ms = sum(a.elapsed_time(e) for a, e in evs) / reps
     tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
     return {"us": round(ms * 1e3, 2), "tflops": round(tf, 1), "frac_of_bf16_burst": round(tf / pk["bf16_tflops"], 3)}
+
+
+FUSION_SET = ["linear_gelu_tanh_bf16_1024x3072x768", "geglu_mlp_8192x3072x768", "relu_aux_4096", "tail_m128",
+              "tail_m2048"]
+
+
+def _time_launch(fn, flush, reps):
+    """Mean CUDA-event time (ms) of fn() on the current stream, each launch after an L2 flush."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in evs:
+        flush()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / reps
+
+
+def time_fusion(suite, fl, reps=10):
+    """What fusion buys, per workload: the fused launch, the bare GEMM (epilogue NONE,
+    same operands and output type) and the unfused twin (the bare GEMM into an
+    intermediate, then one elementwise kernel per epilogue step), each after an L2
+    flush.  epilogue_overhead = fused / bare − 1; round_trip_us = unfused − fused.
+    For GeGLU the dual gate/up GEMM is compared (the down projection is the same plain
+    GEMM either way).  A workload whose measurement fails records the error instead."""
+    import torch
+    flush = L2Flush()
+    sh = torch.cuda.current_stream().cuda_stream
+    out = {}
+    for it in suite.items:
+        w = it["w"]
+        if w.name not in FUSION_SET:
+            continue
+        plans = []
+        try:
+            d = it["dev"]
+            if w.kind == "geglu":
+                h2 = torch.empty(w.M, 2 * w.N, dtype=torch.bfloat16, device="cuda")
+                bare = fl.Plan(w.M, 2 * w.N, w.K, kind="NONE", out_dtype="bf16")
+                unf = fl.Plan(w.M, w.N, w.K, kind="GEGLU_TANH", out_dtype="bf16", unfused=True)
+                plans += [bare, unf]
+                fused_fn = lambda: it["plans"][0].execute(d["x"], d["Wgu"], out=it["h"], stream=sh)
+                bare_fn = lambda: bare.execute(d["x"], d["Wgu"], out=h2, stream=sh)
+                unf_fn = lambda: unf.execute(d["x"], d["Wgu"], out=it["h"], stream=sh)
+            else:
+                compute = "32F_3XTF32" if w.dtype == "f32" else "32F"
+                Wt = d["B"] if w.b_major else d["W"]
+                ob = torch.empty_like(it["out"])
+                bare = fl.Plan(w.M, w.N, w.K, dtype=w.dtype, compute=compute, kind="NONE", out_dtype=w.out_dtype,
+                               b_major=w.b_major)
+                unf = fl.Plan(w.M, w.N, w.K, dtype=w.dtype, compute=compute, kind=w.epilogue, out_dtype=w.out_dtype,
+                              bias_dtype=w.bias_dtype or "bf16", residual_dtype=w.dtype, bias_axis=w.bias_axis,
+                              has_residual=w.residual, scale=w.scale, b_major=w.b_major, unfused=True)
+                plans += [bare, unf]
+                args = (d["A"], Wt, d.get("bias"), it["aux"], d.get("residual"))
+                fused_fn = lambda: it["plans"][0].execute(*args, it["out"], stream=sh)
+                bare_fn = lambda: bare.execute(d["A"], Wt, out=ob, stream=sh)
+                unf_fn = lambda: unf.execute(*args, ob, stream=sh)
+            t_f = _time_launch(fused_fn, flush, reps)
+            t_b = _time_launch(bare_fn, flush, reps)
+            t_u = _time_launch(unf_fn, flush, reps)
+            for p in plans + [it["plans"][0]]:
+                if p.check() != fl.FL_OK:
+                    raise RuntimeError(fl.fl_last_error())
+            out[w.name] = {"fused_us": round(t_f * 1e3, 2), "bare_gemm_us": round(t_b * 1e3, 2),
+                           "unfused_us": round(t_u * 1e3, 2), "unfused_launches": unf.info()["launches_per_execute"],
+                           "epilogue_overhead": round(t_f / t_b - 1.0, 3), "round_trip_us": round((t_u - t_f) * 1e3, 2)}
+        except Exception as e:  # keep the rest of the line
+            out[w.name] = {"error": str(e)[:200]}
+        finally:
+            try:
+                torch.cuda.synchronize()
+                for p in plans:
+                    p.free()
+            except Exception:
+                pass
+    del flush
+    return out
 
 
 def profiled_traffic():
