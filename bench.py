@@ -40,6 +40,11 @@ SUITE = ["relu_bias_100x256x784", "linear_gelu_f32_1024x3072x768", "linear_gelu_
 DOMINANT = "relu_aux_4096"   # the largest single fused launch of the step
 
 
+def workload_desc(names):
+    """The `config.workload` string of both arms: the step's workloads by name and size."""
+    return "all synthetic workloads of the fused linear layer, one fused launch each: " + ", ".join(names)
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -369,8 +374,7 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "all synthetic workloads of the fused linear layer, one fused launch each: "
-                               + ", ".join(it["w"].name for it in suite.items),
+        "config": {"workload": workload_desc([it["w"].name for it in suite.items]),
                    "timed_as": "one CUDA graph of the K steps" if use_graph else "eager launches",
                    "flops_per_step": suite.flops, "parallelism": f"replicas x{ws}",
                    "l2": "inputs larger than L2: every workload owns its operands; a step touches "
@@ -776,8 +780,8 @@ def run_reference(args):
     line = {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * tot_t / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "all synthetic workloads of the fused linear layer (row-sliced sample)",
-                       "parallelism": "host cores"},
+            "config": {"workload": workload_desc(SUITE), "parallelism": "host cores",
+                       "sample": "row slices of every workload, about 0.05-6 s of oracle work per step"},
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": desc + f"; per step about {per_step:.1f} s"},
