@@ -128,6 +128,17 @@ def pin_gelu_erf_series(o):
     assert got[xs == 0.0][0] == 0.0
 
 
+def pin_gelu_closed_forms(o):
+    """GELU(x) = x·Φ(x) at points where Φ is tabulated: the standard normal CDF to 15 digits
+    (Abramowitz & Stegun, Table 26.1): Φ(0.5) = 0.691462461274013, Φ(1) = 0.841344746068543,
+    Φ(2) = 0.977249868051821, and Φ(−x) = 1 − Φ(x)."""
+    table = {0.5: 0.691462461274013, 1.0: 0.841344746068543, 2.0: 0.977249868051821}
+    for x, phi in table.items():
+        got = o.gelu_erf(np.array([x, -x]))
+        assert abs(got[0] - x * phi) < 1e-14, (x, got[0])
+        assert abs(got[1] - (-x) * (1.0 - phi)) < 1e-14, (-x, got[1])
+
+
 def pin_gelu_identities(o):
     x = np.linspace(-8, 8, 4001)
     for f in (o.gelu_erf, o.gelu_tanh):
