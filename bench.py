@@ -536,8 +536,7 @@ def time_gelu_sigmoid(fl, pk, reps=10):
     return {"us": round(ms * 1e3, 2), "tflops": round(tf, 1), "frac_of_bf16_burst": round(tf / pk["bf16_tflops"], 3)}
 
 
-FUSION_SET = ["linear_gelu_tanh_bf16_1024x3072x768", "geglu_mlp_8192x3072x768", "relu_aux_4096", "tail_m128",
-              "tail_m2048"]
+FUSION_SET = ["linear_gelu_tanh_bf16_1024x3072x768", "geglu_mlp_8192x3072x768", "relu_aux_4096", "tail_m2048"]
 
 
 def _time_launch(fn, flush, reps):
