@@ -705,7 +705,7 @@ def e2e_measure(suite, stream, sh, args, ws):
 _ORACLE_INPUTS = {}
 
 
-def _oracle_sample(seconds):
+def _oracle_sample(seconds, rows_per_chunk=64):
     """Run the oracle (as it stands) over row-slices of every workload until about
     `seconds` of CPU work is done; returns (flops, elapsed, cores, description)."""
     import numpy as np
@@ -717,7 +717,6 @@ def _oracle_sample(seconds):
     except Exception:
         cores = os.cpu_count() or 1
     flops, elapsed, parts = 0.0, 0.0, []
-    rows_per_chunk = 64
     names = [n for n in SUITE]
     data = _ORACLE_INPUTS  # generated once per process, outside the timed CPU work
     for n in names:
@@ -768,11 +767,12 @@ def run_reference(args):
         return
     # steps x warmup of bounded oracle samples; the whole run stays within minutes
     per_step = max(0.05, min(6.0, 60.0 / max(1, args.steps + args.warmup)))
+    rows = 64 if per_step >= 0.5 else 16  # short steps: one pass of 16-row slices (about 0.04 s)
     for _ in range(args.warmup):
-        _oracle_sample(per_step / 4)
+        _oracle_sample(per_step / 4, rows)
     tot_f, tot_t, cores, desc = 0.0, 0.0, 1, ""
     for _ in range(args.steps):
-        f, t, cores, desc = _oracle_sample(per_step)
+        f, t, cores, desc = _oracle_sample(per_step, rows)
         tot_f += f
         tot_t += t
     value = tot_f / tot_t / 1e12
