@@ -1,0 +1,76 @@
+"""Register, spill and shared-memory figures of the built kernels (from `ptxas -v`).
+
+build.py keeps the assembler's resource report beside the library.  The launch
+configurations assume these figures, so a change that breaks one shows up here, on the
+CPU, before it shows up as lost occupancy on the GPU:
+- the fused kernel runs 320 threads a CTA, one CTA per SM: at most 204 registers;
+- the dominant launch (ReLU + mask, bf16 out, CTA pair) has no spills;
+- the dReLU and bias-gradient kernels hold four 256-thread CTAs per SM (≤ 64 registers);
+- the whole-vector LayerNorm holds six 128-thread CTAs per SM (≤ 85 registers).
+Skipped when the report is missing (the library was not built here).
+"""
+from __future__ import annotations
+
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+REPORT = os.path.join(ROOT, "gemm_bias_activation_tcgen05_b200", "ptxas_report.txt")
+
+
+def _entries():
+    if not os.path.exists(REPORT):
+        pytest.skip("no ptxas report (library not built here)")
+    out, cur = {}, None
+    for line in open(REPORT):
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            cur = m.group(1)
+            out[cur] = {}
+            continue
+        if cur is None:
+            continue
+        m = re.search(r"(\d+) bytes spill stores, (\d+) bytes spill loads", line)
+        if m:
+            out[cur]["spill"] = int(m.group(1)) + int(m.group(2))
+        m = re.search(r"Used (\d+) registers", line)
+        if m:
+            out[cur]["regs"] = int(m.group(1))
+    return out
+
+
+def _select(entries, prefix):
+    sel = {k: v for k, v in entries.items() if k.startswith(prefix)}
+    assert sel, f"no kernel named {prefix}* in the report"
+    return sel
+
+
+def test_fused_kernel_fits_one_cta_of_320_threads():
+    for name, v in _select(_entries(), "_ZN2fl19fl_gemm_epi_tcgen05").items():
+        assert v["regs"] * 320 <= 65536, (name, v)
+
+
+def test_dominant_launch_has_no_spills():
+    # fl_gemm_epi_tcgen05<ACT_RELU, OUT_BF16, swap=false, tf32=false, pair=true>
+    name = "_ZN2fl19fl_gemm_epi_tcgen05ILi1ELi1ELb0ELb0ELb1EEEv14CUtensorMap_stS1_S1_S1_NS_7KParamsE"
+    e = _entries()
+    assert name in e
+    assert e[name]["spill"] == 0, e[name]
+
+
+@pytest.mark.parametrize("prefix,max_regs", [
+    ("_ZN2fl23fl_relu_backward_kernel", 64),
+    ("_ZN2fl19fl_bwd_bgrad_kernel", 64),
+])
+def test_hbm_kernels_keep_four_ctas_of_256(prefix, max_regs):
+    for name, v in _select(_entries(), prefix).items():
+        assert v["regs"] <= max_regs, (name, v)
+
+
+def test_vector_layernorm_keeps_six_ctas_of_128():
+    for name, v in _select(_entries(), "_ZN2fl23fl_layernorm_vec_kernel").items():
+        if "Li128EEEv" in name:  # the TPB = 128 instantiations
+            assert v["regs"] * 128 * 6 <= 65536, (name, v)
+            assert v["spill"] == 0, (name, v)
