@@ -238,6 +238,53 @@ def pin_geglu_identity(o):
     assert np.array_equal(y, hh)
 
 
+def _geglu_mlp_loops(x, Wg, Wu, Wd, round_h, round_fn):
+    """GeGLU MLP by per-element loops: h = gelu_tanh(x·Wgᵀ)·(x·Wuᵀ) with math.tanh, optionally
+    rounded to bf16, then y[m,j] = Σ_n h[m,n]·Wd[j,n] (Wd is the down projection's [K, N] weight)."""
+    M, K = x.shape
+    N, J = Wg.shape[0], Wd.shape[0]
+    c = math.sqrt(2.0 / math.pi)
+    h = np.zeros((M, N))
+    for m in range(M):
+        for n in range(N):
+            g = sum(x[m, k] * Wg[n, k] for k in range(K))
+            u = sum(x[m, k] * Wu[n, k] for k in range(K))
+            h[m, n] = 0.5 * g * (1.0 + math.tanh(c * (g + 0.044715 * g ** 3))) * u
+    if round_h:
+        h = round_fn(h)
+    y = np.zeros((M, J))
+    for m in range(M):
+        for j in range(J):
+            y[m, j] = sum(h[m, n] * Wd[j, n] for n in range(N))
+    return round_fn(h), round_fn(y)
+
+
+def pin_geglu_mlp_bf16_brute_force(o):
+    """The whole MLP in bf16 against loops, with a rectangular (K≠N) and a square non-symmetric
+    down-projection weight: h is rounded to bf16 before the down projection (h is a bf16 tensor),
+    and Wd is read as [out, in].  The inputs are chosen so that skipping the rounding of h
+    changes y (checked here, so the pin stays sensitive to it)."""
+    def bf16(v):
+        # torch's float32 -> bfloat16 cast on values first rounded to float32 (ties are
+        # not reached by these sums of products of bf16 values at this size)
+        return torch.from_numpy(np.asarray(v, np.float64)).to(torch.float32).to(torch.bfloat16) \
+            .to(torch.float64).numpy()
+    for (M, K, N, seed) in [(4, 6, 10, 100), (3, 7, 7, 105)]:
+        r = _rng(seed)
+        x = bf16(r.standard_normal((M, K)))
+        Wg = bf16(r.standard_normal((N, K)) * 0.5)
+        Wu = bf16(r.standard_normal((N, K)) * 0.5)
+        Wd = bf16(r.standard_normal((K, N)) * 0.5)
+        h_ref, y_ref = _geglu_mlp_loops(x, Wg, Wu, Wd, True, bf16)
+        _, y_unrounded_h = _geglu_mlp_loops(x, Wg, Wu, Wd, False, bf16)
+        assert (y_ref != y_unrounded_h).any()      # the case distinguishes the two readings
+        if K == N:
+            assert not np.array_equal(Wd, Wd.T)    # a transposed Wd gives other values
+        h, y = o.geglu_mlp(x, Wg, Wu, Wd, "bf16")
+        assert np.array_equal(h, h_ref), (M, K, N)
+        assert np.array_equal(y, y_ref), (M, K, N)
+
+
 def pin_gelu_sigmoid_page_form(o):
     """x·σ(1.702x) with the page's constant, per element against math.exp."""
     k = _golden()["gelu_sigmoid_k"]["value"]

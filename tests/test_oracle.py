@@ -155,6 +155,14 @@ MUTANTS = {
         / np.sqrt(np.asarray(x, float).var(-1, keepdims=True) + eps) * g, od)),
     "drelu_inverted": dict(drelu=lambda grad, aux, N, od="bf16": oracle.round_to(
         np.asarray(grad, float)[:, :N] - oracle.drelu(grad, aux, N, od), od)),
+    # the down projection of the unrounded h (h kept in fp64 instead of the bf16 tensor)
+    "geglu_mlp_skips_h_rounding": dict(geglu_mlp=lambda x, Wg, Wu, Wd, od="bf16": (
+        oracle.geglu_h(x, Wg, Wu, od),
+        oracle.round_to(oracle.gemm(oracle.gelu_tanh(oracle.gemm(x, Wg)) * oracle.gemm(x, Wu), Wd), od))),
+    # Wd read as [in, out] (h @ Wd in place of h @ Wdᵀ)
+    "geglu_mlp_transposed_wd": dict(geglu_mlp=lambda x, Wg, Wu, Wd, od="bf16": (
+        oracle.geglu_h(x, Wg, Wu, od),
+        oracle.round_to(oracle.gemm(oracle.geglu_h(x, Wg, Wu, od), Wd, b_major=1), od))),
 }
 
 
