@@ -111,34 +111,77 @@ def job_tflops(ws, flops_per_step, steps, total_ms):
 
 
 # ---------------------------------------------------------------- clocks
+REASON_BITS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
+
+
 class ClockSampler:
-    """nvidia-smi samples every 200 ms while the context is open; summary() keeps the
-    samples taken after mark() (the warm pass and the timed region, both under load)."""
-    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons, sampled while the context is open.
 
-    def __init__(self, gpu_index):
+    NVML is read every 5 ms from a host thread (read-only queries); without NVML,
+    nvidia-smi prints a sample every 200 ms.  Samples are (time.time(), sm MHz, max MHz,
+    reasons).  phase(name) opens a named interval that lasts until the next phase() or
+    the end, so that the summary of an interval holds the samples taken while that
+    work ran: the timed region is preceded by a warm pass of at least one second,
+    which guarantees samples under the same load at any number of steps."""
+    PERIOD_S = 0.005
+
+    def __init__(self, gpu_index, pci_bus_id=None):
         self.idx = gpu_index
+        self.pci = pci_bus_id
         self.proc = None
-        self.t_mark = None
+        self.thread = None
+        self.samples = []
+        self.lines = []
+        self.phases = []  # (name, t_start)
+        self.source = None
+        self._stop = False
 
-    def mark(self):
-        import datetime
-        self.t_mark = datetime.datetime.now()
+    def phase(self, name):
+        self.phases.append((name, time.time()))
+
+    def _nvml_loop(self, nv, h):
+        while not self._stop:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((time.time(), float(sm), float(mx),
+                                     frozenset(n for n, b in REASON_BITS if rs & b)))
+            except Exception:
+                pass
+            time.sleep(self.PERIOD_S)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-        time.sleep(0.3)
+            import threading
+            import pynvml as nv
+            nv.nvmlInit()
+            h = None
+            if self.pci:
+                try:
+                    h = nv.nvmlDeviceGetHandleByPciBusId(self.pci)
+                except Exception:
+                    h = None
+            if h is None:
+                h = nv.nvmlDeviceGetHandleByIndex(self.idx)
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self.thread.start()
+            self.source = "nvml, 5 ms"
+        except Exception:
+            try:
+                self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={SMI_QUERY}",
+                                              "--format=csv,noheader,nounits", "-lms", "200"],
+                                             stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.source = "nvidia-smi, 200 ms"
+            except OSError:
+                self.proc = None
         return self
 
     def __exit__(self, *a):
-        self.lines = []
+        self._stop = True
+        if self.thread is not None:
+            self.thread.join(timeout=2)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -148,33 +191,45 @@ class ClockSampler:
                 out, _ = self.proc.communicate()
             self.lines = [l for l in out.splitlines() if l.strip()]
 
-    def summary(self):
+    def _all(self):
+        """NVML samples, or the nvidia-smi lines parsed into the same form."""
         import datetime
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        out = list(self.samples)
+        for l in self.lines:
             f = [x.strip() for x in l.split(",")]
             if len(f) < 10:
                 continue
-            if self.t_mark is not None:
-                try:
-                    ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f")
-                    if ts < self.t_mark - datetime.timedelta(milliseconds=50):
-                        continue  # taken while the GPU idled before the warm pass
-                except ValueError:
-                    pass
             try:
-                sm.append(float(f[2]))
-                mx = float(f[3])
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                sm, mx = float(f[2]), float(f[3])
             except ValueError:
                 continue
-            for name, val in zip(names, f[6:10]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm), "window": "warm pass + timed region"}
+            rs = frozenset(n for (n, _), v in zip(REASON_BITS, f[6:10]) if v.lower().startswith("active"))
+            out.append((ts, sm, mx, rs))
+        return sorted(out, key=lambda x: x[0])
+
+    def summary(self, name=None):
+        """Median SM clock, max clock and every reason seen, over the samples of phase
+        `name` (all phases when None)."""
+        smp = self._all()
+        if name is not None:
+            bounds = [(n, t, self.phases[i + 1][1] if i + 1 < len(self.phases) else float("inf"))
+                      for i, (n, t) in enumerate(self.phases)]
+            sel = [(t0, t1) for n, t0, t1 in bounds if n == name]
+            smp = [x for x in smp if any(t0 <= x[0] < t1 for t0, t1 in sel)]
+        elif self.phases:
+            smp = [x for x in smp if x[0] >= self.phases[0][1]]
+        mx = max((x[2] for x in smp), default=None)
+        reasons = sorted(set().union(*[x[3] for x in smp])) if smp else []
+        if not smp:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": reasons, "samples": 0, "source": self.source}
+        return {"sm_mhz": statistics.median(x[1] for x in smp), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(smp), "source": self.source}
+
+
+SMI_QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
 
 # ---------------------------------------------------------------- our arm
@@ -310,24 +365,37 @@ def run_ours(args):
             k_steps(torch.cuda.current_stream().cuda_stream, True)
         graph.replay()  # one untimed replay of the captured steps
         torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        # the sampler's start leaves the GPU idle for a moment: one more untimed pass of the
-        # K steps brings the clocks back up before the barrier that opens the timed region
-        clk.mark()
+    pci = None
+    try:
+        pr = torch.cuda.get_device_properties(torch.cuda.current_device())
+        pci = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+    except Exception:
+        pass
+    clk = ClockSampler(local, pci).__enter__()
+    # warm pass: replays of the K steps for at least one second, so that the clocks and
+    # the power draw settle under the step's load and the sampler has samples of it at
+    # any K; then the timed region, bracketed by a barrier and a synchronize
+    clk.phase("warm")
+    t_warm = time.time()
+    while True:
         if graph is not None:
             graph.replay()
         else:
             k_steps(sh, False)
         torch.cuda.synchronize()
-        barrier(ws)
-        torch.cuda.synchronize()
-        t0.record(stream)
-        if graph is not None:
-            graph.replay()
-        else:
-            k_steps(sh, False)
-        t1.record(stream)
-        torch.cuda.synchronize()
+        if time.time() - t_warm >= 1.0:
+            break
+    barrier(ws)
+    torch.cuda.synchronize()
+    clk.phase("timed")
+    t0.record(stream)
+    if graph is not None:
+        graph.replay()
+    else:
+        k_steps(sh, False)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk.phase("after")
     barrier(ws)
     total_ms = max_over_ranks(t0.elapsed_time(t1), ws)
     suite.check()
@@ -360,15 +428,34 @@ def run_ours(args):
     dom = suite.items[[it["w"].name for it in suite.items].index(DOMINANT)]
     dom_w = dom["w"]
     # the dominant fused GEMM launch alone (its dReLU follows inside the same event pair,
-    # so the forward is timed separately below on the same stream)
+    # so the forward is timed separately below on the same stream), each launch after an
+    # L2 flush: a burst of isolated launches, compared with the burst bf16 peak
+    clk.phase("roofline")
     fwd_ms = time_single_launch(suite, dom, stream, sh, reps=max(10, min(100, args.steps // 2)))
+    clk.phase("after")
+    clk.phase("side")
+    hbm = time_backward(fl, pk)
+    sig = time_gelu_sigmoid(fl, pk)
+    fusion = time_fusion(suite, fl)
+    clk.__exit__(None, None, None)
     achieved = dom_w.flops / (fwd_ms * 1e-3) / 1e12
-    peak = pk["bf16_tflops_sustained"]
+    peak = pk["bf16_tflops"]
+    roof_clk = clk.summary("roofline")
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 3), "traffic": profiled_traffic(), "kernel": "fl_gemm_epi_tcgen05",
-                "launch": f"{DOMINANT} forward (M=N=K=4096, RELU_AUX_BIAS)",
-                "peak_kind": f"{pk['src']} bf16 sustained (kernel timed inside a long step)",
-                "frac_of_burst": round(achieved / pk["bf16_tflops"], 3)}
+                "launch": f"{DOMINANT} forward (M=N=K=4096, RELU_AUX_BIAS)", "us": round(fwd_ms * 1e3, 2),
+                "peak_kind": f"{pk['src']} bf16 burst (the launch is timed alone, after an L2 flush each time)",
+                "frac_of_sustained": round(achieved / pk["bf16_tflops_sustained"], 3),
+                "sm_mhz": roof_clk["sm_mhz"],
+                "us_x_ghz": (round(fwd_ms * 1e3 * roof_clk["sm_mhz"] / 1e3, 2) if roof_clk["sm_mhz"] else None)}
+    timed_clk = clk.summary("timed")
+    warm_clk = clk.summary("warm")
+    use = timed_clk if timed_clk["samples"] else warm_clk
+    clocks = {"sm_mhz": use["sm_mhz"], "sm_max_mhz": use["sm_max_mhz"] or warm_clk["sm_max_mhz"],
+              "reasons": sorted(set(timed_clk["reasons"]) | set(warm_clk["reasons"])),
+              "samples_timed": timed_clk["samples"], "samples_warm": warm_clk["samples"],
+              "sm_mhz_warm": warm_clk["sm_mhz"], "source": clk.source,
+              "window": "timed region, and the >= 1 s warm pass of the same replays just before it"}
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
@@ -385,11 +472,11 @@ def run_ours(args):
         "e2e": e2e,
         "gpu_launches": suite.launches_per_step() * args.steps,
         "roofline": roofline,
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "breakdown": breakdown,
-        "hbm_kernels": time_backward(fl, pk),
-        "gelu_sigmoid_1024x3072x768_bf16": time_gelu_sigmoid(fl, pk),
-        "fusion": time_fusion(suite, fl),
+        "hbm_kernels": hbm,
+        "gelu_sigmoid_1024x3072x768_bf16": sig,
+        "fusion": fusion,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
@@ -616,24 +703,29 @@ def time_fusion(suite, fl, reps=10):
     return out
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fl_gemm_epi_relu_aux_4096.json")
+
+
+def kernel_source_hash():
+    """First 16 hex digits of the SHA-256 of the fused kernel's source files."""
+    h = hashlib.sha256()
+    for f in ("fl_gemm.cuh", "fl_ptx.cuh"):
+        h.update(open(os.path.join(ROOT, "gemm_bias_activation_tcgen05_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
 def profiled_traffic():
-    """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
-    or None when the kernel source changed after the counters were taken."""
-    p = os.path.join(ROOT, "profiles", "fl_gemm_epi_relu_aux_4096.md")
-    if not os.path.exists(p):
-        return None
-    src = os.path.join(ROOT, "gemm_bias_activation_tcgen05_b200", "csrc", "fl_gemm.cuh")
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    vals = {}
-    for line in open(p):
-        if ":" in line and line.strip().startswith(("kernel_source_sha256_16", "dram_bytes_per_launch")):
-            k, v = line.split(":", 1)
-            vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel_source_sha256_16") != h:
+    """DRAM bytes (read + write) per launch of the dominant kernel from the committed ncu
+    record (profiles/fl_gemm_epi_relu_aux_4096.json), or None when the kernel source has
+    changed since the counters were taken."""
+    if not os.path.exists(TRAFFIC_FILE):
         return None
     try:
-        return float(vals["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
+        d = json.load(open(TRAFFIC_FILE))
+        if d.get("kernel_source_sha256_16") != kernel_source_hash():
+            return None
+        return float(d["dram_bytes_per_launch"])
+    except (OSError, ValueError, KeyError, TypeError):
         return None
 
 
@@ -705,9 +797,10 @@ def e2e_measure(suite, stream, sh, args, ws):
 _ORACLE_INPUTS = {}
 
 
-def _oracle_sample(seconds, rows_per_chunk=64):
+def _oracle_sample(seconds, rows_per_chunk=64, chunks=None):
     """Run the oracle (as it stands) over row-slices of every workload until about
-    `seconds` of CPU work is done; returns (flops, elapsed, cores, description)."""
+    `seconds` of CPU work is done (or exactly `chunks` chunks of rows);
+    returns (flops, elapsed, cores, description)."""
     import numpy as np
     import oracle
     import workloads
@@ -724,7 +817,9 @@ def _oracle_sample(seconds, rows_per_chunk=64):
             w = workloads.get(n)
             data[n] = (w, {k: v.double().numpy() for k, v in workloads.make_inputs(w, 0).items()})
     r0 = 0
-    while elapsed < seconds and r0 < 8192:
+    done = 0
+    while (elapsed < seconds if chunks is None else done < chunks) and r0 < 8192:
+        done += 1
         for n in names:
             w, inp = data[n]
             if r0 >= w.M:
@@ -754,10 +849,45 @@ def _oracle_sample(seconds, rows_per_chunk=64):
     return flops, elapsed, cores, desc
 
 
+def _oracle_pass(rows):
+    """One pass of the oracle over the row slices [0:rows) of every workload (inputs made
+    once, outside the timing); returns (flops, wall seconds)."""
+    f, t, _, _ = _oracle_sample(0.0, rows, chunks=1)
+    return f, t
+
+
 def cpu_baseline(seconds):
-    flops, elapsed, cores, desc = _oracle_sample(seconds)
-    return {"value": round(flops / elapsed / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": desc}
+    """The oracle as it stands on the host cores: the same sample (row slices [0:64) of every
+    workload, same seeded inputs) timed with all cores and with one thread, wall clock,
+    median of 3 runs each; plus a longer all-core sample of about `seconds`."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    rows = 64
+    _oracle_pass(rows)  # inputs generated and caches warm before the timed runs
+    runs_all = [_oracle_pass(rows) for _ in range(3)]
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            runs_one = [_oracle_pass(rows) for _ in range(3)]
+        one_threads = 1
+    except Exception:
+        runs_one, one_threads = [], None
+    flops = runs_all[0][0]
+    t_all = statistics.median(t for _, t in runs_all)
+    out = {"value": round(flops / t_all / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+           "sample": (f"oracle (numpy/scipy fp64) on row slices [0:{rows}) of every workload "
+                      f"({flops / 1e9:.2f} GFLOP), wall clock, median of 3 runs; all {cores} host cores "
+                      f"(nproc) for BLAS"),
+           "all_cores_s": round(t_all, 3)}
+    if runs_one:
+        t_one = statistics.median(t for _, t in runs_one)
+        out["single_thread"] = {"value": round(flops / t_one / 1e12, 6), "unit": "TFLOP/s", "threads": one_threads,
+                                "s": round(t_one, 3)}
+    f_long, t_long, _, desc = _oracle_sample(seconds)
+    out["long_sample"] = {"value": round(f_long / t_long / 1e12, 6), "sample": desc}
+    return out
 
 
 def run_reference(args):

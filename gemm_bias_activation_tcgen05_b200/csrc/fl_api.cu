@@ -817,8 +817,17 @@ static int resident_grid(const void* kernel, long long units, int num_sms) {
 
 template <int DT>
 static fl_status launch_ew_t(const EwParams& P, int num_sms, cudaStream_t s) {
-  const long long work = P.M * ((P.N + 31) / 32);
-  const cudaError_t err = launch_pdl(fl_ew_step_kernel<DT>, dim3((unsigned)grid_for(work, num_sms)), s, P);
+  constexpr int es = (DT == DT_F32) ? 4 : 2;
+  const bool vec = aligned16(P.src) && aligned16(P.dst) && (P.lds * es) % 16 == 0 && (P.ldd * es) % 16 == 0;
+  cudaError_t err;
+  if (vec) {
+    // one thread per 16-byte vector slot (rows padded to whole mask words)
+    const long long work = P.M * ((P.N + 31) / 32) * (32 / (16 / es));
+    err = launch_pdl(fl_ew_step_vec_kernel<DT>, dim3((unsigned)grid_for(work, num_sms)), s, P);
+  } else {
+    const long long work = P.M * ((P.N + 31) / 32);
+    err = launch_pdl(fl_ew_step_kernel<DT>, dim3((unsigned)grid_for(work, num_sms)), s, P);
+  }
   if (err != cudaSuccess) return fail(FL_ERR_CUDA, "elementwise kernel launch: %s", cudaGetErrorString(err));
   return after_launch(s, "elementwise step kernel");
 }

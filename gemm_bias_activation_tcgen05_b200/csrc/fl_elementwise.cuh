@@ -644,7 +644,153 @@ __device__ __forceinline__ void ew_st(void* p, long long i, float v) {
   store_elem<DT>(p, i, v);
 }
 
+// VE values of type dt from base[i0 ...] widened to fp32: 16- or 8-byte vector loads when
+// `vec` (the first element's address is aligned to the vector) and the vector is whole,
+// else element by element up to cnt (the rest 0).
+template <int VE>
+__device__ __forceinline__ void ew_ld_vals(float (&o)[VE], const void* base, long long i0, int dt, int cnt,
+                                           bool vec) {
+  if (vec && cnt == VE) {
+    if (dt == DT_F32) {
+      const float4* s = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + i0);
+#pragma unroll
+      for (int j = 0; j < VE / 4; ++j) {
+        const float4 f = __ldg(s + j);
+        o[4 * j] = f.x, o[4 * j + 1] = f.y, o[4 * j + 2] = f.z, o[4 * j + 3] = f.w;
+      }
+    } else {
+      uint32_t w[VE / 2];
+      const uint16_t* s = reinterpret_cast<const uint16_t*>(base) + i0;
+      if constexpr (VE == 8) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(s));
+        w[0] = q.x, w[1] = q.y, w[2] = q.z, w[3] = q.w;
+      } else {
+        const uint2 q = __ldg(reinterpret_cast<const uint2*>(s));
+        w[0] = q.x, w[1] = q.y;
+      }
+#pragma unroll
+      for (int j = 0; j < VE; ++j) {
+        const uint16_t h = (uint16_t)(w[j >> 1] >> (16 * (j & 1)));
+        o[j] = (dt == DT_BF16) ? __uint_as_float((uint32_t)h << 16) : __half2float(__ushort_as_half(h));
+      }
+    }
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < VE; ++j) {
+    o[j] = 0.0f;
+    if (j < cnt) o[j] = ldg_pinned(base, i0 + j, dt);
+  }
+}
+
+// One epilogue step over 16-byte vectors: thread i of the grid-stride sweep takes
+// vector v of row m, i = m·nvp + v, where a row has nvp = words·(32/VE) vector slots
+// (VE elements of DT per 16 bytes; the slots past N are idle).  Consecutive lanes read
+// and write consecutive 16 bytes of a row, and the 32/VE lanes of one mask word are
+// aligned lanes of one warp, so the word is formed by shuffles and stored by its first
+// lane.  Requires src and dst rows 16-byte aligned (base and pitch); the operands are
+// read by vectors when aligned, else element by element.  Every access is checked
+// against its buffer's element count (code 100 + op recorded, access skipped).
+template <int DT>
+__global__ void __launch_bounds__(256) fl_ew_step_vec_kernel(const EwParams P) {
+  grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
+  using T = typename ElemT<DT>::T;
+  constexpr int ES = sizeof(T);
+  constexpr int VE = 16 / ES;
+  constexpr int VPW = 32 / VE;  // vectors per 32-column mask word
+  const int lane = threadIdx.x & 31;
+  const long long words = (P.N + 31) / 32;
+  const long long nvp = words * VPW;
+  const long long total = P.M * nvp;
+  const int code = 100 + P.op;
+  const int oes = (P.operand_dtype == DT_F32) ? 4 : 2;
+  // operand vectors: the base aligned to the vector's bytes, and (for a matrix) the pitch too
+  const uint32_t ovec_bytes = (uint32_t)(VE * oes);
+  const uint32_t oalign = ovec_bytes >= 16 ? 16u : ovec_bytes;
+  const bool op_vec = P.operand != nullptr && (reinterpret_cast<uintptr_t>(P.operand) % oalign) == 0 &&
+                      ((P.op != EW_RESIDUAL && P.op != EW_GEGLU_MUL) || ((P.ldop * oes) % oalign) == 0);
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  // the trip count is warp-uniform (i - lane is the warp's first slot), so every lane of a
+  // warp runs the shuffles of a trip
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i - lane < total; i += stride) {
+    const bool live = i < total;
+    const long long m = live ? i / nvp : 0;
+    const long long v = live ? i - m * nvp : 0;
+    const long long n0 = v * VE;
+    const int cnt = live ? (int)max(0LL, min((long long)VE, P.N - n0)) : 0;
+    uint32_t bits = 0u;
+    if (cnt > 0) {
+      const long long is = m * P.lds + n0;
+      const long long id = m * P.ldd + n0;
+      bool ok = ew_in(is, P.src_elems, P.err, code) && ew_in(is + cnt - 1, P.src_elems, P.err, code) &&
+                ew_in(id, P.dst_elems, P.err, code) && ew_in(id + cnt - 1, P.dst_elems, P.err, code);
+      long long io = -1;
+      if (P.op == EW_BIAS_N) io = n0;
+      else if (P.op == EW_RESIDUAL || P.op == EW_GEGLU_MUL) io = m * P.ldop + n0;
+      if (ok && io >= 0)
+        ok = ew_in(io, P.op_elems, P.err, code) && ew_in(io + cnt - 1, P.op_elems, P.err, code);
+      if (ok && P.op == EW_BIAS_M) ok = ew_in(m, P.op_elems, P.err, code);
+      if (ok) {
+        float x[VE], opv[VE], y[VE];
+        ew_ld_vals<VE>(x, P.src, is, DT, cnt, true);
+        if (io >= 0) {
+          ew_ld_vals<VE>(opv, P.operand, io, P.operand_dtype, cnt, op_vec);
+        } else if (P.op == EW_BIAS_M) {
+          const float b = ldg_pinned(P.operand, m, P.operand_dtype);
+#pragma unroll
+          for (int j = 0; j < VE; ++j) opv[j] = b;
+        } else {
+#pragma unroll
+          for (int j = 0; j < VE; ++j) opv[j] = 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < VE; ++j) {
+          switch (P.op) {
+            case EW_BIAS_N:
+            case EW_BIAS_M:
+            case EW_RESIDUAL: y[j] = x[j] + opv[j]; break;
+            case EW_RELU:
+              y[j] = fmaxf(x[j], 0.0f);
+              if (x[j] > 0.0f && j < cnt) bits |= 1u << j;
+              break;
+            case EW_GELU: y[j] = gelu_erf_f(x[j]); break;
+            case EW_GELU_TANH: y[j] = gelu_tanh_f<DT != DT_F32>(x[j]); break;
+            case EW_GELU_SIGMOID: y[j] = gelu_sigmoid_f(x[j]); break;
+            case EW_SCALE: y[j] = x[j] * P.scale; break;
+            default: y[j] = gelu_tanh_f<DT != DT_F32>(x[j]) * opv[j]; break;
+          }
+        }
+        if (cnt == VE) {
+          uint32_t w[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            if constexpr (DT == DT_F32) w[k] = __float_as_uint(y[k]);
+            else w[k] = pack2<DT>(y[2 * k], y[2 * k + 1]);
+          }
+          *reinterpret_cast<uint4*>(reinterpret_cast<T*>(P.dst) + id) = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < VE; ++j)
+            if (j < cnt) store_elem<DT>(P.dst, id + j, y[j]);
+        }
+      }
+    }
+    if (P.op == EW_RELU && P.aux != nullptr) {
+      // the word's VPW lanes are aligned within the warp (nvp and 32 are multiples of VPW)
+      uint32_t word = bits << ((int)(v % VPW) * VE);
+#pragma unroll
+      for (int o = 1; o < VPW; o <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
+      if (live && (v % VPW) == 0) {
+        const long long ia = m * P.ld_aux + v / VPW;
+        if (ew_in(ia, P.aux_elems, P.err, code)) P.aux[ia] = word;
+      }
+    }
+  }
+}
+
 // Storage dtype DT for src/dst (the eager tensors); operands use their own dtype.
+// Element-by-element form, for rows that are not 16-byte aligned.
 template <int DT>
 __global__ void __launch_bounds__(256) fl_ew_step_kernel(const EwParams P) {
   grid_dependency_wait();

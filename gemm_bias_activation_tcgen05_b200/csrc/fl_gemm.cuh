@@ -32,6 +32,14 @@
 
 #include "fl_ptx.cuh"
 
+// Phase-trace points (a device timestamp per CTA and slot).  Empty unless a trace
+// build defines FL_STAMP before including this file.
+#ifndef FL_STAMP
+#define FL_STAMP(slot) \
+  do {                 \
+  } while (0)
+#endif
+
 namespace fl {
 
 enum Act : int { ACT_NONE = 0, ACT_RELU = 1, ACT_GELU = 2, ACT_GELU_TANH = 3, ACT_GEGLU = 4, ACT_GELU_SIGMOID = 5 };
@@ -434,6 +442,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
   const bool have_acc = kb_end > kb_begin;
 
   if (threadIdx.x == 0) {
+    FL_STAMP(0);
     for (int s = 0; s < NS; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
@@ -471,10 +480,14 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (S > 1 || PAIR) cluster_sync_all();  // peers' barriers are initialised before any remote arrive
+  if (threadIdx.x == 0) FL_STAMP(1);
   // Programmatic dependent launch: the prologue above may overlap the previous
   // kernel of the stream; no global memory is touched before this wait.
   grid_dependency_wait();
-  if (threadIdx.x == 0) grid_launch_dependents();
+  if (threadIdx.x == 0) {
+    FL_STAMP(2);
+    grid_launch_dependents();
+  }
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(
       __cvta_shared_to_generic(tmem_slot));
 
@@ -494,6 +507,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           const int s = (int)(it % (uint32_t)NS);
           const uint32_t ph = (it / (uint32_t)NS) & 1u;
           if (!wait_bounded(empty_bar(s), ph ^ 1u, p)) { ok = false; break; }
+          if (it == 0) FL_STAMP(3);
           const uint32_t sa = smem_base + (uint32_t)s * p.stage_stride;
           const uint32_t sb = sa + p.a_stage_bytes;
           const int k0 = kb * p.bk;
@@ -577,6 +591,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           const uint32_t ph = (it / (uint32_t)NS) & 1u;
           if (!wait_bounded(TF32 ? conv_bar(s) : full_bar(s), ph, p, TF32 && PAIR)) { ok = false; break; }
           tc_fence_after();
+          if (it == 0) FL_STAMP(4);
           const uint64_t da = da0 + (uint64_t)s * stage_step;
           const uint64_t db = db0 + (uint64_t)s * stage_step;
           if constexpr (TF32) {
@@ -614,6 +629,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           issued = true;
         }
         if (!ok) break;
+        if (local == 0) FL_STAMP(5);
         if constexpr (PAIR) {
           if (have_acc) {
             umma_commit_pair(tfull_bar(buf));
@@ -698,6 +714,10 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         if (has_bias && p.bias_axis == 1 && m_ok) bias_m = ldg_pinned(p.bias, m, p.bias_dtype);
         if (!warp_wait_bounded(tfull_bar(buf), tph, p, lane, PAIR)) { ok = false; break; }
         tc_fence_after();
+        if (ew == 0 && lane == 0) {
+          if (local == 0) FL_STAMP(6);
+          FL_STAMP(8);
+        }
         const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
         const int c_begin = half * half_cols;
         const int c_end = c_begin + half_cols;
@@ -830,7 +850,9 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
             bulk_commit_group();
           }
         }
+        if (ew == 0 && lane == 0 && local == 0) FL_STAMP(7);
       }
+      if (ew == 0 && lane == 0) FL_STAMP(9);
       if (lane == 0) bulk_wait_group<0>();
     } else {
       // ---------------- swap-AB layout: TMEM lane = output column n, TMEM column = output row m.
@@ -870,6 +892,10 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         if (res_async && rows > 0) stage_residual(p, rst, m_lo, min(32, rows), n_w0, lane);
         if (!warp_wait_bounded(tfull_bar(buf), tph, p, lane)) { ok = false; break; }
         tc_fence_after();
+        if (ew == 0 && lane == 0) {
+          if (local == 0) FL_STAMP(6);
+          FL_STAMP(8);
+        }
         const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
 
         if (S > 1) {
@@ -903,6 +929,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
             for (int rk = 0; rk < S; ++rk) mbar_arrive_remote(mapa_shared(red_ready_bar, (uint32_t)rk));
           }
           if (!warp_wait_bounded(red_ready_bar, 0, p, lane, true)) ok = false;
+          if (ew == 0 && lane == 0) FL_STAMP(12);
           // Every CTA has published and its stages are dead: push slice k of this CTA's
           // partial (rows [k·L, k·L + L), contiguous) into CTA k's receive slot for this
           // rank, with the copy engine.
@@ -918,6 +945,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           // (waited even after a failed wait above: a peer that got through may be
           // writing into this CTA, which must not leave before the bytes land)
           if (!warp_wait_bounded(recv_bar, 0, p, lane, true)) ok = false;
+          if (ew == 0 && lane == 0) FL_STAMP(13);
           // tell the sources their copies have landed (they stay resident until then)
           if (ok && ew == 0 && lane == 0)
             for (int k = 0; k < S; ++k)
@@ -951,6 +979,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
             }
             // every warp's sums are in place before any warp finishes rows
             asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
+            if (ew == 0 && lane == 0) FL_STAMP(14);
           }
         }
 
@@ -1047,6 +1076,10 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
             __syncwarp();  // the block's buffer is refilled two blocks later
           }
         }
+        if (ew == 0 && lane == 0) {
+          if (local == 0) FL_STAMP(7);
+          FL_STAMP(9);
+        }
         if (S == 1) {
           // this warp's TMEM reads of the buffer are done
           tc_fence_before();
@@ -1067,13 +1100,18 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
   // ================================================================ teardown
   // Every thread of every role arrives here converged, after its last TMEM
   // read, MMA (drained) and copy; only then is TMEM released.
+  if (threadIdx.x == 0) FL_STAMP(10);
   __syncthreads();
-  // a pair stays resident until neither CTA can touch the other's barriers or TMEM
-  if (PAIR) cluster_sync_all();
+  // A cluster (CTA pair or split-K group) stays resident until no CTA can still touch
+  // another's barriers, shared memory or TMEM: after a bounded wait gave up in one CTA,
+  // a peer that got through may still arrive on its barriers or copy into it.  Every
+  // wait before this point is bounded, so every CTA of the cluster reaches it.
+  if (S > 1 || PAIR) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
     if constexpr (PAIR) tmem_dealloc_pair(tmem_base, p.tmem_cols);
     else tmem_dealloc(tmem_base, p.tmem_cols);
+    if (lane == 0) FL_STAMP(11);
   }
 }
 

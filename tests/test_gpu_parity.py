@@ -137,6 +137,37 @@ def test_unfused_residual_f32(fl):
                  unfused=True)
 
 
+@pytest.mark.parametrize("M,out_dtype", [(5, "f32"), (77, "f32"), (128, "f32"), (40, "bf16")])
+def test_unfused_twin_small_m(fl, M, out_dtype):
+    # M <= 128: the twin's bare GEMM takes the swap-AB layout with split-K, then the
+    # bias, GELU, residual and scale steps run as separate kernels
+    got = _linear_case(fl, M, 1000, 1000, epilogue="GELU_BIAS", out_dtype=out_dtype, residual=True, scale=0.5,
+                       unfused=True, seed=40 + M)
+    assert got["info"]["launches_per_execute"] == 5
+
+
+@pytest.mark.parametrize("M,N,K", [(200, 300, 136), (77, 264, 200), (257, 136, 768)])
+def test_unfused_twin_geglu(fl, M, N, K):
+    # the twin of GEGLU_TANH: the bare dual GEMM writes [g | u] ([M, 2N]) to an
+    # intermediate in the output type, then one kernel forms gelu_tanh(g)·u
+    inp = workloads.ragged_linear_inputs(M, N, K, "bf16", 9, dual=True)
+    A, W = inp["A"], inp["W"]
+    got = P.run_linear(fl, M=M, N=N, K=K, dtype="bf16", epilogue="GEGLU_TANH", out_dtype="bf16", A=A, W=W,
+                       unfused=True)
+    assert got["info"]["launches_per_execute"] == 2
+    a = P.to64(A)[:, :K]
+    w = P.to64(W)
+    Wg, Wu = w[:N, :K], w[N:2 * N, :K]
+    h = oracle.geglu_h(a, Wg, Wu, "bf16")
+    g = oracle.gemm(a, Wg)
+    u = oracle.gemm(a, Wu)
+    absdot = float((oracle.gemm(np.abs(a), np.abs(Wg)) * np.abs(u) * 1.2
+                    + oracle.gemm(np.abs(a), np.abs(Wu)) * np.abs(oracle.gelu_tanh(g))).max())
+    # g and u pass through the bf16 intermediate: one more rounding of each (2^-9 relative)
+    absdot += float((np.abs(g) * np.abs(u)).max()) * 2.0 ** -8 * 2 ** 14
+    P.check_close(got["out"], h, "bf16", absdot, f"geglu twin {M}x{N}x{K} {got['info']}")
+
+
 @pytest.mark.parametrize("M,N,dtype", [(64, 4096, "bf16"), (33, 1000, "bf16"), (7, 77, "f32"), (5, 40, "f16")])
 def test_relu_backward(fl, M, N, dtype):
     g = torch.Generator().manual_seed(M * N)

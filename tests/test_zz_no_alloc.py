@@ -5,7 +5,8 @@ own pool owns all device memory, or a latency-critical path where allocation
 and its possible device synchronisation are forbidden).  Its scratch lives in
 a fixed device array inside the library and is shared by every call, so this
 file makes two calls in a row on the same array and compares both with
-fl_plan/fl_execute on the same inputs, within the parity tests' tolerance.
+fl_plan/fl_execute on the same inputs and with the oracle, within the parity
+tests' tolerance (the ReLU mask bit-exact where the pre-activation is decided).
 It is collected last and runs alone or after the other tests.
 """
 from __future__ import annotations
@@ -71,14 +72,19 @@ def _run(fl, noalloc, M, N, K, kind, out_dtype, residual, unfused, seed):
 def test_noalloc_matches_planned_entry_point_twice(fl, case):
     M, N, K, kind, out_dtype, residual, unfused = case
     inp, ref, ref_aux = _run(fl, False, *case, seed=31)
-    _, _, _, absdot = P.oracle_linear(A=inp["A"], W=inp["W"], bias=inp["bias"], residual=inp.get("residual"),
+    y, _, v, absdot = P.oracle_linear(A=inp["A"], W=inp["W"], bias=inp["bias"], residual=inp.get("residual"),
                                       scale=0.5 if residual else 1.0, epilogue=kind, out_dtype=out_dtype,
                                       M=M, N=N, K=K)
+    # the unfused path rounds acc = A·Wᵀ to the output type before its bias step
+    acc = v - P.to64(inp["bias"])[None, :]
+    margin = P.ULP_REL[out_dtype] * (np.abs(acc) + np.abs(v)) if unfused else None
     for call in range(2):  # the second call finds the first call's scratch contents
         _, got, got_aux = _run(fl, True, *case, seed=31)
-        P.check_close(got, ref, out_dtype, absdot, f"noalloc call {call} {kind}")
+        P.check_close(got, ref, out_dtype, absdot, f"noalloc call {call} {kind} vs fl_execute")
+        P.check_close(got, y, out_dtype, absdot, f"noalloc call {call} {kind} vs oracle")
         if ref_aux is not None:
             assert np.array_equal(got_aux, ref_aux)
+            P.check_mask(got_aux, v, N, f"noalloc call {call} mask vs oracle", margin)
 
 
 def test_noalloc_rejects_oversized_scratch(fl):
