@@ -508,20 +508,39 @@ class L2Flush:
         self.r.sum()
 
 
-def time_single_launch(suite, it, stream, sh, reps):
+def time_in_graph(fn, reps, flush=None):
+    """Mean CUDA-event time (ms) of fn(), each launch preceded by an L2 flush (outside the
+    event pair).  The whole sequence (flush, event, fn, event) x reps is captured once as a
+    CUDA graph and replayed, so the GPU never waits for the host inside an event pair (timed
+    one launch at a time from Python, a short kernel's events would also hold the host's
+    enqueue latency).  fn must launch on the current stream."""
     import torch
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-    w, d = it["w"], it["dev"]
-    # flush L2 between launches (outside the event pair)
-    flush = L2Flush()
-    for a, b in evs:
-        flush()
-        a.record(stream)
-        it["plans"][0].execute(d["A"], d["W"], d.get("bias"), it["aux"], d.get("residual"), it["out"], stream=sh)
-        b.record(stream)
+    fn()
     torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True, external=True),
+            torch.cuda.Event(enable_timing=True, external=True)) for _ in range(reps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for a, b in evs:
+            if flush is not None:
+                flush()
+            a.record()
+            fn()
+            b.record()
+    g.replay()
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / reps
+    del g
+    return ms
+
+
+def time_single_launch(suite, it, stream, sh, reps):
+    d = it["dev"]
+    flush = L2Flush()
+    ms = time_in_graph(lambda: it["plans"][0].execute(d["A"], d["W"], d.get("bias"), it["aux"], d.get("residual"),
+                                                      it["out"], stream=None), reps, flush)
     del flush
-    return sum(a.elapsed_time(b) for a, b in evs) / reps
+    return ms
 
 
 def hbm_runs(fl, sh):
@@ -573,20 +592,11 @@ def time_backward(fl, pk, reps=10):
     the algorithmic bytes, and the fraction of the measured HBM copy bandwidth."""
     import torch
     sh = torch.cuda.current_stream().cuda_stream
-    runs = hbm_runs(fl, sh)
+    runs = hbm_runs(fl, None)
     flush = L2Flush()
     out = {}
     for name, (fn, algo_bytes) in runs.items():
-        fn()
-        torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-        for a, b in evs:
-            flush()
-            a.record()
-            fn()
-            b.record()
-        torch.cuda.synchronize()
-        ms = sum(a.elapsed_time(b) for a, b in evs) / reps
+        ms = time_in_graph(fn, reps, flush)
         gbs = algo_bytes / (ms * 1e-3) / 1e9
         out[name] = {"us": round(ms * 1e3, 2), "algorithmic_bytes": algo_bytes, "gbs": round(gbs, 1),
                      "frac_of_hbm": round(gbs / pk["hbm_gbs"], 3)}
@@ -606,19 +616,10 @@ def time_gelu_sigmoid(fl, pk, reps=10):
     plan = fl.Plan(M, N, K, kind="GELU_SIGMOID_BIAS", out_dtype="bf16")
     flush = L2Flush()
     try:
-        plan.execute(A, W, b, out=out)
-        torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-        for a, e in evs:
-            flush()
-            a.record()
-            plan.execute(A, W, b, out=out)
-            e.record()
-        torch.cuda.synchronize()
+        ms = time_in_graph(lambda: plan.execute(A, W, b, out=out), reps, flush)
         assert plan.check() == fl.FL_OK
     finally:
         plan.free()
-    ms = sum(a.elapsed_time(e) for a, e in evs) / reps
     tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
     return {"us": round(ms * 1e3, 2), "tflops": round(tf, 1), "frac_of_bf16_burst": round(tf / pk["bf16_tflops"], 3)}
 
@@ -627,18 +628,8 @@ FUSION_SET = ["linear_gelu_tanh_bf16_1024x3072x768", "geglu_mlp_8192x3072x768", 
 
 
 def _time_launch(fn, flush, reps):
-    """Mean CUDA-event time (ms) of fn() on the current stream, each launch after an L2 flush."""
-    import torch
-    fn()
-    torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-    for a, b in evs:
-        flush()
-        a.record()
-        fn()
-        b.record()
-    torch.cuda.synchronize()
-    return sum(a.elapsed_time(b) for a, b in evs) / reps
+    """Mean CUDA-event time (ms) of fn(), each launch after an L2 flush (time_in_graph)."""
+    return time_in_graph(fn, reps, flush)
 
 
 def time_fusion(suite, fl, reps=10):
@@ -650,7 +641,7 @@ def time_fusion(suite, fl, reps=10):
     GEMM either way).  A workload whose measurement fails records the error instead."""
     import torch
     flush = L2Flush()
-    sh = torch.cuda.current_stream().cuda_stream
+    sh = None  # the current stream at launch time (the capture stream inside a graph)
     out = {}
     for it in suite.items:
         w = it["w"]

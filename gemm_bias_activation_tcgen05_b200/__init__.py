@@ -33,6 +33,7 @@ EPILOGUES = {"NONE": 0, "BIAS": 1, "RELU_BIAS": 2, "RELU_AUX_BIAS": 3, "GELU_BIA
              "GELU_SIGMOID_BIAS": 8}
 DTYPES = {"f16": FL_F16, "bf16": FL_BF16, "f32": FL_F32}
 COMPUTES = {"32F": FL_COMPUTE_32F, "32F_3XTF32": FL_COMPUTE_32F_3XTF32}
+SCHEDULES = {"auto": 0, "data_parallel": 1, "stream_k": 2}
 
 EXPORTED = ["fl_plan", "fl_execute", "fl_relu_backward", "fl_check_status", "fl_get_plan_info",
             "fl_free", "fl_last_error", "fl_set_wait_limit_ns", "fl_execute_noalloc",
@@ -45,7 +46,8 @@ class fl_epilogue_desc(ctypes.Structure):
                 ("residual_dtype", ctypes.c_int32), ("bias_axis", ctypes.c_int32),
                 ("has_residual", ctypes.c_int32), ("scale", ctypes.c_float), ("b_major", ctypes.c_int32),
                 ("lda", ctypes.c_int64), ("ldb", ctypes.c_int64), ("ldo", ctypes.c_int64),
-                ("ldr", ctypes.c_int64), ("unfused", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+                ("ldr", ctypes.c_int64), ("unfused", ctypes.c_int32), ("schedule", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 2)]
 
 
 class fl_plan_info(ctypes.Structure):
@@ -53,7 +55,8 @@ class fl_plan_info(ctypes.Structure):
                 ("swap_ab", ctypes.c_int32), ("split_k", ctypes.c_int32), ("stages", ctypes.c_int32),
                 ("grid", ctypes.c_int32), ("smem_bytes", ctypes.c_int32),
                 ("launches_per_execute", ctypes.c_int32), ("cta_pair", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 6)]
+                ("stream_k_tiles", ctypes.c_int32), ("stream_k_pairs", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 4)]
 
 
 def _load() -> ctypes.CDLL:
@@ -143,7 +146,7 @@ def fl_set_wait_limit_ns(ns: int) -> None:
 def make_epilogue(kind: str = "NONE", out_dtype: str = "bf16", bias_dtype: str = "bf16",
                   residual_dtype: str = "bf16", bias_axis: int = 0, has_residual: bool = False,
                   scale: float = 1.0, b_major: int = 0, lda: int = 0, ldb: int = 0, ldo: int = 0,
-                  ldr: int = 0, unfused: bool = False) -> fl_epilogue_desc:
+                  ldr: int = 0, unfused: bool = False, schedule: str = "auto") -> fl_epilogue_desc:
     e = fl_epilogue_desc()
     e.kind = EPILOGUES[kind]
     e.out_dtype = DTYPES[out_dtype]
@@ -155,6 +158,7 @@ def make_epilogue(kind: str = "NONE", out_dtype: str = "bf16", bias_dtype: str =
     e.b_major = int(b_major)
     e.lda, e.ldb, e.ldo, e.ldr = int(lda), int(ldb), int(ldo), int(ldr)
     e.unfused = int(bool(unfused))
+    e.schedule = SCHEDULES[schedule]
     return e
 
 

@@ -205,6 +205,13 @@ struct fl_plan_s {
   int k_atoms;  // 128-byte K atoms per pipeline stage
   int mma_n, out_tile_n, split_k, stages, grid, smem;
   int tiles_a, tiles_b, num_kb;
+  // stream-K (16-bit CTA pairs): the last sk_tiles tiles are split along K over
+  // sk_clusters pairs; no_sk keeps the data-parallel schedule
+  bool no_sk;
+  int sk_tiles, sk_clusters;
+  float* d_skws;  // partial accumulators, sk_ws_bytes()
+  int* d_skflags;
+  size_t skws_bytes, skflags_bytes;
   const void* kernel;
   int* d_err;
   // unfused twin
@@ -298,6 +305,8 @@ static int b_boxes_of(const fl_plan_s* p, bool geglu) {
 static int grid_of(const fl_plan_s* p) {
   const int tiles = p->tiles_a * p->tiles_b;
   if (p->swap && p->split_k > 1) return tiles * p->split_k;
+  // stream-K: every pair takes the same share of the full rounds and a range of the rest
+  if (p->pair && p->sk_tiles > 0) return 2 * (p->num_sms / 2);
   if (p->pair) return 2 * std::min(tiles, p->num_sms / 2);
   return std::min(tiles, p->num_sms);
 }
@@ -305,6 +314,37 @@ static const void* kernel_of(const fl_plan_s* p, int act, int out) {
   if (p->dtype == FL_F32) return p->pair ? pick_kernel_tf32_pair(act, out) : pick_kernel_tf32(act, out);
   if (p->pair) return pick_kernel_pair(act, out);
   return pick_kernel(act, out, p->swap);
+}
+
+// Stream-K for 16-bit CTA pairs.  Data-parallel, T tiles take ⌈T/P⌉ rounds of the P pairs;
+// stream-K spreads the tiles of the last, partial round over every pair, as contiguous
+// ranges of (tile, K-block) units, at the price of a fix-up per cut tile (a 128 KB partial
+// accumulator per CTA stored, then read and added by the tile's finisher, before its
+// epilogue).  A pair saves (⌈T/P⌉ − T/P)·num_kb K blocks; FL_SCHED_AUTO takes stream-K when
+// that is at least kSkMinSavedBlocks, a few times the fix-up's cost in K blocks.
+constexpr double kSkMinSavedBlocks = 8.0;
+
+static bool stream_k_pays(int64_t T, int64_t P, int num_kb, int schedule) {
+  if (schedule == FL_SCHED_DATA_PARALLEL || num_kb < 2 || T % P == 0) return false;
+  if (schedule == FL_SCHED_STREAM_K) return true;
+  const double saved = ((double)cdiv(T, P) - (double)T / (double)P) * num_kb;
+  return saved >= kSkMinSavedBlocks;
+}
+
+// The stream-K split of the chosen configuration: the last partial round of tiles (all
+// tiles when there are fewer than pairs), plus one full round when that leaves the pairs
+// fewer than four K blocks each, over min(P, units) pairs.
+static void choose_stream_k(fl_plan_s* p) {
+  p->sk_tiles = 0;
+  p->sk_clusters = 0;
+  if (!p->pair || p->no_sk || p->dtype == FL_F32) return;
+  const int64_t P = p->num_sms / 2;
+  const int64_t T = (int64_t)p->tiles_a * p->tiles_b;
+  if (!stream_k_pays(T, P, p->num_kb, p->epi.schedule)) return;
+  int64_t sk = T % P;
+  if (T > P && sk * p->num_kb < 4 * P) sk += P;
+  p->sk_tiles = (int)sk;
+  p->sk_clusters = (int)std::min<int64_t>(P, sk * p->num_kb);
 }
 
 static fl_status choose_config(fl_plan_s* p) {
@@ -364,11 +404,15 @@ static fl_status choose_config(fl_plan_s* p) {
       // Cost ~ (rounds of tiles per SM) x (tile width) x (relative cost per column):
       // a 128-wide UMMA tile moves more operand bytes per FLOP and issues twice
       // the instructions, measured at about 1.6x the per-column cost of 256.
+      // With stream-K (CTA pairs) the rounds are fractional: the last, partial round is
+      // spread over every pair.
+      const bool sk_ok = p->pair && !p->no_sk;
       int best = 256;
       double best_cost = 1e300;
       for (int bn : {256, 128}) {
         const int64_t tiles = cdiv(M, rows) * cdiv(N, bn);
-        const double waves = (double)cdiv(tiles, units);
+        const bool sk = sk_ok && stream_k_pays(tiles, units, p->num_kb, p->epi.schedule);
+        const double waves = sk ? (double)tiles / units : (double)cdiv(tiles, units);
         const double cost = waves * bn * (bn == 128 ? 1.6 : 1.0);
         if (cost < best_cost) { best_cost = cost; best = bn; }
       }
@@ -377,8 +421,34 @@ static fl_status choose_config(fl_plan_s* p) {
     }
     p->tiles_a = (int)cdiv(M, rows);
     p->tiles_b = (int)cdiv(N, p->out_tile_n);
+    choose_stream_k(p);
   }
   return FL_OK;
+}
+
+// Stream-K workspace of a configuration: one fp32 partial accumulator per CTA and epilogue
+// warp (mma_n/2 columns x 32 rows), and one flag per CTA and epilogue warp.
+static void sk_sizes(const fl_plan_s* p, size_t* ws, size_t* flags) {
+  *ws = *flags = 0;
+  if (p->sk_tiles <= 0) return;
+  *ws = (size_t)p->grid * 8u * (size_t)(p->mma_n / 2) * 32u * sizeof(float);
+  *flags = (size_t)p->grid * 8u * sizeof(int);
+}
+
+// Configuration of the unfused twin's bare GEMM: the same operands with epilogue NONE,
+// writing the [M, N] (GeGLU: [M, 2N]) intermediate.
+static void twin_config(const fl_plan_s* p, fl_plan_s* q) {
+  *q = *p;
+  q->epi.kind = FL_EPI_NONE;
+  q->epi.ldr = 0;
+  q->epi.has_residual = 0;
+  q->N = (p->epi.kind == FL_EPI_GEGLU_TANH) ? 2 * p->N : p->N;
+  choose_config(q);
+  const int b_boxes = b_boxes_of(q, false);
+  Layout L = layout_for(q, q->mma_n, b_boxes, q->max_smem);
+  q->stages = L.stages;
+  q->smem = (int)L.total;
+  q->grid = grid_of(q);
 }
 
 // Launches of one unfused execute: the bare GEMM, then one elementwise kernel per step.
@@ -402,8 +472,10 @@ static fl_status plan_host_part(fl_plan_s** out, int64_t M, int64_t N, int64_t K
     return fail(FL_ERR_INVALID_ARG, "fl_plan: dimension too large");
   if (epi->kind < FL_EPI_NONE || epi->kind > FL_EPI_GELU_SIGMOID_BIAS)
     return fail(FL_ERR_INVALID_ARG, "fl_plan: unknown epilogue kind %d", epi->kind);
-  for (int i = 0; i < 3; ++i)
+  for (int i = 0; i < 2; ++i)
     if (epi->reserved[i] != 0) return fail(FL_ERR_INVALID_ARG, "fl_plan: reserved fields must be 0");
+  if (epi->schedule < FL_SCHED_AUTO || epi->schedule > FL_SCHED_STREAM_K)
+    return fail(FL_ERR_INVALID_ARG, "fl_plan: unknown schedule %d", epi->schedule);
   if (dtype != FL_F16 && dtype != FL_BF16 && dtype != FL_F32)
     return fail(FL_ERR_INVALID_ARG, "fl_plan: unknown dtype %d", dtype);
   if (compute != FL_COMPUTE_32F && compute != FL_COMPUTE_32F_3XTF32)
@@ -510,6 +582,32 @@ extern "C" fl_status fl_plan(fl_plan_t* out, int64_t M, int64_t N, int64_t K, in
   }
   p->launches = 1;
   p->wait_limit_ns = g_wait_limit_ns;
+  {
+    // stream-K workspace: for this plan's kernel, and for the unfused twin's bare GEMM
+    size_t ws = 0, fb = 0;
+    sk_sizes(p, &ws, &fb);
+    if (epi->unfused) {
+      fl_plan_s q;
+      twin_config(p, &q);
+      size_t ws2 = 0, fb2 = 0;
+      sk_sizes(&q, &ws2, &fb2);
+      ws = std::max(ws, ws2);
+      fb = std::max(fb, fb2);
+    }
+    if (ws > 0) {
+      if (cudaMalloc(&p->d_skws, ws) != cudaSuccess || cudaMalloc(&p->d_skflags, fb) != cudaSuccess) {
+        (void)cudaGetLastError();
+        fl_free(p);
+        return fail(FL_ERR_OOM, "fl_plan: cudaMalloc(stream-K workspace, %zu bytes)", ws + fb);
+      }
+      if (cudaMemset(p->d_skflags, 0, fb) != cudaSuccess) {
+        fl_free(p);
+        return fail(FL_ERR_CUDA, "fl_plan: cudaMemset(stream-K flags)");
+      }
+      p->skws_bytes = ws;
+      p->skflags_bytes = fb;
+    }
+  }
   if (epi->unfused) {
     // the bare GEMM kernels of both layouts may serve this plan's first step
     for (int sw = 0; sw < 3; ++sw) {
@@ -589,6 +687,8 @@ extern "C" fl_status fl_get_plan_info(fl_plan_t p, fl_plan_info* info) {
   info->smem_bytes = p->smem;
   info->launches_per_execute = p->launches;
   info->cta_pair = p->pair ? 1 : 0;
+  info->stream_k_tiles = p->sk_tiles;
+  info->stream_k_pairs = p->sk_clusters;
   return FL_OK;
 }
 
@@ -596,6 +696,8 @@ extern "C" fl_status fl_free(fl_plan_t p) {
   if (!p) return FL_OK;
   if (p->d_err) cudaFree(p->d_err);
   if (p->d_tmp) cudaFree(p->d_tmp);
+  if (p->d_skws) cudaFree(p->d_skws);
+  if (p->d_skflags) cudaFree(p->d_skflags);
   delete p;
   return FL_OK;
 }
@@ -732,6 +834,10 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
   k.scale = g.scale;
   k.err = p->d_err;
   k.wait_limit_ns = p->wait_limit_ns;
+  k.sk_tiles = p->sk_tiles;
+  k.sk_clusters = p->sk_clusters;
+  k.sk_ws = p->d_skws;
+  k.sk_flags = p->d_skflags;
 
   CUtensorMap tmA, tmB, tmB2, tmOut;
   const int ae = 128 / es;  // K elements of one 128-byte swizzle atom: the inner box of K-major maps
@@ -878,19 +984,8 @@ extern "C" fl_status fl_execute(fl_plan_t p, const void* A, const void* W, const
   const int64_t gemm_ld = no_steps ? e.ldo : p->tmp_ld;
   {
     // The unfused GEMM uses the same tcgen05 kernel with no epilogue work.
-    fl_plan_s q = *p;
-    q.epi.kind = FL_EPI_NONE;
-    q.epi.ldr = 0;
-    q.epi.has_residual = 0;
-    q.N = cols;
-    choose_config(&q);
-    const int b_boxes = b_boxes_of(&q, false);
-    Layout L = layout_for(&q, q.mma_n, b_boxes, q.max_smem);
-    q.stages = L.stages;
-    q.smem = (int)L.total;
-    const int tiles = q.tiles_a * q.tiles_b;
-    (void)tiles;
-    q.grid = grid_of(&q);
+    fl_plan_s q;
+    twin_config(p, &q);
     const void* kern = kernel_of(&q, ACT_NONE, odt);
     q.epi.ldr = 0;
     q.epi.has_residual = 0;
@@ -1233,6 +1328,8 @@ extern "C" fl_status fl_check_status(fl_plan_t p, void* stream_) {
   FL_CUDA(cudaMemcpy(&h, p->d_err, sizeof(int), cudaMemcpyDeviceToHost));
   if (h != 0) {
     FL_CUDA(cudaMemset(p->d_err, 0, sizeof(int)));
+    // a launch that gave up may have left stream-K flags set: clear them for the next one
+    if (p->d_skflags) FL_CUDA(cudaMemset(p->d_skflags, 0, p->skflags_bytes));
     if (h >= 100)
       return fail(FL_ERR_DEVICE, "an elementwise kernel skipped an out-of-range access (code %d)", h);
     return fail(FL_ERR_TIMEOUT, "a bounded in-kernel wait gave up (code %d)", h);
@@ -1286,8 +1383,10 @@ extern "C" fl_status fl_execute_noalloc(int64_t M, int64_t N, int64_t K, int32_t
     return fail(FL_ERR_INVALID_ARG, "%s: dimension too large", who);
   if (epi->kind < FL_EPI_NONE || epi->kind > FL_EPI_GELU_SIGMOID_BIAS)
     return fail(FL_ERR_INVALID_ARG, "%s: unknown epilogue kind %d", who, epi->kind);
-  for (int i = 0; i < 3; ++i)
+  for (int i = 0; i < 2; ++i)
     if (epi->reserved[i] != 0) return fail(FL_ERR_INVALID_ARG, "%s: reserved fields must be 0", who);
+  if (epi->schedule < FL_SCHED_AUTO || epi->schedule > FL_SCHED_STREAM_K)
+    return fail(FL_ERR_INVALID_ARG, "%s: unknown schedule %d", who, epi->schedule);
   if (dtype != FL_F16 && dtype != FL_BF16) {
     if (dtype == FL_F32) return fail(FL_ERR_UNSUPPORTED, "%s: fp32 operands are not offered", who);
     return fail(FL_ERR_INVALID_ARG, "%s: unknown dtype %d", who, dtype);
@@ -1313,6 +1412,7 @@ extern "C" fl_status fl_execute_noalloc(int64_t M, int64_t N, int64_t K, int32_t
   // scratch points into the fixed array instead of fresh allocations.
   fl_plan_s p{};
   p.M = M; p.N = N; p.K = K; p.dtype = dtype; p.compute = compute; p.epi = *epi;
+  p.no_sk = true;  // the stream-K schedule needs a workspace: data-parallel tiles only
   if (p.epi.scale == 0.0f) p.epi.scale = 1.0f;
   p.act = act_of(epi->kind);
   p.has_bias = has_bias;

@@ -102,7 +102,70 @@ struct KParams {
   int n_tma;  // columns [0, n_tma) go out by TMA store; n_tma·size is a multiple of 16 bytes
   int* err;
   unsigned long long wait_limit_ns;
+  // stream-K: the last sk_tiles tiles of the tile order are split along K into
+  // sk_clusters contiguous ranges of (tile, K-block) units (0: data-parallel only)
+  int sk_tiles, sk_clusters;
+  float* sk_ws;   // fp32 partial accumulators: [cluster][CTA rank][epilogue warp][mma_n/2 x 32]
+  int* sk_flags;  // [cluster][CTA rank][epilogue warp]: 1 once that warp's partial is stored
 };
+
+// ------------------------------------------------------------------ work schedule
+// A cluster's work is a sequence of items, the same for its producer, MMA and
+// epilogue warps: first its data-parallel tiles (tile cluster, cluster + clusters, ...
+// below dp_tiles = all tiles - sk_tiles, each over the K blocks [kb_a, kb_b)), then
+// (stream-K) its contiguous range [s_c, s_c+1) of the units u = (tile - dp_tiles)·num_kb
+// + kb of the remaining tiles, s_c = ⌊c·U/sk_clusters⌋.  A range cuts at most two
+// tiles: its first segment may start inside a tile (PARTIAL: the accumulator is stored
+// for that tile's finisher), its last segment may hold a tile's first K blocks without
+// its last (FINISH: the partials of the following clusters w0..w1, whose ranges start
+// inside the tile, are added in cluster order before the epilogue).  A finisher
+// processes its segment last and its writers process theirs first, so it rarely waits.
+enum ItemKind : int { IT_FULL = 0, IT_PARTIAL = 1, IT_FINISH = 2 };
+struct Item {
+  int tile, kb0, kb1, kind, w0, w1;
+};
+__host__ __device__ __forceinline__ int sk_start(const KParams& p, int c) {
+  return (int)((long long)p.sk_tiles * p.num_kb * c / p.sk_clusters);
+}
+// Item i of cluster `cl` of `ncl` (false past the last); data-parallel tiles cover the K
+// blocks [kb_a, kb_b).  Stateless, so that a role keeps only its item counter live.
+__host__ __device__ __forceinline__ bool get_item(const KParams& p, int cl, int ncl, int kb_a, int kb_b, int i,
+                                                  Item& it) {
+  const int dp_tiles = p.tiles_a * p.tiles_b - p.sk_tiles;
+  const int n_dp = dp_tiles > cl ? (dp_tiles - cl + ncl - 1) / ncl : 0;
+  it.w0 = 0;
+  it.w1 = -1;
+  if (i < n_dp) {
+    it.tile = cl + i * ncl;
+    it.kb0 = kb_a;
+    it.kb1 = kb_b;
+    it.kind = IT_FULL;
+    return true;
+  }
+  if (cl >= p.sk_clusters) return false;
+  const int nkb = p.num_kb;
+  const int s = sk_start(p, cl), e = sk_start(p, cl + 1);
+  const int j = i - n_dp;
+  // segment j of the range: the first starts at s, the others at tile boundaries
+  const int u = (j == 0) ? s : (s / nkb + j) * nkb;
+  if (u >= e) return false;
+  const int tl = u / nkb, ts = tl * nkb, te = ts + nkb;
+  const int se = e < te ? e : te;
+  it.tile = dp_tiles + tl;
+  it.kb0 = u - ts;
+  it.kb1 = se - ts;
+  if (u == ts && se == te) {
+    it.kind = IT_FULL;
+  } else if (u > ts) {
+    it.kind = IT_PARTIAL;
+  } else {
+    it.kind = IT_FINISH;
+    it.w0 = cl + 1;
+    it.w1 = cl;
+    while (it.w1 + 1 < p.sk_clusters && sk_start(p, it.w1 + 1) < te) ++it.w1;
+  }
+  return true;
+}
 
 // ------------------------------------------------------------------ helpers
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const KParams& p,
@@ -133,6 +196,85 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
     else (void)mbar_try_wait(bar, parity);
   }
   return ok != 0;
+}
+
+// Warp-uniform bounded wait until a GPU-scope flag in global memory is nonzero (set with
+// release semantics by another CTA); every lane then acquires it itself.
+__device__ __forceinline__ bool warp_wait_flag(const int* f, const KParams& p, int lane) {
+  uint32_t ok = 1;
+  if (lane == 0 && ld_acquire_gpu(f) == 0) {
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_gpu(f) == 0) {
+      if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+        atomicCAS(p.err, 0, kErrTimeout);
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) (void)ld_acquire_gpu(f);
+  return ok != 0;
+}
+
+// Stream-K workspace of one epilogue warp: its accumulator columns in blocks of 32
+// columns x 32 rows; inside a block, float4 j4 of lane l (columns 4·j4 .. 4·j4+3 of row l)
+// is at (j4·32 + l)·4, so a warp-wide float4 access covers 512 contiguous bytes.
+__device__ __forceinline__ float* sk_area(const KParams& p, int cluster, int cta_rank, int kcl, int ew) {
+  return p.sk_ws + ((size_t)(cluster * kcl + cta_rank) * 8u + (size_t)ew) * (size_t)(p.mma_n / 2) * 32u;
+}
+// x[0..31] += block `blk` of a stored partial (this lane's row)
+__device__ __forceinline__ void sk_add_block(float* x, const float* area, int blk, int lane) {
+  const float4* src = reinterpret_cast<const float4*>(area + (size_t)blk * 1024u) + lane;
+#pragma unroll
+  for (int j4 = 0; j4 < 8; ++j4) {
+    const float4 q = __ldcg(src + j4 * 32);
+    x[4 * j4] += q.x;
+    x[4 * j4 + 1] += q.y;
+    x[4 * j4 + 2] += q.z;
+    x[4 * j4 + 3] += q.w;
+  }
+}
+
+// Stream-K, out of line (taken at most twice per CTA, so the register-bound epilogue loop
+// keeps its allocation): the warp's accumulator blocks b = 0 .. mma_n/64 - 1 sit at TMEM
+// column c_begin + 32b, or, past gblk blocks (GeGLU's up half), out_tile_n + c_begin +
+// 32(b - gblk).
+__device__ __noinline__ void sk_store_partial(const KParams& p, uint32_t tacc, int c_begin, int gblk, float* area,
+                                              int lane) {
+#pragma unroll 1
+  for (int b = 0; b < p.mma_n / 64; ++b) {
+    const int col = b < gblk ? c_begin + 32 * b : p.out_tile_n + c_begin + 32 * (b - gblk);
+    uint32_t r[32];
+    tmem_ld32(tacc + (uint32_t)col, r);
+    tmem_wait_ld();
+    float4* dst = reinterpret_cast<float4*>(area + (size_t)b * 1024u) + lane;
+#pragma unroll
+    for (int j4 = 0; j4 < 8; ++j4)
+      __stcg(dst + j4 * 32, make_float4(__uint_as_float(r[4 * j4]), __uint_as_float(r[4 * j4 + 1]),
+                                        __uint_as_float(r[4 * j4 + 2]), __uint_as_float(r[4 * j4 + 3])));
+  }
+}
+// acc += the partials of clusters w0..w1 (in that order), block by block in TMEM
+__device__ __noinline__ void sk_add_partials(const KParams& p, uint32_t tacc, int c_begin, int gblk, int cta_rank,
+                                             int kcl, int ew, int w0, int w1, int lane) {
+#pragma unroll 1
+  for (int b = 0; b < p.mma_n / 64; ++b) {
+    const int col = b < gblk ? c_begin + 32 * b : p.out_tile_n + c_begin + 32 * (b - gblk);
+    uint32_t r[32];
+    tmem_ld32(tacc + (uint32_t)col, r);
+    tmem_wait_ld();
+    float x[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(r[j]);
+#pragma unroll 1
+    for (int w = w0; w <= w1; ++w) sk_add_block(x, sk_area(p, w, cta_rank, kcl, ew), b, lane);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(x[j]);
+    tmem_st32(tacc + (uint32_t)col, r);
+  }
+  tmem_wait_st();
 }
 
 __device__ __forceinline__ float load_elem(const void* p, long long i, int dt) {
@@ -433,13 +575,11 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
   const int csize = PAIR ? kCl : S;
   const int cluster_id = blockIdx.x / csize;
   const int num_clusters = gridDim.x / csize;
-  const int total_tiles = p.tiles_a * p.tiles_b;
   const uint32_t krank = PAIR ? 0u : rank;  // split-K slice of this CTA
   const int kb_begin = (int)(((long long)p.num_kb * krank) / S);
   const int kb_end = (int)(((long long)p.num_kb * (krank + 1)) / S);
   const int tile_rows = PAIR ? 256 : 128;   // output rows per tile (both CTAs of a pair)
   const int cta_row_off = PAIR ? (int)rank * 128 : 0;
-  const bool have_acc = kb_end > kb_begin;
 
   if (threadIdx.x == 0) {
     FL_STAMP(0);
@@ -496,14 +636,15 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int t = cluster_id; ok && t < total_tiles; t += num_clusters) {
+      Item itm;
+      for (int ii = 0; ok && get_item(p, cluster_id, num_clusters, kb_begin, kb_end, ii, itm); ++ii) {
         int ta, tb;
-        tile_coords(t, p, ta, tb);
+        tile_coords(itm.tile, p, ta, tb);
         const int a_row = ta * tile_rows + cta_row_off;
         // PAIR: each CTA loads its half of the B tile
         const int b_row = tb * p.mma_n + (PAIR ? (int)rank * (p.mma_n / 2) : 0);
         const int g_row = tb * p.b_box_rows;
-        for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+        for (int kb = itm.kb0; kb < itm.kb1; ++kb, ++it) {
           const int s = (int)(it % (uint32_t)NS);
           const uint32_t ph = (it / (uint32_t)NS) & 1u;
           if (!wait_bounded(empty_bar(s), ph ^ 1u, p)) { ok = false; break; }
@@ -580,13 +721,15 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
       const uint32_t idesc = p.idesc;
       uint32_t it = 0, local = 0;
       bool ok = true, issued = false;
-      for (int t = cluster_id; ok && t < total_tiles; t += num_clusters, ++local) {
+      Item itm;
+      for (; ok && get_item(p, cluster_id, num_clusters, kb_begin, kb_end, (int)local, itm); ++local) {
+        const bool acc_any = itm.kb1 > itm.kb0;
         const uint32_t buf = local & 1u;
         const uint32_t tph = (local >> 1) & 1u;
         if (!wait_bounded(tempty_bar(buf), tph ^ 1u, p, PAIR)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * (uint32_t)p.mma_n;
-        for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+        for (int kb = itm.kb0; kb < itm.kb1; ++kb, ++it) {
           const int s = (int)(it % (uint32_t)NS);
           const uint32_t ph = (it / (uint32_t)NS) & 1u;
           if (!wait_bounded(TF32 ? conv_bar(s) : full_bar(s), ph, p, TF32 && PAIR)) { ok = false; break; }
@@ -600,11 +743,11 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
 #pragma unroll
             for (int k = 0; k < kUmmaSteps; ++k) {
               if constexpr (PAIR) {
-                umma_tf32_pair(d_tmem, dal + k * ak, db + k * bk, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
+                umma_tf32_pair(d_tmem, dal + k * ak, db + k * bk, idesc, (kb > itm.kb0 || k > 0) ? 1u : 0u);
                 umma_tf32_pair(d_tmem, da + k * ak, dbl + k * bk, idesc, 1u);
                 umma_tf32_pair(d_tmem, da + k * ak, db + k * bk, idesc, 1u);
               } else {
-                umma_tf32(d_tmem, dal + k * ak, db + k * bk, idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
+                umma_tf32(d_tmem, dal + k * ak, db + k * bk, idesc, (kb > itm.kb0 || k > 0) ? 1u : 0u);
                 umma_tf32(d_tmem, da + k * ak, dbl + k * bk, idesc, 1u);
                 umma_tf32(d_tmem, da + k * ak, db + k * bk, idesc, 1u);
               }
@@ -613,12 +756,12 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
 #pragma unroll
             for (int k = 0; k < kMaxSteps; ++k)
               if (k < usteps)
-                umma_f16_pair(d_tmem, da + aso[k], db + bso[k], idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
+                umma_f16_pair(d_tmem, da + aso[k], db + bso[k], idesc, (kb > itm.kb0 || k > 0) ? 1u : 0u);
           } else {
 #pragma unroll
             for (int k = 0; k < kMaxSteps; ++k)
               if (k < usteps)
-                umma_f16(d_tmem, da + aso[k], db + bso[k], idesc, (kb > kb_begin || k > 0) ? 1u : 0u);
+                umma_f16(d_tmem, da + aso[k], db + bso[k], idesc, (kb > itm.kb0 || k > 0) ? 1u : 0u);
           }
           if constexpr (PAIR) {  // free the stage in both CTAs once these MMAs have read it
             umma_commit_pair(empty_bar(s));
@@ -631,7 +774,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         if (!ok) break;
         if (local == 0) FL_STAMP(5);
         if constexpr (PAIR) {
-          if (have_acc) {
+          if (acc_any) {
             umma_commit_pair(tfull_bar(buf));
             umma_commit_pair(mapa_shared(tfull_bar(buf), 1));
           } else {
@@ -639,7 +782,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
             mbar_arrive_remote(mapa_shared(tfull_bar(buf), 1));
           }
         } else {
-          if (have_acc) umma_commit(tfull_bar(buf));
+          if (acc_any) umma_commit(tfull_bar(buf));
           else mbar_arrive(tfull_bar(buf));
         }
       }
@@ -669,15 +812,17 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
       const uint32_t stg = smem_base + p.staging_off + (uint32_t)ew * kStagingBuf;
       const int half_cols = p.out_tile_n >> 1;
       uint32_t cit = 0;  // 3xTF32: stage counter, in step with the producer and the MMA warp
-      for (int t = cluster_id; t < total_tiles; t += num_clusters, ++local) {
+      Item itm;
+      for (; get_item(p, cluster_id, num_clusters, kb_begin, kb_end, (int)local, itm); ++local) {
         int ta, tb;
-        tile_coords(t, p, ta, tb);
+        tile_coords(itm.tile, p, ta, tb);
+        const bool acc_any = itm.kb1 > itm.kb0;
         if constexpr (TF32) {
           // write the TF32 lo half of every stage of this tile beside it (the raw words
           // serve as hi); the 256 epilogue threads share the stage's 16-byte words
           const int et = (warp - kEpiWarp0) * 32 + lane;
           const uint32_t words = p.stage_bytes >> 4;
-          for (int kb = kb_begin; ok && kb < kb_end; ++kb, ++cit) {
+          for (int kb = itm.kb0; ok && kb < itm.kb1; ++kb, ++cit) {
             const int s = (int)(cit % (uint32_t)NS);
             const uint32_t ph = (cit / (uint32_t)NS) & 1u;
             if (!warp_wait_bounded(full_bar(s), ph, p, lane)) { ok = false; break; }
@@ -721,6 +866,39 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
         const int c_begin = half * half_cols;
         const int c_end = c_begin + half_cols;
+        const int gblk = half_cols / 32;  // 32-column blocks of this warp's (gate) columns
+        if (itm.kind == IT_PARTIAL) {
+          // stream-K: this cluster's range starts inside the tile.  Store this warp's fp32
+          // accumulator columns for the tile's finisher, free the TMEM buffer, then release
+          // the warp's flag (every lane's stores are fenced before it).
+          sk_store_partial(p, tacc, c_begin, gblk, sk_area(p, cluster_id, (int)rank, kCl, ew), lane);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (PAIR && rank != 0) mbar_arrive_remote(mapa_shared(tempty_bar(buf), 0));
+            else mbar_arrive(tempty_bar(buf));
+          }
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) st_release_gpu(p.sk_flags + (cluster_id * kCl + (int)rank) * kEpiWarps + ew, 1);
+          if (ew == 0 && lane == 0) FL_STAMP(18);
+          continue;
+        }
+        if (itm.kind == IT_FINISH) {
+          // stream-K: add the partials of the clusters whose ranges start inside this tile
+          // (in cluster order) to this warp's accumulator columns in tensor memory; the
+          // epilogue below then reads the whole tile's sums
+          for (int w = itm.w0; ok && w <= itm.w1; ++w)
+            if (!warp_wait_flag(p.sk_flags + (w * kCl + (int)rank) * kEpiWarps + ew, p, lane)) ok = false;
+          if (!ok) break;
+          if (ew == 0 && lane == 0) FL_STAMP(16);
+          sk_add_partials(p, tacc, c_begin, gblk, (int)rank, kCl, ew, itm.w0, itm.w1, lane);
+          if (ew == 0 && lane == 0) FL_STAMP(17);
+          // every lane has read the partials: the flags are ready for the next launch
+          __syncwarp();
+          if (lane == 0)
+            for (int w = itm.w0; w <= itm.w1; ++w) p.sk_flags[(w * kCl + (int)rank) * kEpiWarps + ew] = 0;
+        }
 
         for (int cc = c_begin; cc < c_end; cc += CH) {
           const int nc0 = n_tile0 + cc;
@@ -737,7 +915,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           }
           // ---- accumulator: every TMEM load of the chunk, then one wait
           float v[CH];
-          if (have_acc) {
+          if (acc_any) {
             if constexpr (ACT == ACT_GEGLU) {
               // gate columns [0, out_tile_n) and up columns [out_tile_n, 2·out_tile_n):
               // h = gelu_tanh(g)·u, 32 columns at a time to bound register use
@@ -760,6 +938,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
 #pragma unroll
               for (int j = 0; j < CH; ++j) v[j] = __uint_as_float(ra[j]);
             }
+            if (ew == 0 && lane == 0 && cc == c_begin) FL_STAMP(19);
           } else {
 #pragma unroll
             for (int j = 0; j < CH; ++j) v[j] = (ACT == ACT_GEGLU) ? activate<ACT, OUT != DT_F32>(0.0f, 0.0f) : 0.0f;
@@ -848,12 +1027,15 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           if (lane == 0) {
             tma_store_2d(&tmOut, stg, nc0, row0);
             bulk_commit_group();
+            if (ew == 0 && cc == c_begin) FL_STAMP(20);
           }
         }
+        if (ew == 0 && lane == 0) FL_STAMP(21);
         if (ew == 0 && lane == 0 && local == 0) FL_STAMP(7);
       }
       if (ew == 0 && lane == 0) FL_STAMP(9);
       if (lane == 0) bulk_wait_group<0>();
+      if (ew == 0 && lane == 0) FL_STAMP(22);
     } else {
       // ---------------- swap-AB layout: TMEM lane = output column n, TMEM column = output row m.
       // Split-K (S > 1): every CTA publishes its fp32 partial tile in its own shared
@@ -878,9 +1060,11 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
       const bool res_async = has_res && p.res_async;
       const int res_es = (p.res_dtype == DT_F32) ? 4 : 2;
       constexpr int eo = (OUT == DT_F32) ? 4 : 2;
-      for (int t = cluster_id; t < total_tiles; t += num_clusters, ++local) {
+      Item itm;
+      for (; get_item(p, cluster_id, num_clusters, kb_begin, kb_end, (int)local, itm); ++local) {
         int ta, tb;
-        tile_coords(t, p, ta, tb);
+        tile_coords(itm.tile, p, ta, tb);
+        const bool acc_any = itm.kb1 > itm.kb0;
         const uint32_t buf = local & 1u;
         const uint32_t tph = (local >> 1) & 1u;
         const int m_lo = tb * p.mma_n + mb;                 // first output row of this warp
@@ -903,7 +1087,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
 #pragma unroll 1
           for (int cc = (ew >> 2) * 32; cc < p.mma_n; cc += 64) {
             uint32_t r[32];
-            if (have_acc) {
+            if (acc_any) {
               tmem_ld32(tacc + (uint32_t)cc, r);
               tmem_wait_ld();
             } else {
@@ -1016,7 +1200,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
                 const float4 v1 = ld_shared_f4(sum_row + (uint32_t)mc * 4u + 16u);
                 x[0] = v0.x, x[1] = v0.y, x[2] = v0.z, x[3] = v0.w;
                 x[4] = v1.x, x[5] = v1.y, x[6] = v1.z, x[7] = v1.w;
-              } else if (have_acc) {
+              } else if (acc_any) {
                 uint32_t r0[4], r1[4];
                 tmem_ld4(tacc + (uint32_t)mc, r0);
                 tmem_ld4(tacc + (uint32_t)mc + 4u, r1);

@@ -105,15 +105,28 @@ typedef struct {
                               elementwise kernel per epilogue step — the unfused
                               design of [gelu] §3.1, kept only to measure the
                               round trip that fusion removes */
-  int32_t reserved[3];     /* must be 0 */
+  int32_t schedule;        /* fl_schedule: how CTA pairs share the output tiles */
+  int32_t reserved[2];     /* must be 0 */
 } fl_epilogue_desc;
+
+/* Work schedule of the CTA-pair layouts (16-bit operands, M > 128). */
+typedef enum {
+  FL_SCHED_AUTO = 0,         /* stream-K when it pays (see fl_plan), else data-parallel */
+  FL_SCHED_DATA_PARALLEL = 1,/* whole tiles only, each pair takes tiles p, p+pairs, ... */
+  FL_SCHED_STREAM_K = 2      /* stream-K whenever the last round of pairs is partly idle */
+} fl_schedule;
 
 typedef struct fl_plan_s* fl_plan_t;
 
 /* Plan one fused linear layer of shape M×N×K ([epilog] Matmul(...).plan(epilog)).
  * Validates the combination, chooses the kernel configuration for the shape,
- * and allocates the plan's small device workspace (an error word, plus the
- * intermediate buffer of an unfused plan).  Needs the target device current.
+ * and allocates the plan's device workspace: an error word; the intermediate buffer
+ * of an unfused plan; and, when the shape's tiles leave the last round of CTA pairs
+ * partly idle (16-bit operands, M > 128), the stream-K workspace: one fp32 partial
+ * accumulator of 32 rows x mma_n/2 columns per CTA and epilogue warp (at most
+ * 148 x 8 x 16 KB = 19.4 MB on a B200) and its flags.  Every execute of the plan
+ * reuses this workspace, so two executes of one plan must not overlap on the GPU.
+ * Needs the target device current.
  *   out     receives the plan handle (host pointer, must not be NULL)
  *   M, N, K ≥ 1 for M and N, ≥ 0 for K (K = 0 gives y = epi(0 + bias)); for
  *           GEGLU_TANH, N is the width of h and W has 2N rows
@@ -209,7 +222,9 @@ typedef struct {
   int32_t smem_bytes;          /* dynamic shared memory per CTA */
   int32_t launches_per_execute;/* kernels one fl_execute launches */
   int32_t cta_pair;            /* 1: two CTAs share each 256-row tensor-core tile */
-  int32_t reserved[6];
+  int32_t stream_k_tiles;      /* tiles split along K over the pairs (stream-K), 0: none */
+  int32_t stream_k_pairs;      /* pairs sharing those tiles' (tile, K-block) units */
+  int32_t reserved[4];
 } fl_plan_info;
 fl_status fl_get_plan_info(fl_plan_t plan, fl_plan_info* info);
 

@@ -73,7 +73,7 @@ def poison(shape, dtype: str, device="cuda") -> torch.Tensor:
 
 def run_linear(fl, *, M, N, K, dtype, epilogue, out_dtype, A, W, bias=None, bias_dtype="bf16",
                bias_axis=0, b_major=0, residual=None, residual_dtype="bf16", scale=1.0,
-               unfused=False, out_pad=8, stream=None, check_canary=True) -> Dict[str, np.ndarray]:
+               unfused=False, out_pad=8, stream=None, check_canary=True, schedule="auto") -> Dict[str, np.ndarray]:
     """Run one layer; A/W/bias/residual are CPU tensors in (padded) storage.
 
     Returns the logical [M, N] output and the aux mask as numpy arrays.
@@ -92,7 +92,7 @@ def run_linear(fl, *, M, N, K, dtype, epilogue, out_dtype, A, W, bias=None, bias
                    residual_dtype=residual_dtype, bias_axis=bias_axis,
                    has_residual=residual is not None, scale=scale, b_major=b_major,
                    lda=A.shape[1], ldb=W.shape[1], ldo=ldo,
-                   ldr=residual.shape[1] if residual is not None else 0, unfused=unfused)
+                   ldr=residual.shape[1] if residual is not None else 0, unfused=unfused, schedule=schedule)
     try:
         plan.execute(dA, dW, dB, aux, dR, out, stream)
         st = plan.check(stream)

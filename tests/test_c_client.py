@@ -28,3 +28,20 @@ def test_c_client_builds_and_runs(tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "0 failure(s)" in r.stdout
+
+
+def test_kernel_schedule_on_the_host(tmp_path):
+    """The kernel's own stream-K schedule function, compiled for the host by nvcc
+    (tests/c/schedule_check.cu): every (tile, K block) unit computed once, one finisher
+    per cut tile, whose writer list is exactly the clusters that store a partial."""
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("needs nvcc")
+    exe = tmp_path / "schedule_check"
+    r = subprocess.run([nvcc, "-std=c++17", "-O1", "-gencode", "arch=compute_100a,code=sm_100a",
+                        os.path.join(ROOT, "tests", "c", "schedule_check.cu"), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr[-2000:]
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "schedule ok" in r.stdout

@@ -127,3 +127,57 @@ def test_preview_applies_the_plan_checks():
     with pytest.raises(fl.FusedLinearError) as e:
         preview(64, 256, 256, kind="NONE", num_sms=1)
     assert e.value.status == fl.FL_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("M,N,K,kind,sk_tiles", [
+    (4096, 4096, 4096, "RELU_AUX_BIAS", 34),   # 256 tiles on 74 pairs: the last 34 by stream-K
+    (512, 4096, 4096, "GELU_BIAS", 32),        # 32 tiles: all of them
+    (2048, 4096, 4096, "GELU_BIAS", 54),
+    (8192, 768, 3072, "NONE", 22),             # GeGLU down projection
+    (1024, 3072, 768, "GELU_TANH_BIAS", 0),    # 48 tiles of 6 K blocks: saves 2 blocks a pair, too few
+    (8192, 3072, 768, "GEGLU_TANH", 0),        # 768 tiles: the last round saves under 4 blocks
+    (8192, 8192, 1024, "BIAS", 0),             # 1024 tiles of 8 K blocks: saves about 1 block
+])
+def test_stream_k_choice(M, N, K, kind, sk_tiles):
+    info = preview(M, N, K, kind=kind, out_dtype="bf16")
+    check_invariants(M, N, K, "bf16", kind, info)
+    T = -(-M // 256) * -(-N // info["tile_n"])
+    assert info["stream_k_tiles"] == sk_tiles
+    if sk_tiles:
+        assert info["stream_k_pairs"] == min(74, sk_tiles * -(-K // 128))
+        assert info["grid"] == 148
+        # the tiles before the stream-K ones are whole rounds of the 74 pairs
+        assert (T - sk_tiles) % 74 == 0
+
+
+@pytest.mark.parametrize("M,N,K,kind,sk_tiles", [
+    (1024, 3072, 768, "GELU_TANH_BIAS", 48),
+    (8192, 3072, 768, "GEGLU_TANH", 102),      # 28 left over, ranges under 4 blocks: one more round joins
+    (8192, 8192, 1024, "BIAS", 62),
+])
+def test_stream_k_forced(M, N, K, kind, sk_tiles):
+    info = preview(M, N, K, kind=kind, out_dtype="bf16", schedule="stream_k")
+    check_invariants(M, N, K, "bf16", kind, info)
+    assert info["stream_k_tiles"] == sk_tiles
+    dp = preview(4096, 4096, 4096, kind="RELU_AUX_BIAS", out_dtype="bf16", schedule="data_parallel")
+    assert dp["stream_k_tiles"] == 0 and dp["grid"] == 148
+
+
+def test_stream_k_only_for_16_bit_pairs():
+    for kw in [dict(M=100, N=4096, K=4096), dict(M=128, N=4096, K=4096)]:   # swap-AB
+        assert preview(kw["M"], kw["N"], kw["K"], kind="GELU_BIAS", out_dtype="f32",
+                       schedule="stream_k")["stream_k_tiles"] == 0
+    assert preview(1024, 3072, 768, "f32", kind="GELU_BIAS", out_dtype="f32",
+                   schedule="stream_k")["stream_k_tiles"] == 0
+    # a full last round stays data-parallel
+    assert preview(256 * 74, 256, 1024, kind="BIAS", out_dtype="bf16", schedule="stream_k")["stream_k_tiles"] == 0
+
+
+def test_unknown_schedule_is_rejected():
+    with pytest.raises(fl.FusedLinearError):
+        e = fl.make_epilogue(kind="BIAS")
+        e.schedule = 7
+        info = fl.fl_plan_info()
+        st = fl.LIB.fl_plan_preview(512, 512, 512, fl.FL_BF16, fl.FL_COMPUTE_32F, fl.ctypes.byref(e), 148, 232448,
+                                    fl.ctypes.byref(info))
+        fl._check(st, "preview")

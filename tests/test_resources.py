@@ -4,7 +4,7 @@ build.py keeps the assembler's resource report beside the library.  The launch
 configurations assume these figures, so a change that breaks one shows up here, on the
 CPU, before it shows up as lost occupancy on the GPU:
 - the fused kernel runs 320 threads a CTA, one CTA per SM: at most 204 registers;
-- the dominant launch (ReLU + mask, bf16 out, CTA pair) has no spills;
+- the dominant launch (ReLU + mask, bf16 out, CTA pair) spills only around its stream-K calls;
 - the dReLU and bias-gradient kernels hold four 256-thread CTAs per SM (≤ 64 registers);
 - the whole-vector LayerNorm holds six 128-thread CTAs per SM (≤ 85 registers).
 Skipped when the report is missing (the library was not built here).
@@ -25,10 +25,11 @@ def _entries():
         pytest.skip("no ptxas report (library not built here)")
     out, cur = {}, None
     for line in open(REPORT):
-        m = re.search(r"Compiling entry function '([^']+)'", line)
+        m = re.search(r"Compiling entry function '([^']+)'", line) or \
+            re.search(r"Function properties for (\S+)", line)
         if m:
             cur = m.group(1)
-            out[cur] = {}
+            out.setdefault(cur, {})
             continue
         if cur is None:
             continue
@@ -52,12 +53,19 @@ def test_fused_kernel_fits_one_cta_of_320_threads():
         assert v["regs"] * 320 <= 65536, (name, v)
 
 
-def test_dominant_launch_has_no_spills():
-    # fl_gemm_epi_tcgen05<ACT_RELU, OUT_BF16, swap=false, tf32=false, pair=true>
+def test_dominant_launch_spills_only_around_its_stream_k_calls():
+    # fl_gemm_epi_tcgen05<ACT_RELU, OUT_BF16, swap=false, tf32=false, pair=true>.  The two
+    # stream-K steps (store a partial accumulator, add the others' partials) are out-of-line
+    # calls, taken at most twice per CTA; the register saves around them are the only
+    # spill traffic (the same kernel with empty callees spills as much; without the calls,
+    # nothing).  The stream-K callees themselves do not spill.
     name = "_ZN2fl19fl_gemm_epi_tcgen05ILi1ELi1ELb0ELb0ELb1EEEv14CUtensorMap_stS1_S1_S1_NS_7KParamsE"
     e = _entries()
     assert name in e
-    assert e[name]["spill"] == 0, e[name]
+    assert e[name]["spill"] <= 128, e[name]
+    for callee in ("_ZN2fl16sk_store_partial", "_ZN2fl15sk_add_partials"):
+        hits = {k: v for k, v in e.items() if k.startswith(callee)}
+        assert all(v.get("spill", 0) == 0 for v in hits.values()), hits
 
 
 @pytest.mark.parametrize("prefix,max_regs", [
