@@ -306,7 +306,8 @@ static int grid_of(const fl_plan_s* p) {
   const int tiles = p->tiles_a * p->tiles_b;
   if (p->swap && p->split_k > 1) return tiles * p->split_k;
   // stream-K: every pair takes the same share of the full rounds and a range of the rest
-  if (p->pair && p->sk_tiles > 0) return 2 * (p->num_sms / 2);
+  // (with fewer tiles than pairs, the 2·tiles pairs that share the tiles' K halves)
+  if (p->pair && p->sk_tiles > 0) return 2 * std::max(p->sk_clusters, (tiles - p->sk_tiles > 0) ? p->num_sms / 2 : 0);
   if (p->pair) return 2 * std::min(tiles, p->num_sms / 2);
   return std::min(tiles, p->num_sms);
 }
@@ -316,24 +317,40 @@ static const void* kernel_of(const fl_plan_s* p, int act, int out) {
   return pick_kernel(act, out, p->swap);
 }
 
-// Stream-K for 16-bit CTA pairs.  Data-parallel, T tiles take ⌈T/P⌉ rounds of the P pairs;
-// stream-K spreads the tiles of the last, partial round over every pair, as contiguous
-// ranges of (tile, K-block) units, at the price of a fix-up per cut tile (a 128 KB partial
-// accumulator per CTA stored, then read and added by the tile's finisher, before its
-// epilogue).  A pair saves (⌈T/P⌉ − T/P)·num_kb K blocks; FL_SCHED_AUTO takes stream-K when
-// that is at least kSkMinSavedBlocks, a few times the fix-up's cost in K blocks.
-constexpr double kSkMinSavedBlocks = 8.0;
-
+// Stream-K for 16-bit CTA pairs.  Data-parallel, T tiles take ⌈T/P⌉ rounds of the P pairs.
+// Stream-K spreads tiles over the pairs as contiguous ranges of (tile, K-block) units, at the
+// price of a fix-up per cut tile: a 128 KB partial accumulator per CTA stored by the pair
+// whose range starts inside the tile, then read and added by the pair holding the tile's
+// first K blocks, before its epilogue.  The fix-up stays off the critical path when every
+// range spans at least a whole tile: a writer stores its partial at the start of its range
+// and the finisher adds it at the end of its own.  So:
+//  * T > P: the tiles of the last, partial round plus one full round are split over all P
+//    pairs (each range ≥ 1 tile, each cut tile split once); a pair saves
+//    (⌈T/P⌉ − T/P)·num_kb K blocks;
+//  * T ≤ P/2: each tile is split in two K halves over 2T pairs; a pair saves num_kb/2 K
+//    blocks, and the finisher waits for the other half's store;
+//  * otherwise (P/2 < T < P) the tiles stay whole.
+// FL_SCHED_STREAM_K takes stream-K whenever one of the two forms applies.  FL_SCHED_AUTO keeps
+// whole tiles: measured on a B200 (interleaved runs, CUDA-graph timed, 1965 MHz), stream-K
+// tied or lost on every synthetic shape — 4096^3 119.2 vs 119.2 us, M = 2048 tail 84.8 vs
+// 72.4, M = 512 tail 41.3 vs 39.0, GeGLU gate/up 84.8 vs 76.5 — except the GeGLU down
+// projection (50.0 vs 51.2 us).  Even with the fix-up removed the stream-K ranges ran the
+// main loop slower per K block than whole tiles do (M = 2048 tail: 79.2 vs 72.6 us).
 static bool stream_k_pays(int64_t T, int64_t P, int num_kb, int schedule) {
-  if (schedule == FL_SCHED_DATA_PARALLEL || num_kb < 2 || T % P == 0) return false;
-  if (schedule == FL_SCHED_STREAM_K) return true;
-  const double saved = ((double)cdiv(T, P) - (double)T / (double)P) * num_kb;
-  return saved >= kSkMinSavedBlocks;
+  if (schedule != FL_SCHED_STREAM_K || num_kb < 2) return false;
+  double saved;
+  if (T > P) {
+    if (T % P == 0) return false;
+    saved = ((double)cdiv(T, P) - (double)T / (double)P) * num_kb;  // K blocks a pair saves
+  } else if (2 * T <= P) {
+    saved = (double)(num_kb / 2);
+  } else {
+    return false;
+  }
+  return saved > 0.0;
 }
 
-// The stream-K split of the chosen configuration: the last partial round of tiles (all
-// tiles when there are fewer than pairs), plus one full round when that leaves the pairs
-// fewer than four K blocks each, over min(P, units) pairs.
+// The stream-K split of the chosen configuration (see stream_k_pays).
 static void choose_stream_k(fl_plan_s* p) {
   p->sk_tiles = 0;
   p->sk_clusters = 0;
@@ -341,10 +358,13 @@ static void choose_stream_k(fl_plan_s* p) {
   const int64_t P = p->num_sms / 2;
   const int64_t T = (int64_t)p->tiles_a * p->tiles_b;
   if (!stream_k_pays(T, P, p->num_kb, p->epi.schedule)) return;
-  int64_t sk = T % P;
-  if (T > P && sk * p->num_kb < 4 * P) sk += P;
-  p->sk_tiles = (int)sk;
-  p->sk_clusters = (int)std::min<int64_t>(P, sk * p->num_kb);
+  if (T > P) {
+    p->sk_tiles = (int)(T % P + P);
+    p->sk_clusters = (int)P;
+  } else {
+    p->sk_tiles = (int)T;
+    p->sk_clusters = (int)(2 * T);
+  }
 }
 
 static fl_status choose_config(fl_plan_s* p) {

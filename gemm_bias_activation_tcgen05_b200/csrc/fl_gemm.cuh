@@ -489,6 +489,54 @@ __device__ __forceinline__ void load_row_chunk(float (&dst)[CH], const void* bas
   }
 }
 
+// CH consecutive 16-bit elements of a row, from element offset i0, kept as raw 16-byte
+// vectors (two elements a 32-bit word, low half first).  Pinned volatile loads, so that
+// they are issued here, ahead of their use; a chunk that ends past n_end (ragged row
+// end) is read element by element, with zeros past n_end.  Requires 16-byte aligned
+// rows when the chunk is whole.
+template <int CH>
+__device__ __forceinline__ void prefetch_row16(uint4 (&q)[CH / 8], const void* base, long long i0, int n0, int n_end) {
+  const uint16_t* b = reinterpret_cast<const uint16_t*>(base) + i0;
+  if (n0 + CH <= n_end) {
+#pragma unroll
+    for (int i = 0; i < CH / 8; ++i)
+      asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(q[i].x), "=r"(q[i].y), "=r"(q[i].z), "=r"(q[i].w)
+                   : "l"(b + 8 * i)
+                   : "memory");
+  } else {
+#pragma unroll
+    for (int i = 0; i < CH / 8; ++i) {
+      uint32_t w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t lo = 0, hi = 0;
+        const int j = 8 * i + 2 * k;
+        if (n0 + j < n_end) {
+          unsigned short h;
+          asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(h) : "l"(b + j) : "memory");
+          lo = h;
+        }
+        if (n0 + j + 1 < n_end) {
+          unsigned short h;
+          asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(h) : "l"(b + j + 1) : "memory");
+          hi = h;
+        }
+        w[k] = lo | (hi << 16);
+      }
+      q[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+// element j of a chunk prefetched by prefetch_row16, widened to fp32
+__device__ __forceinline__ float row16_elem(const uint4* q, int j, int dt) {
+  const uint4 v = q[j >> 3];
+  const int k = (j >> 1) & 3;
+  const uint32_t w = k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
+  const uint32_t h = (j & 1) ? (w >> 16) : (w & 0xFFFFu);
+  return dt == DT_BF16 ? __uint_as_float(h << 16) : __half2float(__ushort_as_half((unsigned short)h));
+}
+
 // Eight read-only loads base[i0], base[i0+stride], ... issued by one asm
 // statement, so all eight are in flight before any result is used.  Every
 // address must be valid (callers clamp the row index).
@@ -855,8 +903,27 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         const int m = row0 + lane;
         const bool m_ok = m < p.M;
         const int n_tile0 = tb * p.out_tile_n;
+        const int c_begin = half * half_cols;
+        const int c_end = c_begin + half_cols;
+        // ---- operands that do not depend on the accumulator, read before its barrier so
+        // that their latency overlaps the main loop: the bias (per row; or lane l holds the
+        // bias of columns c_begin + 32h + l of the tile), and the first chunk of a 16-bit
+        // residual, as raw vectors (later chunks are read one chunk ahead)
         float bias_m = 0.0f;
         if (has_bias && p.bias_axis == 1 && m_ok) bias_m = ldg_pinned(p.bias, m, p.bias_dtype);
+        float bias4[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const int n = n_tile0 + c_begin + 32 * h + lane;
+          bias4[h] = 0.0f;
+          if (has_bias && p.bias_axis == 0 && 32 * h < half_cols && n < p.N) bias4[h] = ldg_pinned(p.bias, n, p.bias_dtype);
+        }
+        // (a 64-column chunk's prefetch buffer would not fit the register budget: those read
+        // their residual at the start of the chunk)
+        const bool res16 = CH == 32 && has_res && p.res_dtype != DT_F32;
+        uint4 rq[CH / 8];
+        if (res16 && m_ok && itm.kind != IT_PARTIAL)
+          prefetch_row16<CH>(rq, p.residual, (long long)m * p.ldr + n_tile0 + c_begin, n_tile0 + c_begin, p.N);
         if (!warp_wait_bounded(tfull_bar(buf), tph, p, lane, PAIR)) { ok = false; break; }
         tc_fence_after();
         if (ew == 0 && lane == 0) {
@@ -864,8 +931,6 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           FL_STAMP(8);
         }
         const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
-        const int c_begin = half * half_cols;
-        const int c_end = c_begin + half_cols;
         const int gblk = half_cols / 32;  // 32-column blocks of this warp's (gate) columns
         if (itm.kind == IT_PARTIAL) {
           // stream-K: this cluster's range starts inside the tile.  Store this warp's fp32
@@ -900,50 +965,143 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
             for (int w = itm.w0; w <= itm.w1; ++w) p.sk_flags[(w * kCl + (int)rank) * kEpiWarps + ew] = 0;
         }
 
-        for (int cc = c_begin; cc < c_end; cc += CH) {
+        // The warp's columns as 32-column blocks in a rolled loop: a block's accumulator,
+        // bias, activation, mask, residual and scale live in 32 registers, and its packed
+        // values go straight into the 128B-swizzled staging row of its chunk (CH columns,
+        // 128 bytes a row), which leaves by one TMA store once its last block is in.  The
+        // next block's TMEM read is issued before this block's arithmetic, so its latency
+        // overlaps it.
+        constexpr int GPB = (OUT == DT_F32) ? 8 : 4;  // 16-byte granules per 32-column block
+        constexpr int BPC = CH / 32;                  // blocks per chunk
+        const int nblk = (c_end - c_begin) / 32;
+        uint32_t ga[32], gu[32];  // the block's accumulator (GeGLU: gate and up columns)
+        if (acc_any) {
+          tmem_ld32(tacc + (uint32_t)c_begin, ga);
+          if constexpr (ACT == ACT_GEGLU) tmem_ld32(tacc + (uint32_t)(p.out_tile_n + c_begin), gu);
+          tmem_wait_ld();
+        }
+#pragma unroll 1
+        for (int b = 0; b < nblk; ++b) {
+          const int hh = b % BPC;
+          const int cc = c_begin + 32 * (b - hh);  // first column of the block's chunk
+          const int cb = c_begin + 32 * b;         // TMEM column (and tile column) of the block
           const int nc0 = n_tile0 + cc;
-          const bool full_cols = nc0 + CH <= p.N;
-          // ---- operands that do not depend on the accumulator first (their latency overlaps)
-          float r[CH];
-          if (has_res && m_ok) load_row_chunk<CH>(r, p.residual, (long long)m * p.ldr, nc0, p.N, p.res_dtype, full_cols);
-          float bl[CH / 32];  // lane l holds bias[nc0 + 32i + l]; broadcast by shuffle below
-#pragma unroll
-          for (int i = 0; i < CH / 32; ++i) {
-            const int n = nc0 + i * 32 + lane;
-            bl[i] = 0.0f;
-            if (has_bias && p.bias_axis == 0 && n < p.N) bl[i] = ldg_pinned(p.bias, n, p.bias_dtype);
+          const int n0 = n_tile0 + cb;              // the block's first output column
+          const bool tma_chunk = nc0 < p.n_tma;
+          if (hh == 0 && tma_chunk) {
+            if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read the staging row
+            if (ew == 0 && lane == 0 && b == 0) FL_STAMP(25);
+            __syncwarp();
           }
-          // ---- accumulator: every TMEM load of the chunk, then one wait
-          float v[CH];
+          const bool full32 = n0 + 32 <= p.N;
+          const float blk_bias = b == 0 ? bias4[0] : b == 1 ? bias4[1] : b == 2 ? bias4[2] : bias4[3];
+          // ---- accumulator of this block; the next block's read goes out now
+          float v[32];
           if (acc_any) {
             if constexpr (ACT == ACT_GEGLU) {
-              // gate columns [0, out_tile_n) and up columns [out_tile_n, 2·out_tile_n):
-              // h = gelu_tanh(g)·u, 32 columns at a time to bound register use
 #pragma unroll
-              for (int h = 0; h < CH / 32; ++h) {
-                uint32_t rg[32], ru[32];
-                tmem_ld32(tacc + (uint32_t)(cc + h * 32), rg);
-                tmem_ld32(tacc + (uint32_t)(p.out_tile_n + cc + h * 32), ru);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  v[h * 32 + j] = activate<ACT, OUT != DT_F32>(__uint_as_float(rg[j]), __uint_as_float(ru[j]));
-              }
+              for (int j = 0; j < 32; ++j) v[j] = activate<ACT, OUT != DT_F32>(__uint_as_float(ga[j]), __uint_as_float(gu[j]));
             } else {
-              uint32_t ra[CH];
 #pragma unroll
-              for (int h = 0; h < CH / 32; ++h)
-                tmem_ld32(tacc + (uint32_t)(cc + h * 32), *reinterpret_cast<uint32_t(*)[32]>(&ra[h * 32]));
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < CH; ++j) v[j] = __uint_as_float(ra[j]);
+              for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(ga[j]);
             }
-            if (ew == 0 && lane == 0 && cc == c_begin) FL_STAMP(19);
+            if (b + 1 < nblk) {
+              tmem_ld32(tacc + (uint32_t)(cb + 32), ga);
+              if constexpr (ACT == ACT_GEGLU) tmem_ld32(tacc + (uint32_t)(p.out_tile_n + cb + 32), gu);
+            }
+            if (ew == 0 && lane == 0 && b == 0) FL_STAMP(19);
           } else {
 #pragma unroll
-            for (int j = 0; j < CH; ++j) v[j] = (ACT == ACT_GEGLU) ? activate<ACT, OUT != DT_F32>(0.0f, 0.0f) : 0.0f;
+            for (int j = 0; j < 32; ++j) v[j] = (ACT == ACT_GEGLU) ? activate<ACT, OUT != DT_F32>(0.0f, 0.0f) : 0.0f;
           }
-          if (cc + CH >= c_end) {
+          // ---- bias, activation, aux, residual, scale (all in fp32 registers)
+          if (has_bias) {
+            if (p.bias_axis == 0) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] += __shfl_sync(0xffffffffu, blk_bias, j);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] += bias_m;
+            }
+          }
+          if (ew == 0 && lane == 0 && hh == 0) {
+            if (b == 0) FL_STAMP(23);
+            if (b == BPC) FL_STAMP(27);
+          }
+          if constexpr (ACT == ACT_GELU) {
+            // GELU_AUX_BIAS: the pre-activation v, in the output type, for the backward pass
+            if (has_aux && m_ok) store_row_chunk<OUT, 32>(p.aux, (long long)m * p.ldo + n0, n0, p.N, v);
+          }
+          if (has_mask) {
+            uint32_t word = 0u;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (v[j] > 0.0f && (full32 || n0 + j < p.N)) word |= 1u << j;
+            if (m_ok && (long long)n0 < p.N) p.aux[(long long)m * p.ld_aux + (n0 >> 5)] = word;
+          }
+          if constexpr (ACT != ACT_GEGLU) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = activate<ACT, OUT != DT_F32>(v[j], 0.0f);
+          }
+          if (has_res && m_ok) {
+            if (res16) {
+              // (res16: 32-column chunks, one block a chunk)
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] += row16_elem(rq, j, p.res_dtype);
+              // the next chunk's residual travels while this chunk is stored
+              if (b + 1 < nblk) prefetch_row16<CH>(rq, p.residual, (long long)m * p.ldr + n0 + 32, n0 + 32, p.N);
+            } else {
+              // (an fp32 residual, or 64-column chunks: read where it is added)
+              float r[32];
+              load_row_chunk<32>(r, p.residual, (long long)m * p.ldr, n0, p.N, p.res_dtype, full32);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] += r[j];
+            }
+          }
+          if (scale != 1.0f) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= scale;
+          }
+          if (ew == 0 && lane == 0 && b == 0) FL_STAMP(24);
+          // ---- ragged row end: a TMA store writes whole 16-byte granules, so the
+          // columns past the last full granule are written with plain stores.
+          if (n0 + 32 > p.n_tma && n0 < p.N && m_ok) {
+            const int j0 = max(p.n_tma - n0, 0);
+            const int j1 = min(p.N - n0, 32);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j >= j0 && j < j1) store_elem<OUT>(p.out, (long long)m * p.ldo + n0 + j, v[j]);
+          }
+          if (tma_chunk) {
+            // ---- the block's granules of the 128B-swizzled staging row
+#pragma unroll
+            for (int c = 0; c < GPB; ++c) {
+              uint32_t w4[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                if constexpr (OUT == DT_F32) w4[k] = __float_as_uint(v[4 * c + k]);
+                else w4[k] = pack2<OUT>(v[8 * c + 2 * k], v[8 * c + 2 * k + 1]);
+              }
+              const uint32_t g = (uint32_t)(GPB * hh + c);
+              const uint32_t addr = stg + (uint32_t)lane * 128u + ((g ^ (uint32_t)(lane & 7)) << 4);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w4[0]), "r"(w4[1]),
+                           "r"(w4[2]), "r"(w4[3])
+                           : "memory");
+            }
+            if (hh == BPC - 1 || b + 1 == nblk) {
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (ew == 0 && lane == 0 && b == BPC - 1) FL_STAMP(26);
+              if (lane == 0) {
+                tma_store_2d(&tmOut, stg, nc0, row0);
+                bulk_commit_group();
+                if (ew == 0 && b == BPC - 1) FL_STAMP(20);
+                if (ew == 0 && b == 2 * BPC - 1) FL_STAMP(28);
+              }
+            }
+          }
+          if (acc_any && b + 1 < nblk) tmem_wait_ld();  // the next block's accumulator has arrived
+          if (b + 1 == nblk) {
             // this warp's TMEM reads of the tile are done: hand its share back to the MMA warp
             // (in a pair, to the leader's barrier)
             tc_fence_before();
@@ -952,82 +1110,6 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
               if (PAIR && rank != 0) mbar_arrive_remote(mapa_shared(tempty_bar(buf), 0));
               else mbar_arrive(tempty_bar(buf));
             }
-          }
-          // ---- bias, activation, aux, residual, scale (all in fp32 registers)
-          if (has_bias) {
-            if (p.bias_axis == 0) {
-#pragma unroll
-              for (int j = 0; j < CH; ++j) v[j] += __shfl_sync(0xffffffffu, bl[j >> 5], j & 31);
-            } else {
-#pragma unroll
-              for (int j = 0; j < CH; ++j) v[j] += bias_m;
-            }
-          }
-          uint32_t aux_word[CH / 32];
-#pragma unroll
-          for (int h = 0; h < CH / 32; ++h) aux_word[h] = 0u;
-          if constexpr (ACT == ACT_GELU) {
-            // GELU_AUX_BIAS: the pre-activation v, in the output type, for the backward pass
-            if (has_aux && m_ok) store_row_chunk<OUT, CH>(p.aux, (long long)m * p.ldo + nc0, nc0, p.N, v);
-          }
-          if (has_mask) {
-#pragma unroll
-            for (int j = 0; j < CH; ++j)
-              if (v[j] > 0.0f && (full_cols || nc0 + j < p.N)) aux_word[j >> 5] |= 1u << (j & 31);
-          }
-          if constexpr (ACT != ACT_GEGLU) {
-#pragma unroll
-            for (int j = 0; j < CH; ++j) v[j] = activate<ACT, OUT != DT_F32>(v[j], 0.0f);
-          }
-          if (has_res && m_ok) {
-#pragma unroll
-            for (int j = 0; j < CH; ++j) v[j] += r[j];
-          }
-          if (scale != 1.0f) {
-#pragma unroll
-            for (int j = 0; j < CH; ++j) v[j] *= scale;
-          }
-          if (has_mask && m_ok) {
-#pragma unroll
-            for (int h = 0; h < CH / 32; ++h) {
-              const int w = (nc0 >> 5) + h;
-              if ((long long)w * 32 < p.N) p.aux[(long long)m * p.ld_aux + w] = aux_word[h];
-            }
-          }
-          // ---- ragged row end: a TMA store writes whole 16-byte granules, so the
-          // columns past the last full granule are written with plain stores.
-          if (nc0 + CH > p.n_tma && nc0 < p.N && m_ok) {
-            const int j0 = max(p.n_tma - nc0, 0);
-            const int j1 = min(p.N - nc0, CH);
-#pragma unroll
-            for (int j = 0; j < CH; ++j)
-              if (j >= j0 && j < j1) store_elem<OUT>(p.out, (long long)m * p.ldo + nc0 + j, v[j]);
-          }
-          if (nc0 >= p.n_tma) continue;
-          // ---- stage the 32 x 128-byte block in 128B-swizzled smem, TMA-store it
-          uint32_t words[32];
-          if constexpr (OUT == DT_F32) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) words[j] = __float_as_uint(v[j]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) words[j] = pack2<OUT>(v[2 * j], v[2 * j + 1]);
-          }
-          if (lane == 0) bulk_wait_group_read<0>();  // the previous store has finished reading smem
-          __syncwarp();
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint32_t addr = stg + (uint32_t)lane * 128u + ((uint32_t)(c ^ (lane & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(words[4 * c]),
-                         "r"(words[4 * c + 1]), "r"(words[4 * c + 2]), "r"(words[4 * c + 3])
-                         : "memory");
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmOut, stg, nc0, row0);
-            bulk_commit_group();
-            if (ew == 0 && cc == c_begin) FL_STAMP(20);
           }
         }
         if (ew == 0 && lane == 0) FL_STAMP(21);

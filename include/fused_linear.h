@@ -111,9 +111,13 @@ typedef struct {
 
 /* Work schedule of the CTA-pair layouts (16-bit operands, M > 128). */
 typedef enum {
-  FL_SCHED_AUTO = 0,         /* stream-K when it pays (see fl_plan), else data-parallel */
+  FL_SCHED_AUTO = 0,         /* the library's choice: whole tiles (stream-K measured no faster) */
   FL_SCHED_DATA_PARALLEL = 1,/* whole tiles only, each pair takes tiles p, p+pairs, ... */
-  FL_SCHED_STREAM_K = 2      /* stream-K whenever the last round of pairs is partly idle */
+  FL_SCHED_STREAM_K = 2      /* stream-K when the tiles leave pairs idle: the last partial round
+                                plus one full round split over all pairs as contiguous ranges of
+                                (tile, K block) units, or with at most half as many tiles as
+                                pairs each tile split in two K halves; the cut tiles' fp32
+                                partial sums go through the plan's workspace */
 } fl_schedule;
 
 typedef struct fl_plan_s* fl_plan_t;

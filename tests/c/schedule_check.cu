@@ -79,16 +79,17 @@ static int check(int tiles_a, int tiles_b, int nkb, int sk, int skc, int ncl) {
 
 int main() {
   int cases = 0;
-  // the synthetic workloads on 74 CTA pairs (tiles_a, tiles_b, K blocks, stream-K tiles)
-  const int known[][4] = {{16, 16, 32, 34},  // 4096^3
-                          {2, 16, 32, 32},   // M = 512 tail
-                          {8, 16, 32, 54},   // M = 2048 tail
-                          {4, 12, 6, 48},    // 1024 x 3072 x 768
-                          {32, 3, 24, 22},   // GeGLU down projection
-                          {32, 24, 6, 102}}; // GeGLU gate/up
+  // the synthetic workloads on 74 CTA pairs (tiles_a, tiles_b, K blocks, stream-K tiles,
+  // stream-K pairs, pairs launched), as fl_plan splits them
+  const int known[][6] = {{16, 16, 32, 108, 74, 74},  // 4096^3: 34 left over plus one round
+                          {2, 16, 32, 32, 64, 64},    // M = 512 tail: each tile in two K halves
+                          {8, 16, 32, 128, 74, 74},   // M = 2048 tail
+                          {32, 3, 24, 96, 74, 74},    // GeGLU down projection
+                          {32, 24, 6, 102, 74, 74},   // GeGLU gate/up (stream-K forced)
+                          {16, 16, 32, 34, 74, 74},   // ranges shorter than a tile
+                          {4, 12, 6, 48, 74, 74}};    // ranges shorter than a tile
   for (const auto& k : known) {
-    const int skc = std::min(74, k[3] * k[2]);
-    if (check(k[0], k[1], k[2], k[3], skc, 74)) return 1;
+    if (check(k[0], k[1], k[2], k[3], k[4], k[5])) return 1;
     ++cases;
   }
   // random shapes, with and without stream-K
@@ -104,6 +105,11 @@ int main() {
     const int skc = sk > 0 ? std::min(ncl, sk * nkb) : 0;
     if (check(ta, tb, nkb, sk, skc, ncl)) return 1;
     ++cases;
+    // every tile split in two K halves over 2T clusters
+    if (2 * T <= 160 && nkb >= 2) {
+      if (check(ta, tb, nkb, T, 2 * T, 2 * T)) return 1;
+      ++cases;
+    }
   }
   std::printf("schedule ok: %d cases\n", cases);
   return 0;

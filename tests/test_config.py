@@ -129,31 +129,37 @@ def test_preview_applies_the_plan_checks():
     assert e.value.status == fl.FL_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("M,N,K,kind,sk_tiles", [
-    (4096, 4096, 4096, "RELU_AUX_BIAS", 34),   # 256 tiles on 74 pairs: the last 34 by stream-K
-    (512, 4096, 4096, "GELU_BIAS", 32),        # 32 tiles: all of them
-    (2048, 4096, 4096, "GELU_BIAS", 54),
-    (8192, 768, 3072, "NONE", 22),             # GeGLU down projection
-    (1024, 3072, 768, "GELU_TANH_BIAS", 0),    # 48 tiles of 6 K blocks: saves 2 blocks a pair, too few
-    (8192, 3072, 768, "GEGLU_TANH", 0),        # 768 tiles: the last round saves under 4 blocks
-    (8192, 8192, 1024, "BIAS", 0),             # 1024 tiles of 8 K blocks: saves about 1 block
+@pytest.mark.parametrize("M,N,K,kind,sk_tiles,sk_pairs", [
+    (4096, 4096, 4096, "RELU_AUX_BIAS", 108, 74),  # 256 tiles: the last 34 plus one round of 74
+    (512, 4096, 4096, "GELU_BIAS", 32, 64),        # 32 tiles, each split in two K halves
+    (2048, 4096, 4096, "GELU_BIAS", 128, 74),      # 128 tiles: 54 plus one round, all of them
+    (8192, 768, 3072, "NONE", 96, 74),             # GeGLU down projection
+    (1024, 3072, 768, "GELU_TANH_BIAS", 0, 0),     # 48 tiles on 74 pairs: whole tiles
 ])
-def test_stream_k_choice(M, N, K, kind, sk_tiles):
-    info = preview(M, N, K, kind=kind, out_dtype="bf16")
+def test_stream_k_choice(M, N, K, kind, sk_tiles, sk_pairs):
+    # the default schedule keeps whole tiles; stream-K, when asked for, splits as described
+    auto = preview(M, N, K, kind=kind, out_dtype="bf16")
+    assert auto["stream_k_tiles"] == 0 and auto["stream_k_pairs"] == 0
+    info = preview(M, N, K, kind=kind, out_dtype="bf16", schedule="stream_k")
     check_invariants(M, N, K, "bf16", kind, info)
     T = -(-M // 256) * -(-N // info["tile_n"])
     assert info["stream_k_tiles"] == sk_tiles
+    assert info["stream_k_pairs"] == sk_pairs
     if sk_tiles:
-        assert info["stream_k_pairs"] == min(74, sk_tiles * -(-K // 128))
-        assert info["grid"] == 148
+        # every stream-K range spans at least one whole tile, or (fewer tiles than half the
+        # pairs) each tile is split in exactly two K halves
+        units = sk_tiles * -(-K // 128)
+        assert units // sk_pairs >= -(-K // 128) or sk_pairs == 2 * sk_tiles
         # the tiles before the stream-K ones are whole rounds of the 74 pairs
         assert (T - sk_tiles) % 74 == 0
+        assert info["grid"] == 2 * max(sk_pairs, 74 if T > sk_tiles else 0)
 
 
 @pytest.mark.parametrize("M,N,K,kind,sk_tiles", [
-    (1024, 3072, 768, "GELU_TANH_BIAS", 48),
-    (8192, 3072, 768, "GEGLU_TANH", 102),      # 28 left over, ranges under 4 blocks: one more round joins
-    (8192, 8192, 1024, "BIAS", 62),
+    (1024, 3072, 768, "GELU_TANH_BIAS", 0),    # 48 tiles: more than half the pairs, fewer than all
+    (8192, 3072, 768, "GEGLU_TANH", 102),      # 28 left over plus one round
+    (8192, 8192, 1024, "BIAS", 136),
+    (600, 1000, 1000, "GELU_BIAS", 12),
 ])
 def test_stream_k_forced(M, N, K, kind, sk_tiles):
     info = preview(M, N, K, kind=kind, out_dtype="bf16", schedule="stream_k")
