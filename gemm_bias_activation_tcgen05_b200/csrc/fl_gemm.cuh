@@ -719,15 +719,20 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           } else {
             const uint32_t fb = full_bar(s);
             mbar_arrive_expect_tx(fb, p.stage_bytes);
-            tma_load_2d(sa, &tmA, fb, k0, a_row);
+            for (int a = 0; a < p.k_atoms; ++a) tma_load_2d(sa + a * p.a_atom_bytes, &tmA, fb, k0 + a * ae, a_row);
             if (p.b_mn_major) {
+              // one box covers the stage's bk rows of the N-contiguous B
               for (int i = 0; i < p.b_boxes; ++i) tma_load_2d(sb + i * p.b_box_bytes, &tmB, fb, b_row + i * 64, k0);
             } else if (p.geglu) {
-              tma_load_2d(sb, &tmB, fb, k0, g_row);
-              tma_load_2d(sb + p.b_box_bytes, &tmB2, fb, k0, g_row);
+              for (int a = 0; a < p.k_atoms; ++a) {
+                tma_load_2d(sb + a * p.b_atom_bytes, &tmB, fb, k0 + a * ae, g_row);
+                tma_load_2d(sb + a * p.b_atom_bytes + p.b_box_bytes, &tmB2, fb, k0 + a * ae, g_row);
+              }
             } else {
-              for (int i = 0; i < p.b_boxes; ++i)
-                tma_load_2d(sb + i * p.b_box_bytes, &tmB, fb, k0, b_row + i * p.b_box_rows);
+              for (int a = 0; a < p.k_atoms; ++a)
+                for (int i = 0; i < p.b_boxes; ++i)
+                  tma_load_2d(sb + a * p.b_atom_bytes + i * p.b_box_bytes, &tmB, fb, k0 + a * ae,
+                              b_row + i * p.b_box_rows);
             }
           }
         }

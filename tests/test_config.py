@@ -29,9 +29,9 @@ def preview(M, N, K, dtype="bf16", **kw):
 
 
 def bk_elems(dtype, info):
-    # K elements of one pipeline stage: 128-byte swizzle atoms, two for 16-bit pairs
+    # K elements of one pipeline stage: 128-byte swizzle atoms, two for 16-bit operands
     es = 4 if dtype == "f32" else 2
-    atoms = 2 if (info["cta_pair"] and dtype != "f32") else 1
+    atoms = 2 if dtype != "f32" else 1
     return atoms * 128 // es
 
 
