@@ -49,11 +49,12 @@ struct BwdParams {
   int rows_per_block, row_blocks, vec_ok;
 };
 
-// GELU'(v) = Φ(v) + v·φ(v) in fp32, with erf as in the forward epilogue
+// GELU'(v) = Φ(v) + v·φ(v) in fp32, with erf as in the forward epilogue; the e^(-x²) of
+// that erf at x = v/√2 is e^(-v²/2), so φ(v) = e^(-v²/2)/√(2π) needs no second exponential
 __device__ __forceinline__ float gelu_erf_grad_f(float v) {
-  const float Phi = 0.5f * (1.0f + erf_as(v * 0.70710678118654752f));
-  const float phi = ex2_approx(-0.5f * v * v * 1.4426950408889634f) * 0.39894228040143268f;  // e^(-v²/2)/√(2π)
-  return fmaf(v, phi, Phi);
+  float e;
+  const float Phi = fmaf(0.5f, erf_as_e(v * 0.70710678118654752f, e), 0.5f);
+  return fmaf(v * 0.39894228040143268f, e, Phi);
 }
 
 // Grid (column strips of 32 16-byte vectors, row blocks).  Warp w of a CTA takes rows
@@ -167,15 +168,15 @@ __global__ void __launch_bounds__(256, 4) fl_bwd_bgrad_kernel(const BwdParams P)
     if (c < P.N) {
       const float* src = P.ws + c;
       float s = 0.0f;
-      int b = 0;
-      for (; b + 8 <= P.row_blocks; b += 8) {
-        float t[8];
+      // sixteen row blocks' loads in flight a trip (this tail runs after all other blocks)
+      for (int b = 0; b < P.row_blocks; b += 16) {
+        float t[16];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) t[k] = __ldcg(src + (long long)(b + k) * P.ws_ld);
+        for (int k = 0; k < 16; ++k) t[k] = (b + k < P.row_blocks) ? __ldcg(src + (long long)(b + k) * P.ws_ld) : 0.0f;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) s += t[k];
+        for (int k = 0; k < 16; ++k)
+          if (b + k < P.row_blocks) s += t[k];
       }
-      for (; b < P.row_blocks; ++b) s += __ldcg(src + (long long)b * P.ws_ld);
       P.dbias[c] = s;
     }
   }

@@ -299,7 +299,8 @@ __device__ __forceinline__ void store_elem(void* p, long long i, float v) {
 // absolute error at most 1.5e-7; erf is odd.  e^(-x²) and 1/(1 + p|x|) come from the
 // special-function unit (relative errors near 2^-22), which keeps the total error
 // near 2e-7, far inside the fp32 tolerance of the layer.
-__device__ __forceinline__ float erf_as(float x) {
+// (erf_as_e also returns the e^(-x²) it used)
+__device__ __forceinline__ float erf_as_e(float x, float& e) {
   const float ax = fabsf(x);
   const float t = rcp_approx(fmaf(0.3275911f, ax, 1.0f));
   float q = fmaf(1.061405429f, t, -1.453152027f);
@@ -307,8 +308,12 @@ __device__ __forceinline__ float erf_as(float x) {
   q = fmaf(q, t, -0.284496736f);
   q = fmaf(q, t, 0.254829592f);
   q *= t;
-  const float e = ex2_approx(-(ax * ax) * 1.4426950408889634f);  // e^(-x²)
+  e = ex2_approx(-(ax * ax) * 1.4426950408889634f);  // e^(-x²)
   return copysignf(fmaf(-q, e, 1.0f), x);
+}
+__device__ __forceinline__ float erf_as(float x) {
+  float e;
+  return erf_as_e(x, e);
 }
 // tanh(u) = 1 - 2/(e^(2u) + 1): saturates to ±1 exactly (e^(2u) = inf or 0), absolute
 // error near 2^-22 elsewhere.
