@@ -182,6 +182,20 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, cons
   }
 }
 
+// Position in the shared-memory ring: stage index and the parity of its current fill.
+// Kept incrementally: the UMMA issuer's per-stage work between two batches of UMMAs
+// leaves the tensor pipe idle (it queues little), and a division by the runtime stage
+// count there costs more than a stage's barrier wait.
+struct StageRing {
+  uint32_t s = 0, ph = 0;
+  __device__ __forceinline__ void next(uint32_t ns) {
+    if (++s == ns) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+};
+
 // Warp-uniform bounded wait: lane 0 spins, the verdict is broadcast.
 __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity, const KParams& p,
                                                   int lane, bool cluster_scope = false) {
@@ -688,6 +702,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
     // ================================================================ TMA producer
     if (lane == 0) {
       uint32_t it = 0;
+      StageRing rs;
       bool ok = true;
       Item itm;
       for (int ii = 0; ok && get_item(p, cluster_id, num_clusters, kb_begin, kb_end, ii, itm); ++ii) {
@@ -697,9 +712,9 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         // PAIR: each CTA loads its half of the B tile
         const int b_row = tb * p.mma_n + (PAIR ? (int)rank * (p.mma_n / 2) : 0);
         const int g_row = tb * p.b_box_rows;
-        for (int kb = itm.kb0; kb < itm.kb1; ++kb, ++it) {
-          const int s = (int)(it % (uint32_t)NS);
-          const uint32_t ph = (it / (uint32_t)NS) & 1u;
+        for (int kb = itm.kb0; kb < itm.kb1; ++kb, ++it, rs.next((uint32_t)NS)) {
+          const int s = (int)rs.s;
+          const uint32_t ph = rs.ph;
           if (!wait_bounded(empty_bar(s), ph ^ 1u, p)) { ok = false; break; }
           if (it == 0) FL_STAMP(3);
           const uint32_t sa = smem_base + (uint32_t)s * p.stage_stride;
@@ -778,6 +793,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
       const int usteps = p.usteps;
       const uint32_t idesc = p.idesc;
       uint32_t it = 0, local = 0;
+      StageRing rs;
       bool ok = true, issued = false;
       Item itm;
       for (; ok && get_item(p, cluster_id, num_clusters, kb_begin, kb_end, (int)local, itm); ++local) {
@@ -787,9 +803,9 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         if (!wait_bounded(tempty_bar(buf), tph ^ 1u, p, PAIR)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * (uint32_t)p.mma_n;
-        for (int kb = itm.kb0; kb < itm.kb1; ++kb, ++it) {
-          const int s = (int)(it % (uint32_t)NS);
-          const uint32_t ph = (it / (uint32_t)NS) & 1u;
+        for (int kb = itm.kb0; kb < itm.kb1; ++kb, ++it, rs.next((uint32_t)NS)) {
+          const int s = (int)rs.s;
+          const uint32_t ph = rs.ph;
           if (!wait_bounded(TF32 ? conv_bar(s) : full_bar(s), ph, p, TF32 && PAIR)) { ok = false; break; }
           tc_fence_after();
           if (it == 0) FL_STAMP(4);
@@ -822,8 +838,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
                 umma_f16(d_tmem, da + aso[k], db + bso[k], idesc, (kb > itm.kb0 || k > 0) ? 1u : 0u);
           }
           if constexpr (PAIR) {  // free the stage in both CTAs once these MMAs have read it
-            umma_commit_pair(empty_bar(s));
-            umma_commit_pair(mapa_shared(empty_bar(s), 1));
+            umma_commit_pair_both(empty_bar(s));
           } else {
             umma_commit(empty_bar(s));  // frees the stage once these MMAs have read it
           }
@@ -833,8 +848,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         if (local == 0) FL_STAMP(5);
         if constexpr (PAIR) {
           if (acc_any) {
-            umma_commit_pair(tfull_bar(buf));
-            umma_commit_pair(mapa_shared(tfull_bar(buf), 1));
+            umma_commit_pair_both(tfull_bar(buf));
           } else {
             mbar_arrive(tfull_bar(buf));
             mbar_arrive_remote(mapa_shared(tfull_bar(buf), 1));
@@ -869,7 +883,7 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
       const int half = ew >> 2;
       const uint32_t stg = smem_base + p.staging_off + (uint32_t)ew * kStagingBuf;
       const int half_cols = p.out_tile_n >> 1;
-      uint32_t cit = 0;  // 3xTF32: stage counter, in step with the producer and the MMA warp
+      StageRing crs;  // 3xTF32: ring position, in step with the producer and the MMA warp
       Item itm;
       for (; get_item(p, cluster_id, num_clusters, kb_begin, kb_end, (int)local, itm); ++local) {
         int ta, tb;
@@ -880,9 +894,9 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           // serve as hi); the 256 epilogue threads share the stage's 16-byte words
           const int et = (warp - kEpiWarp0) * 32 + lane;
           const uint32_t words = p.stage_bytes >> 4;
-          for (int kb = itm.kb0; ok && kb < itm.kb1; ++kb, ++cit) {
-            const int s = (int)(cit % (uint32_t)NS);
-            const uint32_t ph = (cit / (uint32_t)NS) & 1u;
+          for (int kb = itm.kb0; ok && kb < itm.kb1; ++kb, crs.next((uint32_t)NS)) {
+            const int s = (int)crs.s;
+            const uint32_t ph = crs.ph;
             if (!warp_wait_bounded(full_bar(s), ph, p, lane)) { ok = false; break; }
             const uint32_t st0 = smem_base + (uint32_t)s * p.stage_stride;
             for (uint32_t w = (uint32_t)et; w < words; w += kEpiWarps * 32) {

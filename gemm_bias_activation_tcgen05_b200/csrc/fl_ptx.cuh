@@ -186,6 +186,15 @@ __device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t adesc, u
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// One arrive on the barrier at shared-memory offset `bar` in BOTH CTAs of the pair (cta mask
+// 0b11), once every CTA-pair UMMA issued so far by this thread has completed.  One commit
+// instead of one per CTA: the issuing thread's per-stage work sits between UMMA batches.
+__device__ __forceinline__ void umma_commit_pair_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"((unsigned short)3)
+      : "memory");
+}
 // Arrive once on `bar` (a shared::cluster address, possibly the peer CTA's) when
 // every CTA-pair UMMA issued so far by this thread has completed.
 __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
