@@ -1057,10 +1057,16 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
             if (has_aux && m_ok) store_row_chunk<OUT, 32>(p.aux, (long long)m * p.ldo + n0, n0, p.N, v);
           }
           if (has_mask) {
-            uint32_t word = 0u;
+            // bit j = (v_j > 0), in four independent partial words (the OR chains stay
+            // short); the columns past N are cleared once for the whole word
+            uint32_t w4[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (v[j] > 0.0f && (full32 || n0 + j < p.N)) word |= 1u << j;
+            for (int j = 0; j < 32; ++j) w4[j & 3] |= (v[j] > 0.0f ? 1u : 0u) << j;
+            uint32_t word = (w4[0] | w4[1]) | (w4[2] | w4[3]);
+            if (!full32) {
+              const int rem = p.N - n0;  // columns of the word inside the matrix, < 32
+              word = rem > 0 ? word & ((1u << rem) - 1u) : 0u;
+            }
             if (m_ok && (long long)n0 < p.N) p.aux[(long long)m * p.ld_aux + (n0 >> 5)] = word;
           }
           if constexpr (ACT != ACT_GEGLU) {
