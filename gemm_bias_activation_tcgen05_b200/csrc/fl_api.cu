@@ -1128,26 +1128,26 @@ extern "C" fl_status fl_relu_backward(const void* grad, const uint32_t* aux, voi
 }
 
 // ------------------------------------------------------------------ backward with bias gradient
-// Launch geometry of fl_bwd_bgrad_kernel: column strips of 32 16-byte vectors, and
-// row blocks enough for about four CTAs per SM.
+// Launch geometry of fl_bwd_bgrad_kernel: column groups of eight strips of 32 16-byte
+// vectors, and row blocks enough for one resident wave of three CTAs per SM; the
+// workspace holds one row of fp32 column partial sums per row block.
 struct BwdGeom {
-  int strips, row_blocks, rows_per_block;
+  int groups, row_blocks, rows_per_block;
   long long ws_ld;
-  size_t counters_bytes, bytes;
+  size_t bytes;
 };
 static fl_status bwd_geom(int64_t M, int64_t N, int dtype, BwdGeom* g) {
   int dev = 0, sms = 148;
   FL_CUDA(cudaGetDevice(&dev));
   FL_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   const int ve = 16 / esize(dtype);
-  g->strips = (int)std::max<int64_t>(1, cdiv(N, 32LL * ve));
-  int64_t rb = std::max<int64_t>(1, cdiv(4LL * sms, g->strips));
-  rb = std::min<int64_t>(rb, std::max<int64_t>(1, cdiv(M, 8)));
+  g->groups = (int)std::max<int64_t>(1, cdiv(N, 8LL * 32LL * ve));
+  int64_t rb = std::max<int64_t>(1, cdiv(3LL * sms, g->groups));
+  rb = std::min<int64_t>(rb, std::max<int64_t>(1, M));
   g->rows_per_block = (int)std::max<int64_t>(1, cdiv(M, rb));
   g->row_blocks = (int)std::max<int64_t>(1, cdiv(M, g->rows_per_block));
-  g->ws_ld = (long long)g->strips * 32LL * ve;
-  g->counters_bytes = (size_t)cdiv((int64_t)g->strips * 4, 256) * 256;
-  g->bytes = g->counters_bytes + (size_t)g->row_blocks * (size_t)g->ws_ld * sizeof(float);
+  g->ws_ld = (long long)g->groups * 8LL * 32LL * ve;
+  g->bytes = (size_t)g->row_blocks * (size_t)g->ws_ld * sizeof(float);
   return FL_OK;
 }
 
@@ -1186,7 +1186,7 @@ static fl_status bwd_bgrad(int mode, const char* who, const void* grad, const ui
   fl_status st = bwd_geom(M, N, dtype, &g);
   if (st) return st;
   if (dbias && (!workspace || workspace_bytes < g.bytes || !aligned16(workspace)))
-    return fail(FL_ERR_INVALID_ARG, "%s: the bias gradient needs a 16-byte aligned, zero-initialised workspace of "
+    return fail(FL_ERR_INVALID_ARG, "%s: the bias gradient needs a 16-byte aligned workspace of "
                 "%zu bytes (fl_bias_grad_workspace_size)", who, g.bytes);
   if (M == 0 || N == 0) {
     if (dbias && N > 0) FL_CUDA(cudaMemsetAsync(dbias, 0, (size_t)N * sizeof(float), (cudaStream_t)stream_));
@@ -1198,8 +1198,7 @@ static fl_status bwd_bgrad(int mode, const char* who, const void* grad, const ui
   P.v = v;
   P.dpre = dpre;
   P.dbias = dbias;
-  P.counters = reinterpret_cast<int*>(workspace);
-  P.ws = dbias ? reinterpret_cast<float*>(static_cast<char*>(workspace) + g.counters_bytes) : nullptr;
+  P.ws = dbias ? reinterpret_cast<float*>(workspace) : nullptr;
   P.M = M;
   P.N = N;
   P.ldg = ld_grad;
@@ -1212,7 +1211,7 @@ static fl_status bwd_bgrad(int mode, const char* who, const void* grad, const ui
   P.vec_ok = aligned16(grad) && aligned16(dpre) && (ld_grad * es) % 16 == 0 && (ld_dpre * es) % 16 == 0 &&
              (mode == BWD_DRELU || (aligned16(v) && (ld_v * es) % 16 == 0));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
-  const dim3 grid((unsigned)g.strips, (unsigned)g.row_blocks);
+  const dim3 grid((unsigned)g.groups, (unsigned)g.row_blocks);
   cudaError_t err;
   if (mode == BWD_DRELU) {
     err = dtype == FL_BF16 ? launch_pdl(fl_bwd_bgrad_kernel<DT_BF16, BWD_DRELU>, grid, s, P)
@@ -1224,6 +1223,12 @@ static fl_status bwd_bgrad(int mode, const char* who, const void* grad, const ui
                            : launch_pdl(fl_bwd_bgrad_kernel<DT_F32, BWD_DGELU>, grid, s, P);
   }
   if (err != cudaSuccess) return fail(FL_ERR_CUDA, "%s: kernel launch: %s", who, cudaGetErrorString(err));
+  if (dbias) {
+    // the column sums of the row blocks' partials, in a fixed order
+    err = launch_pdl_b(fl_bgrad_reduce_kernel, dim3((unsigned)cdiv(N, 32)), 1024u, s, (const float*)P.ws, dbias,
+                       (long long)N, (long long)g.ws_ld, g.row_blocks);
+    if (err != cudaSuccess) return fail(FL_ERR_CUDA, "%s: reduction kernel launch: %s", who, cudaGetErrorString(err));
+  }
   return after_launch(s, who);
 }
 

@@ -43,8 +43,7 @@ struct BwdParams {
   const void* v;         // DGELU: [M, ldv] of DT, the stored pre-activation
   void* dpre;            // [M, ldd] of DT
   float* dbias;          // [N] fp32, or null (no bias gradient)
-  float* ws;             // row_blocks x ws_ld fp32 partial column sums
-  int* counters;         // per column strip: row blocks that have stored their partials
+  float* ws;             // row_blocks x ws_ld fp32 column partial sums, one row per row block
   long long M, N, ldg, ldv, ldd, words, ws_ld;
   int rows_per_block, row_blocks, vec_ok;
 };
@@ -57,24 +56,30 @@ __device__ __forceinline__ float gelu_erf_grad_f(float v) {
   return fmaf(v * 0.39894228040143268f, e, Phi);
 }
 
-// Grid (column strips of 32 16-byte vectors, row blocks).  Warp w of a CTA takes rows
-// r ≡ w (mod 8) of the block, lane l the l-th vector of the strip, so every warp-wide
-// access is 512 contiguous bytes of one row.  Each thread keeps fp32 column partials;
-// the CTA adds its eight warps' partials in warp order, stores them for its row block,
-// and the last row block of a strip to finish adds all row blocks in order: the result
-// does not depend on the schedule.
+// Grid (column groups, row blocks).  A strip is 32 16-byte vectors of a row; warp w of a
+// CTA takes strip 8·blockIdx.x + w (lane l its l-th vector) and all eight warps walk the
+// same rows of the block, RU rows a trip, so the CTA reads and writes each row as
+// 8·512 contiguous bytes (strips of eight different rows per CTA stream a third slower).
+// Each thread keeps fp32 partial sums of its VE columns over the block's rows and stores
+// them as the block's row of the workspace; fl_bgrad_reduce_kernel then adds the row
+// blocks in a fixed order, so the result does not depend on the schedule.
+// Three CTAs of 256 threads per SM: the loop's four rows of packed vectors, the
+// partial sums and the row pointers fit 85 registers without spills (at four CTAs they spill).
 template <int DT, int MODE>
-__global__ void __launch_bounds__(256, 4) fl_bwd_bgrad_kernel(const BwdParams P) {
+__global__ void __launch_bounds__(256, 3) fl_bwd_bgrad_kernel(const BwdParams P) {
   using T = typename ElemT<DT>::T;
   grid_dependency_wait();
   if (threadIdx.x == 0) grid_launch_dependents();
   constexpr int ESZ = sizeof(T);
   constexpr int VE = 16 / ESZ;  // elements per 16-byte vector
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int strip = blockIdx.x, rb = blockIdx.y;
-  const long long c0 = (long long)strip * 32 * VE + (long long)lane * VE;
+  const long long strip0 = ((long long)blockIdx.x * 8 + warp) * 32 * VE;  // first column of the strip
+  if (strip0 >= P.N) return;  // a strip past the last column (no CTA-wide barrier below)
+  const int rb = blockIdx.y;
+  const long long c0 = strip0 + (long long)lane * VE;
   const long long r0 = (long long)rb * P.rows_per_block;
   const long long r1 = min(P.M, r0 + P.rows_per_block);
+  const bool any = c0 < P.N;
   const bool vec = P.vec_ok && c0 + VE <= P.N;
   const T* grad = reinterpret_cast<const T*>(P.grad);
   const T* vv = reinterpret_cast<const T*>(P.v);
@@ -82,105 +87,121 @@ __global__ void __launch_bounds__(256, 4) fl_bwd_bgrad_kernel(const BwdParams P)
   float part[VE];
 #pragma unroll
   for (int i = 0; i < VE; ++i) part[i] = 0.0f;
-  // four rows a trip (rows m, m+8, m+16, m+24 of this warp): every load of the trip is
-  // in flight before the first use; the vectors stay packed until then
+  // four rows a trip: every load of the trip is in flight before the first use; the
+  // vectors stay packed until then.  Row pointers advance by the pitch (no per-row
+  // 64-bit index products in the loop).
   constexpr int RU = 4;
-  for (long long mb = r0 + warp; mb < r1; mb += 8 * RU) {
+  const char* gp = reinterpret_cast<const char*>(grad + r0 * P.ldg + c0);
+  const char* vp = reinterpret_cast<const char*>(vv + (MODE == BWD_DGELU ? r0 * P.ldv + c0 : 0));
+  char* dp = reinterpret_cast<char*>(dpre + r0 * P.ldd + c0);
+  const uint32_t* mp = P.mask + (MODE == BWD_DRELU ? r0 * P.words + (c0 >> 5) : 0);
+  const long long gs = P.ldg * ESZ, vs = P.ldv * ESZ, ds = P.ldd * ESZ;
+  const int sh = (int)(c0 & 31);
+  for (long long mb = r0; mb < r1 && any; mb += RU) {
+    const int nrow = (int)min((long long)RU, r1 - mb);
     uint4 gq[RU], vq[RU];
     uint32_t word[RU];
 #pragma unroll
     for (int u = 0; u < RU; ++u) {
-      const long long m = mb + 8 * u;
       gq[u] = make_uint4(0u, 0u, 0u, 0u);
       vq[u] = make_uint4(0u, 0u, 0u, 0u);
       word[u] = 0u;
-      if (m >= r1) continue;
+      if (u >= nrow) continue;
       if (vec) {
-        gq[u] = __ldg(reinterpret_cast<const uint4*>(grad + m * P.ldg + c0));
-        if (MODE == BWD_DGELU) vq[u] = __ldg(reinterpret_cast<const uint4*>(vv + m * P.ldv + c0));
+        gq[u] = __ldg(reinterpret_cast<const uint4*>(gp + u * gs));
+        if (MODE == BWD_DGELU) vq[u] = __ldg(reinterpret_cast<const uint4*>(vp + u * vs));
       } else {
         T* ge = reinterpret_cast<T*>(&gq[u]);
         T* ve = reinterpret_cast<T*>(&vq[u]);
 #pragma unroll
         for (int i = 0; i < VE; ++i) {
           if (c0 + i < P.N) {
-            ge[i] = grad[m * P.ldg + c0 + i];
-            if (MODE == BWD_DGELU) ve[i] = vv[m * P.ldv + c0 + i];
+            ge[i] = reinterpret_cast<const T*>(gp + u * gs)[i];
+            if (MODE == BWD_DGELU) ve[i] = reinterpret_cast<const T*>(vp + u * vs)[i];
           }
         }
       }
       // the VE columns lie in one mask word (VE divides 32)
-      if (MODE == BWD_DRELU && c0 < P.N) word[u] = __ldg(P.mask + m * P.words + (c0 >> 5));
+      if (MODE == BWD_DRELU) word[u] = __ldg(mp + u * P.words);
     }
 #pragma unroll
     for (int u = 0; u < RU; ++u) {
-      const long long m = mb + 8 * u;
-      if (m >= r1) continue;
+      if (u >= nrow) continue;
       const T* ge = reinterpret_cast<const T*>(&gq[u]);
       const T* ve = reinterpret_cast<const T*>(&vq[u]);
       float d[VE];
 #pragma unroll
       for (int i = 0; i < VE; ++i) {
         const float gi = static_cast<float>(ge[i]);
-        if (MODE == BWD_DRELU) d[i] = ((word[u] >> ((c0 & 31) + i)) & 1u) ? gi : gi * 0.0f;  // keeps grad's sign
+        if (MODE == BWD_DRELU) d[i] = ((word[u] >> (sh + i)) & 1u) ? gi : gi * 0.0f;  // keeps grad's sign
         else d[i] = gi * gelu_erf_grad_f(static_cast<float>(ve[i]));
       }
+      T* de = reinterpret_cast<T*>(dp + u * ds);
       if (vec) {
         uint4 q;
         T* e = reinterpret_cast<T*>(&q);
 #pragma unroll
         for (int i = 0; i < VE; ++i) e[i] = static_cast<T>(d[i]);
-        *reinterpret_cast<uint4*>(dpre + m * P.ldd + c0) = q;
+        *reinterpret_cast<uint4*>(de) = q;
       } else {
 #pragma unroll
         for (int i = 0; i < VE; ++i)
-          if (c0 + i < P.N) dpre[m * P.ldd + c0 + i] = static_cast<T>(d[i]);
+          if (c0 + i < P.N) de[i] = static_cast<T>(d[i]);
       }
 #pragma unroll
       for (int i = 0; i < VE; ++i) part[i] += d[i];
     }
+    gp += RU * gs;
+    if (MODE == BWD_DGELU) vp += RU * vs;
+    dp += RU * ds;
+    if (MODE == BWD_DRELU) mp += RU * P.words;
   }
-  if (P.dbias == nullptr) return;
-  // ---- bias gradient: the CTA's eight warps in warp order, then the row blocks in order
-  __shared__ float red[8][32 * 8];
-  __shared__ int last;
+  if (P.dbias == nullptr || !any) return;
+  float* dst = P.ws + (long long)rb * P.ws_ld + c0;
+  if (c0 + VE <= P.N) {  // (ws rows and c0 are 16-byte aligned)
 #pragma unroll
-  for (int i = 0; i < VE; ++i) red[warp][lane * VE + i] = part[i];
-  __syncthreads();
-  if (warp == 0) {
+    for (int i = 0; i < VE; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(part[i], part[i + 1], part[i + 2], part[i + 3]);
+  } else {
 #pragma unroll
-    for (int i = 0; i < VE; ++i) {
-      float s = red[0][lane * VE + i];
-#pragma unroll
-      for (int w = 1; w < 8; ++w) s += red[w][lane * VE + i];
-      if (c0 + i < P.N) P.ws[(long long)rb * P.ws_ld + c0 + i] = s;
-    }
-    __threadfence();  // this block's partials before its count
+    for (int i = 0; i < VE; ++i)
+      if (c0 + i < P.N) dst[i] = part[i];
   }
-  __syncthreads();
-  if (threadIdx.x == 0) last = (atomicAdd(P.counters + strip, 1) == P.row_blocks - 1);
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  // every thread of the last block adds one column over the row blocks, in order
-  if (threadIdx.x < 32 * VE) {
-    const long long c = (long long)strip * 32 * VE + threadIdx.x;
-    if (c < P.N) {
-      const float* src = P.ws + c;
-      float s = 0.0f;
-      // sixteen row blocks' loads in flight a trip (this tail runs after all other blocks)
-      for (int b = 0; b < P.row_blocks; b += 16) {
-        float t[16];
+}
+
+// dbias[c] = Σ over the row blocks of ws[rb][c].  A CTA of 32 x 32 threads takes 32
+// columns; thread (g, l) adds row blocks g, g + 32, g + 64, ... of column l in ascending
+// order (all its loads in flight at once for up to 512 row blocks), then thread (0, l)
+// adds the 32 group sums in group order: a fixed order, whatever the schedule.
+// Launched after fl_bwd_bgrad_kernel with programmatic dependent launch; the wait
+// below covers that kernel's stores.
+__global__ void __launch_bounds__(1024, 1) fl_bgrad_reduce_kernel(const float* __restrict__ ws, float* dbias,
+                                                                  long long N, long long ws_ld, int row_blocks) {
+  grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
+  const int g = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const long long c = (long long)blockIdx.x * 32 + l;
+  __shared__ float red[32][33];
+  float s = 0.0f;
+  if (c < N) {
+    for (int b0 = g; b0 < row_blocks; b0 += 32 * 16) {
+      float t[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) t[k] = (b + k < P.row_blocks) ? __ldcg(src + (long long)(b + k) * P.ws_ld) : 0.0f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-          if (b + k < P.row_blocks) s += t[k];
+      for (int k = 0; k < 16; ++k) {
+        const int b = b0 + 32 * k;
+        t[k] = b < row_blocks ? __ldcg(ws + (long long)b * ws_ld + c) : 0.0f;
       }
-      P.dbias[c] = s;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) s += t[k];
     }
   }
-  if (threadIdx.x == 0) P.counters[strip] = 0;  // ready for the next launch
+  red[g][l] = s;
+  __syncthreads();
+  if (g == 0 && c < N) {
+    float r = red[0][l];
+#pragma unroll
+    for (int k = 1; k < 32; ++k) r += red[k][l];
+    dbias[c] = r;
+  }
 }
 
 // ---------------------------------------------------------------- LayerNorm after the tail
@@ -413,7 +434,11 @@ __global__ void __launch_bounds__(TPB, TPB == 128 ? 6 : 3) fl_layernorm_kernel(c
 // with 16-byte row pitches, N a multiple of the vector width and at most TPB·VMAX
 // vectors.  Column offsets are 32-bit, the validity of each of a thread's vectors is
 // fixed for the whole launch, and every access is a whole vector, which keeps the
-// instruction count per element small.  Rows are prefetched as in fl_layernorm_kernel.
+// instruction count per element small.  Each thread keeps its vectors of the CTA's next
+// LN_DEPTH rows in flight (one cp.async group per row, in LN_DEPTH shared-memory slots).
+// (Two rows deep measured slower on 2048 x 4096 fp32: 15.7 vs 13.4 us; the second slot
+// doubles the shared memory of a CTA.)
+constexpr int LN_DEPTH = 1;  // rows a CTA of the vector LayerNorm keeps in flight
 template <int XT, int ZT, int TPB>
 __global__ void __launch_bounds__(TPB, TPB == 128 ? 6 : 3) fl_layernorm_vec_kernel(const LnParams P) {
   using TX = typename ElemT<XT>::T;
@@ -424,27 +449,36 @@ __global__ void __launch_bounds__(TPB, TPB == 128 ? 6 : 3) fl_layernorm_vec_kern
   constexpr int NW = TPB / 32;
   constexpr int EZ = (ZT == DT_F32) ? 4 : 2;
   __shared__ float red[NW];
-  __shared__ __align__(16) uint4 stage[VMAX * TPB];
+  __shared__ __align__(16) uint4 stage[LN_DEPTH][VMAX * TPB];
   const int t = threadIdx.x;
   const int nvec = (int)(P.N / VE);
   const float inv_n = 1.0f / (float)P.N;
   const uint32_t stage_base = (uint32_t)__cvta_generic_to_shared(stage);
-  auto prefetch = [&](long long m) {
+  // copy this thread's vectors of row m into slot `slot` (the caller commits the group)
+  auto prefetch = [&](long long m, int slot) {
     const uint4* x = reinterpret_cast<const uint4*>(reinterpret_cast<const TX*>(P.x) + m * P.ldx);
 #pragma unroll
     for (int k = 0; k < VMAX; ++k)
-      if (k * TPB + t < nvec) cp_async_16(stage_base + (uint32_t)(k * TPB + t) * 16u, x + k * TPB + t, 16u);
-    cp_async_commit();
+      if (k * TPB + t < nvec)
+        cp_async_16(stage_base + (uint32_t)((slot * VMAX + k) * TPB + t) * 16u, x + k * TPB + t, 16u);
   };
-  if (blockIdx.x < P.M) prefetch(blockIdx.x);
+  // one group per row slot, empty past the last row, so that at the row of iteration i
+  // exactly LN_DEPTH - 1 younger groups exist
+#pragma unroll
+  for (int d = 0; d < LN_DEPTH; ++d) {
+    const long long m = blockIdx.x + (long long)d * gridDim.x;
+    if (m < P.M) prefetch(m, d);
+    cp_async_commit();
+  }
+  int slot = 0;
   for (long long m = blockIdx.x; m < P.M; m += gridDim.x) {
     float xv[VMAX][VE];
-    cp_async_wait<0>();
+    cp_async_wait<LN_DEPTH - 1>();  // this row's group has landed
     float s = 0.0f;
 #pragma unroll
     for (int k = 0; k < VMAX; ++k) {
       if (k * TPB + t < nvec) {
-        const uint4 q = stage[k * TPB + t];
+        const uint4 q = stage[slot][k * TPB + t];
         const TX* e = reinterpret_cast<const TX*>(&q);
 #pragma unroll
         for (int i = 0; i < VE; ++i) xv[k][i] = static_cast<float>(e[i]);
@@ -455,7 +489,11 @@ __global__ void __launch_bounds__(TPB, TPB == 128 ? 6 : 3) fl_layernorm_vec_kern
 #pragma unroll
       for (int i = 0; i < VE; ++i) s += xv[k][i];
     }
-    if (m + gridDim.x < P.M) prefetch(m + gridDim.x);  // the slots' values are used above
+    // the slot's values are used above: refill it with the row LN_DEPTH rows ahead
+    const long long mn = m + (long long)LN_DEPTH * gridDim.x;
+    if (mn < P.M) prefetch(mn, slot);
+    cp_async_commit();
+    slot = (slot + 1 == LN_DEPTH) ? 0 : slot + 1;
     const float mean = block_sum<NW>(s, red) * inv_n;
     float q = 0.0f;
 #pragma unroll

@@ -177,8 +177,9 @@ fl_status fl_relu_backward(const void* grad, const uint32_t* aux, void* dpre, in
  *   aux            [M, ceil(N/32)] uint32 packed mask (4-byte aligned)
  *   dbias          [N] fp32, or null (then no workspace is needed)
  *   workspace      fl_bias_grad_workspace_size bytes, 16-byte aligned, owned by the
- *                  caller and zero-filled once before its first use; every call leaves
- *                  it ready for the next.  Calls that overlap on the GPU must not share it.
+ *                  caller (no initial contents needed): one row of fp32 column partial
+ *                  sums per block of rows, which a second kernel adds in a fixed order.
+ *                  Calls that overlap on the GPU must not share it.
  * dpre may alias grad.  Errors: FL_ERR_INVALID_ARG (null operand, negative size, ld < N,
  * workspace missing or too small), FL_ERR_ALIGNMENT, FL_ERR_CUDA. */
 fl_status fl_bias_grad_workspace_size(int64_t M, int64_t N, int32_t dtype, size_t* bytes);
