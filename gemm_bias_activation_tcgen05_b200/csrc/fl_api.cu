@@ -1277,8 +1277,7 @@ static void (*ln_kernel(bool vec))(LnParams) {
   return vec ? fl_layernorm_vec_kernel<XT, ZT, TPB> : fl_layernorm_kernel<XT, ZT, TPB>;
 }
 
-// 128 threads per row when the row fits their registers (32 elements a thread).  The
-// kernel loops over rows: the grid is one resident wave, or M CTAs if fewer.
+// The kernel loops over rows: the grid is one resident wave, or M CTAs if fewer.
 template <int XT, int TPB>
 static cudaError_t launch_ln_w(int z_dtype, cudaStream_t s, const LnParams& P) {
   int dev = 0, sms = 148, per_sm = 0;
@@ -1298,9 +1297,12 @@ static cudaError_t launch_ln_w(int z_dtype, cudaStream_t s, const LnParams& P) {
   return launch_pdl_b(k, dim3((unsigned)std::min<long long>(P.M, wave)), TPB, s, P);
 }
 
+// Rows of up to 8 KB take 128 threads (32 elements a thread); longer rows 256 (on
+// 2048 x 4096 fp32 rows, 256 threads measured 11.2 us against 13.3 us for 128).
 template <int XT>
 static cudaError_t launch_ln(int z_dtype, cudaStream_t s, const LnParams& P) {
-  if (P.N <= 128 * 32) return launch_ln_w<XT, 128>(z_dtype, s, P);
+  const long long row_bytes = P.N * (XT == DT_F32 ? 4 : 2);
+  if (P.N <= 128 * 32 && row_bytes <= 8192) return launch_ln_w<XT, 128>(z_dtype, s, P);
   return launch_ln_w<XT, 256>(z_dtype, s, P);
 }
 
