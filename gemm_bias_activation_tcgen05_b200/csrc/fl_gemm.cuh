@@ -270,48 +270,22 @@ __device__ __noinline__ void sk_store_partial(const KParams& p, uint32_t tacc, i
                                         __uint_as_float(r[4 * j4 + 2]), __uint_as_float(r[4 * j4 + 3])));
   }
 }
-// The partials of clusters w0..w1, summed in that order, into the idle accumulator buffer
-// at `tspare` (same column layout as the accumulator), block by block: run while the tile's
-// own K blocks still accumulate in the other buffer.
-__device__ __noinline__ void sk_load_partials(const KParams& p, uint32_t tspare, int c_begin, int gblk, int cta_rank,
-                                              int kcl, int ew, int w0, int w1, int lane) {
-  const int nb = p.mma_n / 64;
-  float x[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) x[j] = 0.0f;
-#pragma unroll 1
-  for (int w = w0; w <= w1; ++w) sk_add_block(x, sk_area(p, w, cta_rank, kcl, ew), 0, lane);
-#pragma unroll 1
-  for (int b = 0; b < nb; ++b) {
-    // the next block's partials are read before this block goes to TMEM
-    float y[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) y[j] = 0.0f;
-    if (b + 1 < nb) {
-#pragma unroll 1
-      for (int w = w0; w <= w1; ++w) sk_add_block(y, sk_area(p, w, cta_rank, kcl, ew), b + 1, lane);
-    }
-    const int col = b < gblk ? c_begin + 32 * b : p.out_tile_n + c_begin + 32 * (b - gblk);
-    uint32_t r[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(x[j]);
-    tmem_st32(tspare + (uint32_t)col, r);
-#pragma unroll
-    for (int j = 0; j < 32; ++j) x[j] = y[j];
-  }
-  tmem_wait_st();
-}
-// acc += the summed partials at `tspare`, in TMEM only
-__device__ __noinline__ void sk_add_spare(const KParams& p, uint32_t tacc, uint32_t tspare, int c_begin, int gblk) {
+// acc += the partials of clusters w0..w1 (in that order), block by block in TMEM
+__device__ __noinline__ void sk_add_partials(const KParams& p, uint32_t tacc, int c_begin, int gblk, int cta_rank,
+                                             int kcl, int ew, int w0, int w1, int lane) {
 #pragma unroll 1
   for (int b = 0; b < p.mma_n / 64; ++b) {
     const int col = b < gblk ? c_begin + 32 * b : p.out_tile_n + c_begin + 32 * (b - gblk);
-    uint32_t r[32], q[32];
+    uint32_t r[32];
     tmem_ld32(tacc + (uint32_t)col, r);
-    tmem_ld32(tspare + (uint32_t)col, q);
     tmem_wait_ld();
+    float x[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) + __uint_as_float(q[j]));
+    for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(r[j]);
+#pragma unroll 1
+    for (int w = w0; w <= w1; ++w) sk_add_block(x, sk_area(p, w, cta_rank, kcl, ew), b, lane);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(x[j]);
     tmem_st32(tacc + (uint32_t)col, r);
   }
   tmem_wait_st();
@@ -955,24 +929,6 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
         const int n_tile0 = tb * p.out_tile_n;
         const int c_begin = half * half_cols;
         const int c_end = c_begin + half_cols;
-        const int gblk = half_cols / 32;  // 32-column blocks of this warp's (gate) columns
-        const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16);  // this warp's TMEM lane quarter
-        if (itm.kind == IT_FINISH) {
-          // stream-K: the partials of the clusters whose ranges start inside this tile are
-          // summed (in cluster order) into the other accumulator buffer, idle since this is the
-          // cluster's last item, while the tile's own K blocks still run; after the
-          // accumulator barrier a TMEM-only add folds them in
-          for (int w = itm.w0; ok && w <= itm.w1; ++w)
-            if (!warp_wait_flag(p.sk_flags + (w * kCl + (int)rank) * kEpiWarps + ew, p, lane)) ok = false;
-          if (!ok) break;
-          if (ew == 0 && lane == 0) FL_STAMP(16);
-          sk_load_partials(p, tq + (buf ^ 1u) * (uint32_t)p.mma_n, c_begin, gblk, (int)rank, kCl, ew, itm.w0, itm.w1,
-                           lane);
-          // every lane has read the partials: the flags are ready for the next launch
-          __syncwarp();
-          if (lane == 0)
-            for (int w = itm.w0; w <= itm.w1; ++w) p.sk_flags[(w * kCl + (int)rank) * kEpiWarps + ew] = 0;
-        }
         // ---- operands that do not depend on the accumulator, read before its barrier so
         // that their latency overlaps the main loop: the bias (per row; or lane l holds the
         // bias of columns c_begin + 32h + l of the tile), and the first chunk of a 16-bit
@@ -998,7 +954,8 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           if (local == 0) FL_STAMP(6);
           FL_STAMP(8);
         }
-        const uint32_t tacc = tq + buf * (uint32_t)p.mma_n;
+        const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)p.mma_n;
+        const int gblk = half_cols / 32;  // 32-column blocks of this warp's (gate) columns
         if (itm.kind == IT_PARTIAL) {
           // stream-K: this cluster's range starts inside the tile.  Store this warp's fp32
           // accumulator columns for the tile's finisher, free the TMEM buffer, then release
@@ -1017,8 +974,19 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           continue;
         }
         if (itm.kind == IT_FINISH) {
-          sk_add_spare(p, tacc, tq + (buf ^ 1u) * (uint32_t)p.mma_n, c_begin, gblk);
+          // stream-K: add the partials of the clusters whose ranges start inside this tile
+          // (in cluster order) to this warp's accumulator columns in tensor memory; the
+          // epilogue below then reads the whole tile's sums
+          for (int w = itm.w0; ok && w <= itm.w1; ++w)
+            if (!warp_wait_flag(p.sk_flags + (w * kCl + (int)rank) * kEpiWarps + ew, p, lane)) ok = false;
+          if (!ok) break;
+          if (ew == 0 && lane == 0) FL_STAMP(16);
+          sk_add_partials(p, tacc, c_begin, gblk, (int)rank, kCl, ew, itm.w0, itm.w1, lane);
           if (ew == 0 && lane == 0) FL_STAMP(17);
+          // every lane has read the partials: the flags are ready for the next launch
+          __syncwarp();
+          if (lane == 0)
+            for (int w = itm.w0; w <= itm.w1; ++w) p.sk_flags[(w * kCl + (int)rank) * kEpiWarps + ew] = 0;
         }
 
         // The warp's columns as 32-column blocks in a rolled loop: a block's accumulator,
