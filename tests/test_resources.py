@@ -89,8 +89,8 @@ def test_vector_layernorm_keeps_six_ctas_of_128():
 def test_launchable_fused_kernels_do_not_spill():
     # Every instantiation of the fused kernel that a plan can launch keeps its epilogue in
     # registers: at most 16 bytes of spill stores and loads together (a register save or
-    # two).  GeGLU with an
-    # fp32 output (act 4, out 2) is rejected by fl_plan and never launched.  A change that
+    # two).  GeGLU with an fp32 output (act 4, out 2) is rejected by fl_plan and never
+    # launched.  A change that
     # pushes one of these over the 168-register budget showed up as a slower whole-tile
     # schedule (tail_m2048 65.9 -> 70.9 us with 100 bytes of spills).
     e = _select(_entries(), "_ZN2fl19fl_gemm_epi_tcgen05")
