@@ -424,18 +424,19 @@ static fl_status choose_config(fl_plan_s* p) {
     } else {
       // Pick the N tile that minimises (waves x tile width) on this GPU.
       // Cost ~ (rounds of tiles per SM) x (tile width) x (relative cost per column):
-      // a 128-wide UMMA tile moves more operand bytes per FLOP and issues twice
-      // the instructions, measured at about 1.6x the per-column cost of 256.
-      // With stream-K (CTA pairs) the rounds are fractional: the last, partial round is
-      // spread over every pair.
+      // narrower UMMA tiles move more operand bytes per FLOP and issue more instructions
+      // per column; measured against 256 on a B200: 192 about 1.2-1.3x per column (a
+      // 192-wide tile of a 16-bit output stores its warps' last 32 columns without TMA),
+      // 128 about 1.5-1.6x.  With stream-K (CTA pairs) the rounds are fractional: the last,
+      // partial round is spread over every pair.
       const bool sk_ok = p->pair && !p->no_sk;
       int best = 256;
       double best_cost = 1e300;
-      for (int bn : {256, 128}) {
+      for (int bn : {256, 192, 128}) {
         const int64_t tiles = cdiv(M, rows) * cdiv(N, bn);
         const bool sk = sk_ok && stream_k_pays(tiles, units, p->num_kb, p->epi.schedule);
         const double waves = sk ? (double)tiles / units : (double)cdiv(tiles, units);
-        const double cost = waves * bn * (bn == 128 ? 1.6 : 1.0);
+        const double cost = waves * bn * (bn == 128 ? 1.6 : bn == 192 ? 1.25 : 1.0);
         if (cost < best_cost) { best_cost = cost; best = bn; }
       }
       p->mma_n = best;

@@ -1011,7 +1011,11 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           const int cb = c_begin + 32 * b;         // TMEM column (and tile column) of the block
           const int nc0 = n_tile0 + cc;
           const int n0 = n_tile0 + cb;              // the block's first output column
-          const bool tma_chunk = nc0 < p.n_tma;
+          // a chunk that reaches past this warp's columns (a 192-wide tile's last 32 columns of
+          // a 16-bit output) is not stored by TMA: its 64-column box would cover the other
+          // warp's columns.  Its block goes out by 16-byte stores from registers.
+          const bool full_chunk = cc + CH <= c_end;
+          const bool tma_chunk = nc0 < p.n_tma && full_chunk;
           if (hh == 0 && tma_chunk) {
             if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read the staging row
             if (ew == 0 && lane == 0 && b == 0) FL_STAMP(25);
@@ -1095,6 +1099,24 @@ __global__ void __launch_bounds__(Cfg<SWAP>::kThreads, 1)
           if (ew == 0 && lane == 0 && b == 0) FL_STAMP(24);
           // ---- ragged row end: a TMA store writes whole 16-byte granules, so the
           // columns past the last full granule are written with plain stores.
+          if (!full_chunk && m_ok && n0 < p.n_tma) {
+            // every whole 16-byte granule below n_tma (the columns from n_tma on follow below)
+            constexpr int EPG = (OUT == DT_F32) ? 4 : 8;  // elements per granule
+            char* dst = reinterpret_cast<char*>(p.out) + ((long long)m * p.ldo + n0) * (OUT == DT_F32 ? 4 : 2);
+#pragma unroll
+            for (int c = 0; c < GPB; ++c) {
+              if (n0 + (c + 1) * EPG > p.n_tma) break;
+              uint32_t w4[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                if constexpr (OUT == DT_F32) w4[k] = __float_as_uint(v[4 * c + k]);
+                else w4[k] = pack2<OUT>(v[8 * c + 2 * k], v[8 * c + 2 * k + 1]);
+              }
+              asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 16 * c), "r"(w4[0]), "r"(w4[1]),
+                           "r"(w4[2]), "r"(w4[3])
+                           : "memory");
+            }
+          }
           if (n0 + 32 > p.n_tma && n0 < p.N && m_ok) {
             const int j0 = max(p.n_tma - n0, 0);
             const int j1 = min(p.N - n0, 32);

@@ -68,6 +68,20 @@ def test_epilogues_ragged(fl, epilogue, out_dtype):
     _linear_case(fl, 300, 520, 200, epilogue=epilogue, out_dtype=out_dtype, seed=11)
 
 
+@pytest.mark.parametrize("epilogue,out_dtype,dtype", [("RELU_AUX_BIAS", "bf16", "bf16"),
+                                                       ("GELU_TANH_BIAS", "f16", "f16"),
+                                                       ("GELU_BIAS", "f32", "bf16")])
+def test_192_wide_tiles(fl, epilogue, out_dtype, dtype):
+    # 1000 x 2568: 192-wide pair tiles are the cheapest (56 tiles in one round, against 84
+    # 128-wide ones).  With a 16-bit output each warp's last 32 columns of a tile go out by
+    # direct stores instead of TMA, and the last column tile (72 wide) ends inside those 32
+    import gemm_bias_activation_tcgen05_b200 as m
+    info = m.fl_plan_preview(1000, 2568, 200, dtype, kind=epilogue, out_dtype=out_dtype)
+    assert info["tile_n"] == 192 and info["cta_pair"] == 1, info
+    _linear_case(fl, 1000, 2568, 200, dtype=dtype, epilogue=epilogue, out_dtype=out_dtype, seed=17,
+                 bias_dtype="f32" if out_dtype == "f32" else dtype)
+
+
 def test_fp16_operands(fl):
     _linear_case(fl, 257, 264, 136, dtype="f16", epilogue="GELU_TANH_BIAS", out_dtype="f16", bias_dtype="f16")
 
