@@ -425,6 +425,12 @@ def run_ours(args):
         roof_t = max(w.flops / (pk["bf16_tflops"] * 1e12), suite.min_bytes[w.name] / (pk["hbm_gbs"] * 1e9))
         breakdown[w.name] = {"us": round(t * 1e3, 2), "tflops": round(tfl, 1), "gbs_min_bytes": round(gbs, 1),
                              "roofline_us": round(roof_t * 1e6, 2), "roofline_frac": round(roof_t / (t * 1e-3), 3)}
+    # each workload's launches alone, as the time they add to a stream (L2 flushed before each)
+    flush_b = L2Flush()
+    for it in suite.items:
+        fn = lambda it=it: suite.run_item(it, torch.cuda.current_stream().cuda_stream)  # noqa: E731
+        breakdown[it["w"].name]["us_in_stream"] = round(time_in_stream(fn, 20, flush_b) * 1e3, 2)
+    del flush_b
     dom = suite.items[[it["w"].name for it in suite.items].index(DOMINANT)]
     dom_w = dom["w"]
     # the dominant fused GEMM launch alone (its dReLU follows inside the same event pair,
