@@ -73,14 +73,22 @@ def poison(shape, dtype: str, device="cuda") -> torch.Tensor:
 
 def run_linear(fl, *, M, N, K, dtype, epilogue, out_dtype, A, W, bias=None, bias_dtype="bf16",
                bias_axis=0, b_major=0, residual=None, residual_dtype="bf16", scale=1.0,
-               unfused=False, out_pad=8, stream=None, check_canary=True, schedule="auto") -> Dict[str, np.ndarray]:
+               unfused=False, out_pad=8, stream=None, check_canary=True, schedule="auto",
+               bias_offset=0) -> Dict[str, np.ndarray]:
     """Run one layer; A/W/bias/residual are CPU tensors in (padded) storage.
+
+    bias_offset > 0 places the bias that many elements into its device buffer (a pointer
+    off the 16-byte grid for odd offsets).
 
     Returns the logical [M, N] output and the aux mask as numpy arrays.
     """
     dev = "cuda"
     dA, dW = A.to(dev), W.to(dev)
-    dB = bias.to(dev) if bias is not None else None
+    dB = None
+    if bias is not None:
+        buf = torch.zeros(bias.numel() + bias_offset, dtype=bias.dtype, device=dev)
+        dB = buf[bias_offset:]
+        dB.copy_(bias.to(dev))
     dR = residual.to(dev) if residual is not None else None
     ldo = -(-N // out_pad) * out_pad
     out = poison((M, ldo), out_dtype)

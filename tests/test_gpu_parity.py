@@ -27,7 +27,8 @@ def fl():
 
 
 def _linear_case(fl, M, N, K, *, dtype="bf16", epilogue="GELU_BIAS", out_dtype="bf16", bias_axis=0,
-                 residual=False, scale=1.0, b_major=0, seed=0, bias_dtype=None, unfused=False, schedule="auto"):
+                 residual=False, scale=1.0, b_major=0, seed=0, bias_dtype=None, unfused=False, schedule="auto",
+                 bias_offset=0):
     bias_dtype = bias_dtype or ("f32" if dtype == "f32" else dtype)
     has_bias = epilogue not in ("NONE",)
     inp = workloads.ragged_linear_inputs(M, N, K, dtype, seed, bias_dtype=bias_dtype if has_bias else None,
@@ -36,11 +37,11 @@ def _linear_case(fl, M, N, K, *, dtype="bf16", epilogue="GELU_BIAS", out_dtype="
     got = P.run_linear(fl, M=M, N=N, K=K, dtype=dtype, epilogue=epilogue, out_dtype=out_dtype, A=inp["A"],
                        W=W, bias=inp.get("bias"), bias_dtype=bias_dtype, bias_axis=bias_axis, b_major=b_major,
                        residual=inp.get("residual"), residual_dtype=dtype, scale=scale, unfused=unfused,
-                       schedule=schedule)
+                       schedule=schedule, bias_offset=bias_offset)
     y, aux, v, absdot = P.oracle_linear(A=inp["A"], W=W, bias=inp.get("bias"), bias_axis=bias_axis,
                                         b_major=b_major, residual=inp.get("residual"), scale=scale,
                                         epilogue=epilogue, out_dtype=out_dtype, M=M, N=N, K=K)
-    what = f"{epilogue} {dtype}->{out_dtype} M{M} N{N} K{K} info={got['info']}"
+    what = f"{epilogue} {dtype}->{out_dtype} M{M} N{N} K{K} bias+{bias_offset} info={got['info']}"
     P.check_close(got["out"], y, out_dtype, absdot, what)
     if epilogue == "RELU_AUX_BIAS":
         margin = None
@@ -80,6 +81,16 @@ def test_192_wide_tiles(fl, epilogue, out_dtype, dtype):
     assert info["tile_n"] == 192 and info["cta_pair"] == 1, info
     _linear_case(fl, 1000, 2568, 200, dtype=dtype, epilogue=epilogue, out_dtype=out_dtype, seed=17,
                  bias_dtype="f32" if out_dtype == "f32" else dtype)
+
+
+@pytest.mark.parametrize("bias_dtype", ["bf16", "f16", "f32"])
+@pytest.mark.parametrize("bias_offset", [0, 1, 8])
+@pytest.mark.parametrize("M,epilogue", [(200, "GELU_TANH_BIAS"), (100, "RELU_AUX_BIAS")])
+def test_bias_alignment(fl, bias_dtype, bias_offset, M, epilogue):
+    # a per-column bias on and off the 16-byte grid, over whole and ragged 32-column
+    # blocks (N = 300), on CTA pairs and single CTAs
+    _linear_case(fl, M, 300, 136, epilogue=epilogue, out_dtype="bf16", bias_dtype=bias_dtype,
+                 bias_offset=bias_offset, seed=21)
 
 
 def test_fp16_operands(fl):
