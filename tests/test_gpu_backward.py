@@ -176,7 +176,9 @@ def _ln_check(got, x64, g64, b64, eps, out_dtype, what):
     (16, 6000, "bf16", "f32", "bf16", 1e-5), (9, 5000, "f32", "f16", "f32", 1e-5), (3, 4097, "f32", "f32", "f32", 1e-5),
     # more rows than one resident wave: CTAs loop over rows (prefetching the next when aligned)
     (3000, 1032, "bf16", "f16", "f32", 1e-5), (4000, 300, "bf16", "bf16", "bf16", 1e-5),
-    (1200, 4100, "f32", "f32", "f32", 1e-5), (2000, 6000, "bf16", "bf16", "f32", 1e-5)])
+    (1200, 4100, "f32", "f32", "f32", 1e-5), (2000, 6000, "bf16", "bf16", "f32", 1e-5),
+    # whole vectors in warp 0 alone (the statistics merge warps without elements)
+    (256, 40, "f32", "f32", "f32", 1e-5)])
 def test_layernorm(fl, M, N, x_dtype, z_dtype, p_dtype, eps):
     g = torch.Generator().manual_seed(M + N)
     x = (torch.randn(M, N, generator=g) * 2 + 0.7).to(P.TD[x_dtype])
@@ -187,6 +189,22 @@ def test_layernorm(fl, M, N, x_dtype, z_dtype, p_dtype, eps):
     torch.cuda.synchronize()
     _ln_check(P.to64(z), P.to64(x), P.to64(gamma)[None, :], P.to64(beta)[None, :], eps, z_dtype,
               f"LN {M}x{N} {x_dtype}->{z_dtype}")
+
+
+@pytest.mark.parametrize("M,N", [(600, 4096), (300, 1000)])
+def test_layernorm_large_offset(fl, M, N):
+    # |μ|/σ ≈ 6000 per row: the per-warp two-pass sums and their merge keep the variance
+    g = torch.Generator().manual_seed(N)
+    x = torch.randn(M, N, generator=g, dtype=torch.float64) * 0.05 + 300.0
+    x += torch.linspace(-20.0, 20.0, M, dtype=torch.float64)[:, None]
+    x = x.float()
+    gamma = (torch.rand(N, generator=g) + 0.5).float()
+    beta = torch.randn(N, generator=g).float()
+    z = P.poison((M, N), "bf16")
+    fl.fl_layernorm(x.cuda(), gamma.cuda(), beta.cuda(), z, M, N, "f32", "bf16", "f32", eps=1e-5)
+    torch.cuda.synchronize()
+    _ln_check(P.to64(z), P.to64(x), P.to64(gamma)[None, :], P.to64(beta)[None, :], 1e-5, "bf16",
+              f"LN {M}x{N} offset 300")
 
 
 def test_layernorm_in_place_without_affine(fl):
