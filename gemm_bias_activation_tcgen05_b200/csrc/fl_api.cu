@@ -859,6 +859,7 @@ static fl_status launch_gemm(fl_plan_s* p, const GemmArgs& g, cudaStream_t strea
   k.wait_limit_ns = p->wait_limit_ns;
   k.sk_tiles = p->sk_tiles;
   k.sk_clusters = p->sk_clusters;
+  set_dp_split(k, p->grid / (p->pair ? 2 : std::max(1, p->split_k)));
   k.sk_ws = p->d_skws;
   k.sk_flags = p->d_skflags;
 

@@ -105,6 +105,9 @@ struct KParams {
   // stream-K: the last sk_tiles tiles of the tile order are split along K into
   // sk_clusters contiguous ranges of (tile, K-block) units (0: data-parallel only)
   int sk_tiles, sk_clusters;
+  // the data-parallel tiles (all but the stream-K ones) over the launch's clusters:
+  // quotient and remainder, so that a cluster's count needs no division on the device
+  int dp_q, dp_r;
   float* sk_ws;   // fp32 partial accumulators: [cluster][CTA rank][epilogue warp][mma_n/2 x 32]
   int* sk_flags;  // [cluster][CTA rank][epilogue warp]: 1 once that warp's partial is stored
 };
@@ -127,12 +130,20 @@ struct Item {
 __host__ __device__ __forceinline__ int sk_start(const KParams& p, int c) {
   return (int)((long long)p.sk_tiles * p.num_kb * c / p.sk_clusters);
 }
-// Item i of cluster `cl` of `ncl` (false past the last); data-parallel tiles cover the K
-// blocks [kb_a, kb_b).  Stateless, so that a role keeps only its item counter live.
+// dp_q, dp_r of a launch of `ncl` clusters (set on the host beside the grid).
+__host__ __device__ inline void set_dp_split(KParams& p, int ncl) {
+  const int dp_tiles = p.tiles_a * p.tiles_b - p.sk_tiles;
+  p.dp_q = dp_tiles / ncl;
+  p.dp_r = dp_tiles % ncl;
+}
+// Item i of cluster `cl` (0 <= cl < ncl) of `ncl` (false past the last); data-parallel
+// tiles cover the K blocks [kb_a, kb_b).  Stateless, so that a role keeps only its item
+// counter live.  Cluster cl holds the data-parallel tiles cl, cl + ncl, ...: dp_q of
+// them, one more when cl < dp_r.
 __host__ __device__ __forceinline__ bool get_item(const KParams& p, int cl, int ncl, int kb_a, int kb_b, int i,
                                                   Item& it) {
   const int dp_tiles = p.tiles_a * p.tiles_b - p.sk_tiles;
-  const int n_dp = dp_tiles > cl ? (dp_tiles - cl + ncl - 1) / ncl : 0;
+  const int n_dp = p.dp_q + (cl < p.dp_r ? 1 : 0);
   it.w0 = 0;
   it.w1 = -1;
   if (i < n_dp) {

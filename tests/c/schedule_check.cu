@@ -31,6 +31,7 @@ static int check(int tiles_a, int tiles_b, int nkb, int sk, int skc, int ncl) {
   p.num_kb = nkb;
   p.sk_tiles = sk;
   p.sk_clusters = skc;
+  fl::set_dp_split(p, ncl);
   const int T = tiles_a * tiles_b;
   std::vector<int> cover((size_t)T * nkb, 0), finisher(T, -1), nfinish(T, 0);
   std::vector<std::vector<int>> writers(T), listed(T);
