@@ -108,6 +108,7 @@ struct KParams {
   // the data-parallel tiles (all but the stream-K ones) over the launch's clusters:
   // quotient and remainder, so that a cluster's count needs no division on the device
   int dp_q, dp_r;
+  float inv_group;  // 1 / (8 * tiles_b): the tile raster's group size, inverted on the host
   float* sk_ws;   // fp32 partial accumulators: [cluster][CTA rank][epilogue warp][mma_n/2 x 32]
   int* sk_flags;  // [cluster][CTA rank][epilogue warp]: 1 once that warp's partial is stored
 };
@@ -130,11 +131,13 @@ struct Item {
 __host__ __device__ __forceinline__ int sk_start(const KParams& p, int c) {
   return (int)((long long)p.sk_tiles * p.num_kb * c / p.sk_clusters);
 }
-// dp_q, dp_r of a launch of `ncl` clusters (set on the host beside the grid).
+// dp_q, dp_r of a launch of `ncl` clusters and the raster's inverse group size (set on
+// the host beside the grid).
 __host__ __device__ inline void set_dp_split(KParams& p, int ncl) {
   const int dp_tiles = p.tiles_a * p.tiles_b - p.sk_tiles;
   p.dp_q = dp_tiles / ncl;
   p.dp_r = dp_tiles % ncl;
+  p.inv_group = 1.0f / (float)(8 * (p.tiles_b > 0 ? p.tiles_b : 1));
 }
 // Item i of cluster `cl` (0 <= cl < ncl) of `ncl` (false past the last); data-parallel
 // tiles cover the K blocks [kb_a, kb_b).  Stateless, so that a role keeps only its item
@@ -389,17 +392,27 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   }
 }
 
-__device__ __forceinline__ void tile_coords(int t, const KParams& p, int& ta, int& tb) {
+__host__ __device__ __forceinline__ void tile_coords(int t, const KParams& p, int& ta, int& tb) {
   // Grouped raster: 8 A-side tiles per group, B-side swept inside the group,
-  // so concurrently resident CTAs share operand panels in L2.
+  // so concurrently resident CTAs share operand panels in L2.  No integer division on
+  // the way (it runs at every tile boundary): the group index is t times the host's
+  // inverse group size, truncated and corrected by one step either way (exact for
+  // t < 2^24), and a full group of 8 splits r by shifts.
   constexpr int G = 8;
   const int group_size = G * p.tiles_b;
-  const int g = t / group_size;
+  int g = (int)((float)t * p.inv_group);
+  if (g * group_size > t) --g;
+  if ((g + 1) * group_size <= t) ++g;
   const int first = g * G;
-  const int ga = min(G, p.tiles_a - first);
   const int r = t - g * group_size;
-  ta = first + r % ga;
-  tb = r / ga;
+  const int ga = p.tiles_a - first;
+  if (ga >= G) {
+    ta = first + (r & (G - 1));
+    tb = r >> 3;
+  } else {
+    ta = first + r % ga;
+    tb = r / ga;
+  }
 }
 
 // Pinned read-only global loads: volatile with a memory clobber, so a batch of

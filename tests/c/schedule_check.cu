@@ -10,6 +10,7 @@
 //   * a FINISH item's writers all have higher cluster indices.
 // Prints "schedule ok: N cases" and exits 0, or the first violation and exits 1.
 #include <cstdio>
+#include <algorithm>
 #include <cstdlib>
 #include <vector>
 
@@ -78,8 +79,33 @@ static int check(int tiles_a, int tiles_b, int nkb, int sk, int skc, int ncl) {
   return 0;
 }
 
+// The kernel's tile raster (division-free) against the plain formula: group g of 8 A-side
+// tiles, B-side swept inside it, and every tile exactly once.
+static int check_coords(int tiles_a, int tiles_b) {
+  KParams p{};
+  p.tiles_a = tiles_a;
+  p.tiles_b = tiles_b;
+  fl::set_dp_split(p, 1);
+  const int T = tiles_a * tiles_b;
+  std::vector<char> seen((size_t)T, 0);
+  for (int t = 0; t < T; ++t) {
+    int ta, tb;
+    fl::tile_coords(t, p, ta, tb);
+    const int gs = 8 * tiles_b, g = t / gs, first = 8 * g, ga = std::min(8, tiles_a - first), r = t - g * gs;
+    if (ta != first + r % ga || tb != r / ga) return fail("tile coordinates", tiles_a, tiles_b, t);
+    if (seen[(size_t)ta * tiles_b + tb]++) return fail("tile visited twice", tiles_a, tiles_b, t);
+  }
+  return 0;
+}
+
 int main() {
   int cases = 0;
+  for (int a = 1; a <= 40; ++a)
+    for (int b = 1; b <= 40; ++b)
+      if (check_coords(a, b)) return 1;
+  const int big[][2] = {{2048, 3}, {7, 4099}, {600, 600}, {4096, 16}, {33, 1025}, {9, 1}};
+  for (const auto& s : big)
+    if (check_coords(s[0], s[1])) return 1;
   // the synthetic workloads on 74 CTA pairs (tiles_a, tiles_b, K blocks, stream-K tiles,
   // stream-K pairs, pairs launched), as fl_plan splits them
   const int known[][6] = {{16, 16, 32, 108, 74, 74},  // 4096^3: 34 left over plus one round
@@ -112,6 +138,6 @@ int main() {
       ++cases;
     }
   }
-  std::printf("schedule ok: %d cases\n", cases);
+  std::printf("schedule ok: %d cases, tile raster on 1606 grids\n", cases);
   return 0;
 }
