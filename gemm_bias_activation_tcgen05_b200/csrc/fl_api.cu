@@ -1299,8 +1299,9 @@ static cudaError_t launch_ln_w(int z_dtype, cudaStream_t s, const LnParams& P) {
   return launch_pdl_b(k, dim3((unsigned)std::min<long long>(P.M, wave)), TPB, s, P);
 }
 
-// Rows of up to 8 KB take 128 threads (32 elements a thread); longer rows 256 (on
-// 2048 x 4096 fp32 rows, 256 threads measured 11.2 us against 13.3 us for 128).
+// Rows of up to 8 KB take 128 threads (32 elements a thread); longer rows 256, four CTAs
+// per SM (on 2048 x 4096 fp32 rows, 256 threads measured 11.2 us against 13.3 us for 128,
+// and four 256-thread CTAs per SM 11.1-11.4 against 11.4-11.8 for three).
 template <int XT>
 static cudaError_t launch_ln(int z_dtype, cudaStream_t s, const LnParams& P) {
   const long long row_bytes = P.N * (XT == DT_F32 ? 4 : 2);

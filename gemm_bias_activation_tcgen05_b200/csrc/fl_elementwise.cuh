@@ -440,7 +440,7 @@ __global__ void __launch_bounds__(TPB, TPB == 128 ? 6 : 3) fl_layernorm_kernel(c
 // doubles the shared memory of a CTA.)
 constexpr int LN_DEPTH = 1;  // rows a CTA of the vector LayerNorm keeps in flight
 template <int XT, int ZT, int TPB>
-__global__ void __launch_bounds__(TPB, TPB == 128 ? 6 : 3) fl_layernorm_vec_kernel(const LnParams P) {
+__global__ void __launch_bounds__(TPB, TPB == 128 ? 6 : 4) fl_layernorm_vec_kernel(const LnParams P) {
   using TX = typename ElemT<XT>::T;
   grid_dependency_wait();
   if (threadIdx.x == 0) grid_launch_dependents();

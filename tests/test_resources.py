@@ -6,7 +6,8 @@ CPU, before it shows up as lost occupancy on the GPU:
 - the fused kernel runs 320 threads a CTA, one CTA per SM: at most 204 registers;
 - the dominant launch (ReLU + mask, bf16 out, CTA pair) spills only around its stream-K calls;
 - the dReLU and bias-gradient kernels hold four 256-thread CTAs per SM (≤ 64 registers);
-- the whole-vector LayerNorm holds six 128-thread CTAs per SM (≤ 85 registers).
+- the whole-vector LayerNorm holds six 128-thread CTAs per SM (≤ 85 registers) or four
+  256-thread ones (≤ 64 registers).
 Skipped when the report is missing (the library was not built here).
 """
 from __future__ import annotations
@@ -79,11 +80,11 @@ def test_hbm_kernels_keep_their_ctas_of_256(prefix, ctas, no_spill):
             assert v["spill"] == 0, (name, v)
 
 
-def test_vector_layernorm_keeps_six_ctas_of_128():
+def test_vector_layernorm_keeps_its_ctas_per_sm():
     for name, v in _select(_entries(), "_ZN2fl23fl_layernorm_vec_kernel").items():
-        if "Li128EEEv" in name:  # the TPB = 128 instantiations
-            assert v["regs"] * 128 * 6 <= 65536, (name, v)
-            assert v["spill"] == 0, (name, v)
+        threads, ctas = (128, 6) if "Li128EEEv" in name else (256, 4)
+        assert v["regs"] * threads * ctas <= 65536, (name, v)
+        assert v["spill"] == 0, (name, v)
 
 
 def test_launchable_fused_kernels_do_not_spill():
